@@ -1,0 +1,170 @@
+"""fp64 CPU oracle for decode / small-Q attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import or run anything in this package;
+the product path (``decode_flashattention_b200``) never does, and this package
+never imports it.  The two share no code: the oracle decodes fp16/bf16 bit
+patterns itself and evaluates the plain definition
+
+    O = softmax(Q K^T * scale) V,   scale = 1/sqrt(headDim) by default
+
+("SmallQ FlashAttention for Ascend 910B", section "接口"; "昇腾CANN上的
+FlashAttention工程实战", section on standard attention), with grouped-query
+heads (hkv = hq // (Hq // Hkv)), a bottom-right aligned causal mask (key j is
+visible to query i iff j <= i + n - Lq) and the natural-log log-sum-exp of the
+scaled scores.  Rows with no visible key give O = 0, lse = -inf.
+
+Modules:
+  * ``attention_oracle.c`` -- the definition in C, fp64, threaded over rows.
+  * ``online``             -- the pages' tiled online-softmax algorithm with
+                              split-KV partials and a log-sum-exp combine, in
+                              numpy fp64 (small inputs only).
+
+Every function here is pinned by ``tests/test_oracle.py`` to closed forms,
+invariants, a library routine (torch fp64 ``scaled_dot_product_attention``)
+and exhaustive format checks; no function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attention_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+F16, BF16, F64 = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc into ``oracle/liboracle.so``."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-pthread", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        p = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        lib.oracle_attention.restype = ctypes.c_int
+        lib.oracle_attention.argtypes = [
+            p, p, p, p, p, p, ctypes.c_int,
+            i64, i64, i64, i64, i64, i64, i64,
+            p, ctypes.c_int, ctypes.c_double, i64, p, p, p, ctypes.c_int,
+        ]
+        lib.oracle_f16_to_f64.restype = ctypes.c_double
+        lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        _lib = lib
+    return _lib
+
+
+def f16_bits_to_f64(bits: int) -> float:
+    return _load().oracle_f16_to_f64(bits)
+
+
+def bf16_bits_to_f64(bits: int) -> float:
+    return _load().oracle_bf16_to_f64(bits)
+
+
+def _as_raw(x):
+    """Accept a numpy array (float16 / uint16-with-dtype / float64) or a CPU
+    torch tensor (float16 / bfloat16 / float64); return (array, dtype code,
+    element strides).  No value is converted: 16-bit inputs are passed as
+    their bit patterns."""
+    try:
+        import torch  # torch is only used as a container here
+    except ImportError:  # pragma: no cover
+        torch = None
+    if torch is not None and isinstance(x, torch.Tensor):
+        if x.device.type != "cpu":
+            raise ValueError("oracle inputs must live in host memory")
+        code = {torch.float16: F16, torch.bfloat16: BF16, torch.float64: F64}.get(x.dtype)
+        if code is None:
+            raise TypeError(f"unsupported dtype {x.dtype}")
+        strides = tuple(int(s) for s in x.stride())
+        # the caller keeps the tensor alive; hand out its data pointer and strides
+        return x, code, strides, x.data_ptr()
+    a = np.asarray(x)
+    if a.dtype == np.float16:
+        code = F16
+    elif a.dtype == np.float64:
+        code = F64
+    else:
+        raise TypeError(f"unsupported numpy dtype {a.dtype} (bf16 must come as a torch tensor)")
+    strides = tuple(s // a.itemsize for s in a.strides)
+    return a, code, strides, a.ctypes.data
+
+
+def attention(q, k, v, *, causal: bool = False, scale: float | None = None, seqlens=None,
+              rows=None, nthreads: int | None = None):
+    """Evaluate the definition.
+
+    q: [B, Lq, Hq, Dqk]; k: [B, Lk, Hkv, Dqk]; v: [B, Lk, Hkv, Dv] (any strides,
+    fp16 / bf16 / fp64, all the same type).  seqlens: optional int [B] with
+    0 <= seqlens[b] <= Lk (the number of keys present for batch b).  rows:
+    optional int array [n, 3] of (b, hq, i); when None every row is computed.
+
+    Returns (o, lse): with rows=None, o is [B, Lq, Hq, Dv] and lse is
+    [B, Hq, Lq]; with rows given, o is [n, Dv] and lse is [n].  Both fp64.
+    """
+    qa, qc, qs, qp = _as_raw(q)
+    ka, kc, ks, kp = _as_raw(k)
+    va, vc, vs, vp = _as_raw(v)
+    if not (qc == kc == vc):
+        raise TypeError("q, k, v must share one element type")
+    if len(q.shape) != 4 or len(k.shape) != 4 or len(v.shape) != 4:
+        raise ValueError("q, k, v must be 4-D [B, L, H, D]")
+    B, Lq, Hq, Dqk = (int(s) for s in q.shape)
+    Bk, Lk, Hkv, Dk = (int(s) for s in k.shape)
+    Bv, Lv, Hv, Dv = (int(s) for s in v.shape)
+    if (Bk, Dk) != (B, Dqk) or (Bv, Lv, Hv) != (Bk, Lk, Hkv) or Hq % Hkv:
+        raise ValueError("inconsistent q/k/v shapes")
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dqk)
+    sl = None
+    if seqlens is not None:
+        sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+        if sl.shape[0] != B:
+            raise ValueError("seqlens must have B entries")
+    if rows is None:
+        n = B * Hq * Lq
+        rr = None
+    else:
+        rr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        n = rr.shape[0]
+    o = np.empty((n, Dv), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    st = [np.asarray(s, dtype=np.int64) for s in (qs, ks, vs)]
+    lib = _load()
+    ret = lib.oracle_attention(
+        qp, st[0].ctypes.data, kp, st[1].ctypes.data, vp, st[2].ctypes.data, qc,
+        B, Lq, Hq, Lk, Hkv, Dqk, Dv,
+        sl.ctypes.data if sl is not None else None, int(bool(causal)), float(scale),
+        n, rr.ctypes.data if rr is not None else None, o.ctypes.data, lse.ctypes.data,
+        int(max(1, nthreads)),
+    )
+    del qa, ka, va
+    if ret == -1:
+        raise ValueError("oracle_attention: invalid argument")
+    if ret != 0:
+        raise MemoryError("oracle_attention: out of memory or threads")
+    if rows is None:
+        o = o.reshape(B, Hq, Lq, Dv).transpose(0, 2, 1, 3).copy()
+        lse = lse.reshape(B, Hq, Lq)
+    return o, lse
