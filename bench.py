@@ -1,0 +1,496 @@
+"""Benchmark: achieved K/V HBM bandwidth and time per call of the decode
+attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one full call of the public API (host plan, split-KV kernel and,
+when needed, the LSE combine kernel) over one batch of synthetic input
+already resident in HBM.  Inputs rotate over enough copies to exceed 4x the
+126 MB L2, so K/V bytes come from HBM.  The timed steps are replayed from
+CUDA graphs (captured calls of the same API) and timed with CUDA events on
+the launching stream; N > 1 runs independent replicas (one per GPU) and
+reports the max time over ranks.
+
+Printed (rank 0, one JSON line): value = algorithmic K/V bytes of all ranks
+per second (TB/s); ms_per_step; roofline of the split-KV kernel (its own
+CUDA-event duration, measured in a second pass with the library's event
+profiling); e2e = the same metric through the public API with pinned host
+buffers and the host<->device copies inside the timed region; cpu_baseline =
+the fp64 oracle on the host cores over a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "decode attention achieved K/V HBM TB/s (% of B200 peak) and µs/call"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: about 2 s worth)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of graph replays")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound of the oracle CPU sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_init(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier(device_ids=[device.index]) if device is not None else dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # no NVML: report clocks as unknown
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(s)}
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "decode_flashattention_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the split-KV kernel from a committed ncu
+    capture, if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("kernel_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def cpu_baseline(w, q, k, v, seqlens, seconds: float):
+    """The fp64 oracle as it stands, on this host's cores, over a bounded
+    sample of the workload's rows; throughput scaled to the same metric."""
+    import numpy as np
+
+    import oracle
+    from decode_flashattention_b200 import workloads as wl
+
+    oracle.build()
+    cores = os.cpu_count() or 1
+    rows_total = w.B * w.Hq * w.Lq
+    qc, kc, vc = q.cpu(), None, None
+    # estimate: time a handful of rows, then size the sample to the bound
+    rng = np.random.default_rng(0)
+    all_rows = [(b, h, i) for b in range(w.B) for h in range(w.Hq) for i in range(w.Lq)]
+    kc, vc = k.cpu(), v.cpu()
+    sl = None if seqlens is None else seqlens.numpy()
+    probe = min(rows_total, max(cores, 8))
+    idx = rng.choice(rows_total, probe, replace=False)
+    t0 = time.perf_counter()
+    oracle.attention(qc, kc, vc, causal=w.causal, seqlens=sl, rows=np.array([all_rows[i] for i in idx]),
+                     nthreads=cores)
+    per_row = (time.perf_counter() - t0) / probe
+    n = int(min(rows_total, max(probe, seconds / max(per_row, 1e-9) * 0.8)))
+    pick = sorted(rng.choice(rows_total, n, replace=False).tolist()) if n < rows_total else range(rows_total)
+    rows = np.array([all_rows[i] for i in pick])
+    t0 = time.perf_counter()
+    oracle.attention(qc, kc, vc, causal=w.causal, seqlens=sl, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    bytes_sample = wl.kv_bytes(w, seqlens) * (len(rows) / rows_total)
+    return {"value": bytes_sample / dt / 1e12, "unit": "TB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} of {rows_total} output rows of {w.name} (fp64 C oracle, "
+                      f"{dt:.2f} s); K/V bytes scaled by the sampled share of rows",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+
+    import decode_flashattention_b200 as fa
+    from decode_flashattention_b200 import workloads as wl
+
+    world, rank, local = dist_init(args)
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    fa.load_library()
+    name = args.workload or wl.DEFAULT_BENCH
+    w = wl.WORKLOADS[name]
+    q0, k0, v0, sl0 = wl.make_inputs(w, device, seed=w.seed + 1000 * rank)
+    per_copy = wl.kv_bytes(w, sl0) + q0.numel() * 2
+    n_copies = max(1, math.ceil(4 * L2_BYTES / max(per_copy, 1)))
+    copies = [(q0, k0, v0)]
+    for c in range(1, n_copies):
+        q, k, v, _ = wl.make_inputs(w, device, seed=w.seed + 1000 * rank + c)
+        copies.append((q, k, v))
+    sl_dev = sl0.to(device) if sl0 is not None else None
+    outs = [wl.empty_output(w, q0) for _ in range(n_copies)]
+    lses = [torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device) for _ in range(n_copies)]
+    if w.call == "kvcache":
+        ws_bytes = fa.kvcache_workspace_size(q0, k0, v0, args.num_splits)
+    else:
+        ws_bytes = fa.fwd_workspace_size(q0, k0, v0, w.causal, args.num_splits)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+    bytes_per_step = wl.kv_bytes(w, sl0)
+
+    def step(i):
+        q, k, v = copies[i % n_copies]
+        o, l = outs[i % n_copies], lses[i % n_copies]
+        if w.call == "kvcache":
+            fa.fa_decode_kvcache(q, k, v, sl_dev, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
+                                 workspace=ws)
+        else:
+            fa.fa_fwd(q, k, v, causal=w.causal, num_splits=args.num_splits, out=o, lse=l, workspace=ws)
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    fa.check_status()
+    dispatch = fa.last_dispatch()
+    launches_per_step = 1 + dispatch["combine_launched"] if dispatch["grid"] > 0 else dispatch["combine_launched"]
+
+    # steps: about 2 s of work unless given
+    if args.steps > 0:
+        K = args.steps
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(20):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        per = e0.elapsed_time(e1) / 20 / 1e3
+        K = int(min(200000, max(50, 2.0 / max(per, 1e-7))))
+        K = max_over_ranks(K, world, device) if world > 1 else K
+        K = int(K)
+
+    # --- pass A: value (graph replays of the public call) -----------------------------
+    graphs = []
+    use_graph = not args.no_graph
+    G = min(K, 2000)
+    if use_graph:
+        n0 = fa.launch_count()
+        g_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_full):
+            for i in range(G):
+                step(i)
+        captured = fa.launch_count() - n0
+        rem = K % G
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem):
+                for i in range(rem):
+                    step(i)
+        reps = K // G
+        launches = captured * reps + (launches_per_step * rem if rem else 0)
+        g_full.replay()  # warm the graph itself
+        torch.cuda.synchronize()
+    else:
+        launches = launches_per_step * K
+    barrier(world, device)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        e0.record(stream)
+        if use_graph:
+            for _ in range(K // G):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
+        else:
+            for i in range(K):
+                step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world, device)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local, world, device)
+    fa.check_status()
+
+    # --- pass B: the split-KV kernel's own duration (library event profiling, eager) ---
+    Kb = int(min(K, 2000))
+    fa.profile_enable(True)
+    for i in range(Kb):
+        step(i)
+    torch.cuda.synchronize()
+    prof = fa.profile_read()
+    fa.profile_enable(False)
+
+    # --- e2e: through the public API from pinned host buffers -------------------------
+    hq = q0.cpu().pin_memory()
+    hk = k0.cpu().pin_memory()
+    hv = v0.cpu().pin_memory()
+    hsl = sl0.pin_memory() if sl0 is not None else None
+    ho = torch.empty(outs[0].shape, dtype=w.dtype).pin_memory()
+    hl = torch.empty(lses[0].shape, dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0)
+    dsl = torch.empty_like(sl_dev) if sl_dev is not None else None
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + (hsl.numel() * 4 if hsl is not None else 0)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    E = max(1, args.e2e_steps)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if dsl is not None:
+            dsl.copy_(hsl, non_blocking=True)
+        qv = dq if w.layout == "blhd" else dq
+        if w.call == "kvcache":
+            o, l = fa.fa_decode_kvcache(dq, dk, dv, dsl, causal=w.causal, num_splits=args.num_splits,
+                                        out=outs[0], lse=lses[0], workspace=ws)
+        else:
+            o, l = fa.fa_fwd(dq, dk, dv, causal=w.causal, num_splits=args.num_splits, out=outs[0],
+                             lse=lses[0], workspace=ws)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, device)
+    fa.check_status()
+
+    total_bytes = sum_over_ranks(bytes_per_step * K, world, device)
+    value = total_bytes / (ms / 1e3) / 1e12
+    e2e_value = sum_over_ranks(bytes_per_step * E, world, device) / (e2e_ms / 1e3) / 1e12
+    peak, peak_kind = peaks()
+    main_ms = prof["main_ms"] / max(prof["main_launches"], 1)
+    achieved = bytes_per_step / (main_ms / 1e3) / 1e9 if main_ms > 0 else None
+    traffic = recorded_traffic(name)
+    clocks = sampler.summary()
+    if rank != 0:
+        return
+    res = {
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "TB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms / K,
+        "us_per_call": ms / K * 1e3,
+        "pct_of_peak": round(100 * value * 1e3 / peak / 1, 2),
+        "tokens_per_s": round(sum_over_ranks(wl.tokens_per_call(w) * K, 1, device) * world / (ms / 1e3), 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16" if w.dtype.__repr__().endswith("float16") else "bf16",
+        "data": "synthetic: Q/K/V i.i.d. N(0,1), seeded; no dataset or weights",
+        "config": {
+            "workload": name, "description": w.description, "call": w.call, "layout": w.layout,
+            "B": w.B, "Lq": w.Lq, "Hq": w.Hq, "Hkv": w.Hkv, "Lk": w.Lk, "Dqk": w.Dqk, "Dv": w.Dv,
+            "causal": w.causal, "num_splits": args.num_splits or "auto",
+            "kv_bytes_per_step": bytes_per_step,
+            "l2": f"inputs rotate over {n_copies} copies ({n_copies * per_copy / 1e6:.0f} MB > 4x L2)",
+            "launch": "cuda_graph_replay" if use_graph else "eager",
+            "parallelism": f"replicas{world}" if world > 1 else "single_gpu",
+            "dispatch": dispatch,
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "splitkv main kernel",
+            "achieved": round(achieved, 1) if achieved else None,
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4) if achieved else None,
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": bytes_per_step,
+            "main_us_avg": main_ms * 1e3,
+            "combine_us_avg": prof["combine_ms"] / max(prof["combine_launches"], 1) * 1e3,
+            "timed_launches": prof["main_launches"],
+        },
+        "e2e": {"value": round(e2e_value, 5), "unit": "TB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    res["cpu_baseline"] = cpu_baseline(w, q0, k0, v0, sl0, args.cpu_seconds) if world == 1 else None
+    print(json.dumps(res), flush=True)
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from decode_flashattention_b200 import workloads as wl
+
+    name = args.workload or wl.DEFAULT_BENCH
+    w = wl.WORKLOADS[name]
+    q, k, v, sl = wl.make_inputs(w, "cpu")
+    W = max(args.warmup, 3)
+    K = args.steps if args.steps > 0 else 3
+    per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(K + W, 1)))
+    for _ in range(min(W, 1)):
+        cpu_baseline(w, q, k, v, sl, per_step / 4)
+    vals, secs = [], 0.0
+    for _ in range(K):
+        r = cpu_baseline(w, q, k, v, sl, per_step)
+        vals.append(r["value"])
+        secs += r["seconds"]
+    value = sum(vals) / len(vals)
+    res = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s", "n_gpus": world,
+           "steps": K, "warmup": W, "ms_per_step": secs / K * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic: Q/K/V i.i.d. N(0,1), seeded; no dataset or weights",
+           "config": {"workload": name, "description": w.description},
+           "cpu_baseline": {"value": value, "unit": "TB/s", "cores": r["cores"], "kind": "oracle",
+                            "sample": r["sample"]},
+           "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    try:
+        import torch.distributed as dist
+
+        if dist.is_initialized():
+            dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+if __name__ == "__main__":
+    main()

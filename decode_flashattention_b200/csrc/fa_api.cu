@@ -1,0 +1,650 @@
+// fa_api.cu -- host side of libfa_b200.so: the C ABI declared in include/fa.h.
+//
+// Each compute call validates its arguments on the host (nothing is launched
+// for a bad call), plans the launch (variant, CTA count, work partition,
+// workspace), encodes the K/V TMA tensor maps, then enqueues the split-KV
+// kernel and, when some unit is shared between CTAs or has no visible key,
+// the LSE combine kernel with programmatic dependent launch.  The caller
+// owns every buffer; the library allocates no device memory and never
+// synchronises a stream in the compute calls (the aclnn-style two-phase
+// call of "SmallQ FlashAttention for Ascend 910B", section "aclnn API 调用":
+// ask for the workspace size, let the caller allocate it, run on a stream).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "fa.h"
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+// Device status word: bit 0 set when a kernel gave up waiting on its pipeline.
+__device__ unsigned int g_fa_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kDefaultMinShare = 2;
+
+thread_local std::string t_err;
+thread_local fa_dispatch_info t_disp = {};
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_force_variant{FA_VARIANT_AUTO};
+
+fa_status fail(fa_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    t_err = buf;
+    return s;
+}
+
+fa_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(FA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ------------------------------------------------------------ per-device state
+struct DeviceState {
+    bool ready = false;
+    int sms = 0;
+    unsigned *status = nullptr;
+};
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+struct FnState {
+    const void *fn;
+    int device;
+    int smem;
+    int occupancy;
+};
+std::vector<FnState> g_fns;
+
+fa_status device_state(DeviceState **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (major != 10 || minor != 0)
+            return fail(FA_ERR_UNSUPPORTED, "compiled for sm_100a only; device %d is sm_%d%d", dev, major, minor);
+        if ((e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute(sm count)");
+        void *ptr = nullptr;
+        if ((e = cudaGetSymbolAddress(&ptr, g_fa_status)) != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(status)");
+        d.status = static_cast<unsigned *>(ptr);
+        d.ready = true;
+    }
+    *out = &d;
+    return FA_OK;
+}
+
+// Sets the kernel's shared-memory limit once per device and returns its
+// resident CTAs per SM.
+fa_status prepare_fn(const void *fn, int threads, int smem, int *occupancy) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (const FnState &f : g_fns)
+        if (f.fn == fn && f.device == dev && f.smem >= smem) {
+            *occupancy = f.occupancy;
+            return FA_OK;
+        }
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic smem)");
+    int occ = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (occ < 1) return fail(FA_ERR_UNSUPPORTED, "kernel does not fit on an SM (%d B shared memory)", smem);
+    g_fns.push_back({fn, dev, smem, occ});
+    *occupancy = occ;
+    return FA_OK;
+}
+
+// ------------------------------------------------------------ validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_tensor(const fa_tensor *t, const char *name) {
+    if (!t) return fail(FA_ERR_INVALID_ARG, "%s: null descriptor", name);
+    if (t->dtype != FA_F16 && t->dtype != FA_BF16)
+        return fail(FA_ERR_UNSUPPORTED, "%s: element type %d is not fp16/bf16", name, t->dtype);
+    int64_t numel = 1;
+    for (int i = 0; i < 4; ++i) {
+        if (t->shape[i] < 0 || t->shape[i] > INT32_MAX)
+            return fail(FA_ERR_INVALID_ARG, "%s: shape[%d] = %lld out of range", name, i, (long long)t->shape[i]);
+        numel *= t->shape[i];
+    }
+    if (t->stride[3] != 1) return fail(FA_ERR_UNSUPPORTED, "%s: last dimension must be contiguous", name);
+    for (int i = 0; i < 3; ++i) {
+        if (t->stride[i] < 0 || (t->stride[i] % 8) != 0 || t->stride[i] >= (int64_t(1) << 38))
+            return fail(FA_ERR_UNSUPPORTED, "%s: stride[%d] = %lld must be a non-negative multiple of 8 elements",
+                        name, i, (long long)t->stride[i]);
+    }
+    if (numel > 0) {
+        if (!t->data) return fail(FA_ERR_INVALID_ARG, "%s: null data pointer", name);
+        if (!aligned16(t->data)) return fail(FA_ERR_UNSUPPORTED, "%s: data must be 16-byte aligned", name);
+    }
+    return FA_OK;
+}
+
+struct Shapes {
+    int dtype;
+    int B, Lq, Hq, Lk, Hkv, Dqk, Dv, g, R, RB, BR;
+};
+
+fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *o,
+                       Shapes *s) {
+    fa_status st;
+    if ((st = check_tensor(q, "q")) || (st = check_tensor(k, "k")) || (st = check_tensor(v, "v")))
+        return st;
+    if (o && (st = check_tensor(o, "o"))) return st;
+    if (k->dtype != q->dtype || v->dtype != q->dtype || (o && o->dtype != q->dtype))
+        return fail(FA_ERR_INVALID_ARG, "q, k, v and o must share one element type");
+    s->dtype = q->dtype;
+    s->B = (int)q->shape[0];
+    s->Lq = (int)q->shape[1];
+    s->Hq = (int)q->shape[2];
+    s->Dqk = (int)q->shape[3];
+    s->Lk = (int)k->shape[1];
+    s->Hkv = (int)k->shape[2];
+    s->Dv = (int)v->shape[3];
+    if (k->shape[0] != s->B || v->shape[0] != s->B)
+        return fail(FA_ERR_INVALID_ARG, "batch mismatch: q %d, k %lld, v %lld", s->B, (long long)k->shape[0],
+                    (long long)v->shape[0]);
+    if (k->shape[3] != s->Dqk) return fail(FA_ERR_INVALID_ARG, "k head dim %lld != q head dim %d", (long long)k->shape[3], s->Dqk);
+    if (v->shape[1] != s->Lk || v->shape[2] != s->Hkv)
+        return fail(FA_ERR_INVALID_ARG, "v must be [B, Lk, Hkv, Dv] matching k");
+    if (o && (o->shape[0] != s->B || o->shape[1] != s->Lq || o->shape[2] != s->Hq || o->shape[3] != s->Dv))
+        return fail(FA_ERR_INVALID_ARG, "o must be [B, Lq, Hq, Dv]");
+    if (s->Hkv <= 0 || s->Hq <= 0) return fail(FA_ERR_INVALID_ARG, "head counts must be positive");
+    if (s->Hq % s->Hkv) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", s->Hq, s->Hkv);
+    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128)))
+        return fail(FA_ERR_UNSUPPORTED, "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128)}", s->Dqk,
+                    s->Dv);
+    s->g = s->Hq / s->Hkv;
+    int64_t R = (int64_t)s->g * s->Lq;
+    if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * Lq too large");
+    s->R = (int)R;
+    s->RB = (s->R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
+    int64_t BR = (int64_t)s->B * s->RB;
+    if (BR > fa::kMaxPrefixEntries)
+        return fail(FA_ERR_UNSUPPORTED, "B * ceil(g * Lq / 8) = %lld exceeds %d", (long long)BR, fa::kMaxPrefixEntries);
+    s->BR = (int)BR;
+    return FA_OK;
+}
+
+// ------------------------------------------------------------ planning
+struct Plan {
+    fa::KernelInfo main, comb;
+    int occupancy;
+    int P;           // CTAs launched for the main kernel
+    int P_param;     // CTA count the schedule is computed with
+    int min_share;
+    int64_t W;       // host-known total tiles (-1 for kvcache)
+    bool need_combine;
+    size_t ws_o_floats;
+    size_t ws_bytes;
+    int comb_smem;
+    int comb_grid;
+};
+
+int choose_variant(const Shapes &s) {
+    int forced = g_force_variant.load();
+    if (forced != FA_VARIANT_AUTO) return forced;
+    fa::KernelInfo tmp;
+    if (s.R == 1 && fa::get_scalar_kernel(s.dtype, s.Dqk, s.Dv, &tmp)) return FA_VARIANT_SCALAR;
+    return FA_VARIANT_MMA;
+}
+
+// Host copy of the device schedule for dense inputs (every batch has Lk keys):
+// returns W, and whether some unit is cut between CTAs or has no tiles.
+void host_schedule(const Shapes &s, int causal, int TK, int64_t P, int64_t min_share, int64_t *W_out,
+                   int64_t *Peff_out, bool *need_combine) {
+    std::vector<int64_t> pre(s.BR + 1, 0);
+    bool empty_unit = false;
+    for (int x = 0; x < s.BR; ++x) {
+        int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, TK);
+        if (t == 0) empty_unit = true;
+        pre[x + 1] = pre[x] + (int64_t)s.Hkv * t;
+    }
+    int64_t W = pre[s.BR];
+    int64_t Peff = fa::eff_parts(W, P, min_share);
+    bool split = false;
+    for (int64_t c = 1; c < Peff && !split; ++c) {
+        int64_t pos = fa::part_start(c, W, Peff);
+        // entry containing pos
+        int lo = 0, hi = s.BR - 1;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) / 2;
+            if (pre[mid] <= pos) lo = mid; else hi = mid - 1;
+        }
+        int64_t t = (pre[lo + 1] - pre[lo]) / s.Hkv;
+        if (t > 0 && (pos - pre[lo]) % t != 0) split = true;
+    }
+    *W_out = W;
+    *Peff_out = Peff;
+    *need_combine = split || empty_unit;
+}
+
+fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl) {
+    DeviceState *dev = nullptr;
+    fa_status st = device_state(&dev);
+    if (st) return st;
+    int variant = choose_variant(s);
+    bool ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.Dqk, s.Dv, &pl->main)
+                                           : fa::get_mma_kernel(s.dtype, s.Dqk, s.Dv, &pl->main);
+    if (variant == FA_VARIANT_SCALAR && ok && s.R != 1)
+        return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
+    if (!ok) return fail(FA_ERR_UNSUPPORTED, "no kernel for variant %d, dtype %d, head dims (%d, %d)", variant,
+                         s.dtype, s.Dqk, s.Dv);
+    if (!fa::get_combine_kernel(s.dtype, s.Dv, &pl->comb))
+        return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.Dv);
+    if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
+    pl->comb_smem = (s.BR + 1) * 8;
+    int comb_occ = 0;
+    if ((st = prepare_fn(pl->comb.fn, pl->comb.threads, pl->comb_smem, &comb_occ))) return st;
+
+    const int TK = pl->main.tile_keys;
+    const int64_t units = (int64_t)s.B * s.RB * s.Hkv;
+    int64_t P;
+    if (num_splits > 0) {
+        P = units * num_splits;
+        pl->min_share = 1;
+    } else {
+        P = (int64_t)dev->sms * pl->occupancy;
+        pl->min_share = kDefaultMinShare;
+    }
+    if (P > (1 << 20)) P = 1 << 20;
+    if (P < 1) P = 1;
+    pl->P_param = (int)P;
+    if (!kvcache) {
+        int64_t W, Peff;
+        bool need;
+        host_schedule(s, causal, TK, P, pl->min_share, &W, &Peff, &need);
+        pl->W = W;
+        pl->P = (int)Peff;
+        pl->P_param = (int)Peff;  // same partition, no idle CTAs
+        pl->need_combine = need;
+        if (W == 0) pl->P = 0;    // nothing to stream: the combine writes every row
+    } else {
+        pl->W = -1;
+        pl->P = max_keys > 0 ? (int)P : 0;  // an empty cache: the combine writes every row
+        pl->need_combine = true;
+    }
+    const bool any_partial = kvcache || pl->need_combine;
+    pl->ws_o_floats = any_partial ? (size_t)pl->P_param * 2 * fa::kRowsPerCta * s.Dv : 0;
+    size_t lse_floats = any_partial ? (size_t)pl->P_param * 2 * fa::kRowsPerCta : 0;
+    size_t o_bytes = (pl->ws_o_floats * 4 + 255) & ~size_t(255);
+    pl->ws_bytes = any_partial ? o_bytes + ((lse_floats * 4 + 255) & ~size_t(255)) : 0;
+    int64_t rows = (int64_t)s.B * s.Hq * s.Lq;
+    pl->comb_grid = (int)((rows + 3) / 4);
+    return FA_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// [B, L, H, D] tensor as a 4-D TMA map {D, L, H, B}; box = 64 elements x TK
+// rows of one head of one batch, 128-byte swizzle, zero fill out of bounds.
+fa_status encode_kv_map(const fa_tensor *t, int TK, CUtensorMap *map, const char *name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int64_t elt = 2;
+    cuuint64_t dims[4] = {(cuuint64_t)t->shape[3], (cuuint64_t)t->shape[1], (cuuint64_t)t->shape[2],
+                          (cuuint64_t)t->shape[0]};
+    int64_t st[3] = {t->stride[1], t->stride[2], t->stride[0]};
+    // A dimension of extent 1 is never stepped; give it a harmless legal stride.
+    int64_t packed = t->shape[3];
+    for (int i = 0; i < 3; ++i) {
+        if (dims[i + 1] == 1 || st[i] == 0) st[i] = packed;
+        packed = st[i] * (int64_t)dims[i + 1];
+        if (st[i] % 8) st[i] = (st[i] + 7) / 8 * 8;
+    }
+    cuuint64_t strides[3] = {(cuuint64_t)(st[0] * elt), (cuuint64_t)(st[1] * elt), (cuuint64_t)(st[2] * elt)};
+    cuuint32_t box[4] = {64, (cuuint32_t)TK, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMapDataType dt = t->dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_UNSUPPORTED, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
+    return FA_OK;
+}
+
+// ------------------------------------------------------------ profiling
+struct ProfRec {
+    cudaEvent_t e0, e1, e2;
+    bool has_comb;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+size_t g_prof_used = 0;
+
+fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
+    cudaError_t e = cudaEventRecord(*ev, stream);
+    return e == cudaSuccess ? FA_OK : cuda_fail(e, "cudaEventRecord");
+}
+
+// ------------------------------------------------------------ the call
+fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
+              const int32_t *seqlens, float *lse, int causal, float scale, int num_splits, void *workspace,
+              size_t workspace_bytes, cudaStream_t stream) {
+    if (s.B == 0 || s.Lq == 0) {
+        t_disp = {};
+        return FA_OK;
+    }
+    Plan pl;
+    fa_status st = make_plan(s, causal, num_splits, seqlens != nullptr, s.Lk, &pl);
+    if (st) return st;
+    if (workspace_bytes < pl.ws_bytes)
+        return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
+                    pl.ws_bytes);
+    if (pl.ws_bytes && !workspace) return fail(FA_ERR_WORKSPACE, "workspace pointer is null");
+    if (pl.ws_bytes && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(FA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(FA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+
+    DeviceState *dev = nullptr;
+    if ((st = device_state(&dev))) return st;
+
+    fa::Params p = {};
+    p.q = q->data;
+    p.q_sb = q->stride[0];
+    p.q_sl = q->stride[1];
+    p.q_sh = q->stride[2];
+    p.o = o->data;
+    p.o_sb = o->stride[0];
+    p.o_sl = o->stride[1];
+    p.o_sh = o->stride[2];
+    p.lse = lse;
+    p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
+    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                       ((pl.ws_o_floats * 4 + 255) & ~size_t(255)))
+                           : nullptr;
+    p.seqlens = seqlens;
+    p.status = dev->status;
+    p.B = s.B;
+    p.Lq = s.Lq;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.g = s.g;
+    p.R = s.R;
+    p.RB = s.RB;
+    p.Lk = s.Lk;
+    p.causal = causal ? 1 : 0;
+    float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)s.Dqk);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.P = pl.P_param;
+    p.min_share = pl.min_share;
+    p.tile_keys = pl.main.tile_keys;
+
+    bool prof = false;
+    ProfRec *rec = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_prof_mu);
+        if (g_prof_on) {
+            if (g_prof_used == g_prof.size() && g_prof.size() < 65536) {
+                ProfRec r = {};
+                if (cudaEventCreate(&r.e0) == cudaSuccess && cudaEventCreate(&r.e1) == cudaSuccess &&
+                    cudaEventCreate(&r.e2) == cudaSuccess)
+                    g_prof.push_back(r);
+            }
+            if (g_prof_used < g_prof.size()) {
+                rec = &g_prof[g_prof_used++];
+                prof = true;
+            }
+        }
+    }
+
+    const bool launch_main = pl.P > 0;
+    if (launch_main) {
+        CUtensorMap tmK, tmV;
+        if ((st = encode_kv_map(k, pl.main.tile_keys, &tmK, "k"))) return st;
+        if ((st = encode_kv_map(v, pl.main.tile_keys, &tmV, "v"))) return st;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)pl.P);
+        cfg.blockDim = dim3((unsigned)pl.main.threads);
+        cfg.dynamicSmemBytes = (size_t)pl.main.smem;
+        cfg.stream = stream;
+        void *args[] = {&tmK, &tmV, &p};
+        if (prof && (st = prof_record(&rec->e0, stream))) return st;
+        cudaError_t e = cudaLaunchKernelExC(&cfg, pl.main.fn, args);
+        if (e != cudaSuccess) return cuda_fail(e, "launch of the split-KV kernel");
+        g_launches.fetch_add(1);
+        if (prof && (st = prof_record(&rec->e1, stream))) return st;
+    } else if (prof) {
+        if ((st = prof_record(&rec->e0, stream)) || (st = prof_record(&rec->e1, stream))) return st;
+    }
+    if (pl.need_combine) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)pl.comb_grid);
+        cfg.blockDim = dim3((unsigned)pl.comb.threads);
+        cfg.dynamicSmemBytes = (size_t)pl.comb_smem;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        if (launch_main && !prof) {  // an event between the kernels would break the overlap anyway
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+        }
+        if (!launch_main) p.P = 1;
+        void *args[] = {&p};
+        cudaError_t e = cudaLaunchKernelExC(&cfg, pl.comb.fn, args);
+        if (e != cudaSuccess) return cuda_fail(e, "launch of the combine kernel");
+        g_launches.fetch_add(1);
+    }
+    if (prof) {
+        rec->has_comb = pl.need_combine;
+        if ((st = prof_record(&rec->e2, stream))) return st;
+    }
+
+    fa_dispatch_info d = {};
+    d.variant = pl.main.variant;
+    d.grid = pl.P;
+    d.block = pl.main.threads;
+    d.smem_bytes = pl.main.smem;
+    d.tile_keys = pl.main.tile_keys;
+    d.stages = pl.main.stages;
+    d.rows_per_cta = fa::kRowsPerCta;
+    d.units = (int)((int64_t)s.B * s.RB * s.Hkv);
+    d.min_share_tiles = pl.min_share;
+    d.combine_launched = pl.need_combine ? 1 : 0;
+    d.work_tiles = pl.W;
+    t_disp = d;
+    t_err.clear();
+    return FA_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+fa_status fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o, float *lse, int causal,
+                 float scale, int num_splits, void *workspace, size_t workspace_bytes, void *stream) {
+    Shapes s;
+    fa_status st = check_shapes(q, k, v, o, &s);
+    if (st) return st;
+    if (!o) return fail(FA_ERR_INVALID_ARG, "o: null descriptor");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+    return run(s, q, k, v, o, nullptr, lse, causal, scale, num_splits, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int causal,
+                                int num_splits, size_t *bytes) {
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes: null pointer");
+    Shapes s;
+    fa_status st = check_shapes(q, k, v, nullptr, &s);
+    if (st) return st;
+    if (s.B == 0 || s.Lq == 0) {
+        *bytes = 0;
+        return FA_OK;
+    }
+    Plan pl;
+    if ((st = make_plan(s, causal, num_splits, false, s.Lk, &pl))) return st;
+    *bytes = pl.ws_bytes;
+    return FA_OK;
+}
+
+fa_status fa_decode_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                            const int32_t *cache_seqlens, fa_tensor *o, float *lse, int num_splits, int causal,
+                            float scale, void *workspace, size_t workspace_bytes, void *stream) {
+    Shapes s;
+    fa_status st = check_shapes(q, k_cache, v_cache, o, &s);
+    if (st) return st;
+    if (!o) return fail(FA_ERR_INVALID_ARG, "o: null descriptor");
+    if (!cache_seqlens && s.B > 0) return fail(FA_ERR_INVALID_ARG, "cache_seqlens: null pointer");
+    if (cache_seqlens && (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+        return fail(FA_ERR_INVALID_ARG, "cache_seqlens must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+    return run(s, q, k_cache, v_cache, o, cache_seqlens, lse, causal, scale, num_splits, workspace,
+               workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                                           int num_splits, size_t *bytes) {
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes: null pointer");
+    Shapes s;
+    fa_status st = check_shapes(q, k_cache, v_cache, nullptr, &s);
+    if (st) return st;
+    if (s.B == 0 || s.Lq == 0) {
+        *bytes = 0;
+        return FA_OK;
+    }
+    Plan pl;
+    if ((st = make_plan(s, 0, num_splits, true, s.Lk, &pl))) return st;
+    *bytes = pl.ws_bytes;
+    return FA_OK;
+}
+
+fa_status fa_check_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    DeviceState *dev = nullptr;
+    fa_status st = device_state(&dev);
+    if (st) return st;
+    unsigned v = 0;
+    e = cudaMemcpy(&v, dev->status, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+    if (v) {
+        unsigned zero = 0;
+        cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        return fail(FA_ERR_TIMEOUT, "a kernel gave up waiting on its copy pipeline (status 0x%x)", v);
+    }
+    t_err.clear();
+    return FA_OK;
+}
+
+const char *fa_last_error(void) { return t_err.c_str(); }
+
+void fa_last_dispatch(fa_dispatch_info *info) {
+    if (info) *info = t_disp;
+}
+
+fa_status fa_force_variant(int variant) {
+    if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_SCALAR)
+        return fail(FA_ERR_INVALID_ARG, "unknown variant %d", variant);
+    g_force_variant.store(variant);
+    return FA_OK;
+}
+
+fa_status fa_profile_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = on != 0;
+    g_prof_used = 0;
+    return FA_OK;
+}
+
+fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double *combine_ms, int64_t *combine_launches) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    double mm = 0, cm = 0;
+    int64_t mn = 0, cn = 0;
+    for (size_t i = 0; i < g_prof_used; ++i) {
+        float a = 0, b = 0;
+        cudaError_t e = cudaEventElapsedTime(&a, g_prof[i].e0, g_prof[i].e1);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+        mm += a;
+        ++mn;
+        if (g_prof[i].has_comb) {
+            e = cudaEventElapsedTime(&b, g_prof[i].e1, g_prof[i].e2);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+            cm += b;
+            ++cn;
+        }
+    }
+    if (main_ms) *main_ms = mm;
+    if (main_launches) *main_launches = mn;
+    if (combine_ms) *combine_ms = cm;
+    if (combine_launches) *combine_launches = cn;
+    return FA_OK;
+}
+
+fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens, int num_ctas,
+                      int min_share, int tile_keys, int64_t *work_tiles, int64_t *ctas_used, int32_t *unit_tiles,
+                      int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units) {
+    if (B < 0 || Lq < 0 || Hq <= 0 || Hkv <= 0 || Lk < 0 || Hq % Hkv || num_ctas < 1 || min_share < 1 ||
+        tile_keys < 1 || max_units < 0)
+        return fail(FA_ERR_INVALID_ARG, "fa_schedule: inconsistent sizes");
+    const int g = Hq / Hkv, R = g * Lq, RB = (R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
+    const int64_t BR = (int64_t)B * RB;
+    std::vector<int64_t> pre(BR + 1, 0);
+    std::vector<int32_t> tx(BR, 0);
+    for (int64_t x = 0; x < BR; ++x) {
+        int n = fa::batch_keys(seqlens, (int)(x / RB), Lk);
+        tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, tile_keys);
+        pre[x + 1] = pre[x] + (int64_t)Hkv * tx[x];
+    }
+    const int64_t W = pre[BR];
+    const int64_t P = fa::eff_parts(W, num_ctas, min_share);
+    if (work_tiles) *work_tiles = W;
+    if (ctas_used) *ctas_used = P;
+    int64_t u = 0;
+    for (int64_t x = 0; x < BR && u < max_units; ++x)
+        for (int h = 0; h < Hkv && u < max_units; ++h, ++u) {
+            const int64_t u0 = pre[x] + (int64_t)h * tx[x];
+            if (unit_tiles) unit_tiles[u] = tx[x];
+            const bool has = tx[x] > 0;
+            if (unit_first_cta) unit_first_cta[u] = has ? fa::part_of(u0, W, P) : -1;
+            if (unit_last_cta) unit_last_cta[u] = has ? fa::part_of(u0 + tx[x] - 1, W, P) : -1;
+        }
+    t_err.clear();
+    return FA_OK;
+}
+
+int64_t fa_launch_count(void) { return g_launches.load(); }
+
+const char *fa_version(void) { return "fa_b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,195 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) decode / small-Q attention library
+ * (libfa_b200.so).
+ *
+ * Operation (every entry point that computes):
+ *
+ *   O = softmax(Q K^T * scale) V
+ *
+ *   "SmallQ FlashAttention for Ascend 910B", section "接口" (interface):
+ *   O = softmax(Q·Kᵀ/√headDim)·V on fp16 inputs with fp32 accumulation;
+ *   the MXFlashAttn README (section "前向算子 API") gives the FlashAttention
+ *   style forward calls flash_attn_func / flash_attn_with_kvcache with
+ *   causal=True, GQA ratios 2/4/8 and head_dim 64/128 in fp16 and bf16;
+ *   the same README's M1 kernel is a split-KV decode kernel.
+ *
+ * Conventions shared by all calls
+ *   - Tensors are described by fa_tensor: a DEVICE pointer, an element type,
+ *     a 4-D shape in [B, L, H, D] order and element strides.  The last
+ *     dimension (D) must be contiguous (stride 1); the other strides are free,
+ *     so a [H, L, D] buffer is passed as shape [1, L, H, D] with strides
+ *     {H*L*D, D, L*D, 1}.  Base pointers must be 16-byte aligned and every
+ *     stride a multiple of 8 elements (16 bytes).
+ *   - q is [B, Lq, Hq, Dqk]; k is [B, Lk, Hkv, Dqk]; v is [B, Lk, Hkv, Dv];
+ *     o is [B, Lq, Hq, Dv] of the same element type; Hq = g * Hkv (GQA:
+ *     query head hq reads kv head hq / g).  Supported (Dqk, Dv): (64, 64),
+ *     (128, 128), (192, 128).  q, k, v and o share one type: FA_F16 or FA_BF16.
+ *   - lse, when not NULL, is a DEVICE fp32 array [B, Hq, Lq] (contiguous)
+ *     receiving the natural-log log-sum-exp of each row's scaled scores.
+ *   - causal != 0 applies a causal mask aligned to the bottom-right corner:
+ *     key j is visible to query i iff j <= i + n - Lq, n being the number of
+ *     keys of that batch.  A row with no visible key gets O = 0, lse = -inf.
+ *   - scale <= 0 selects 1/sqrt(Dqk).
+ *   - num_splits <= 0 lets the library choose how the key range is split
+ *     across CTAs; num_splits > 0 asks for about that many splits per
+ *     (batch, kv-head, row block) unit (the result does not depend on it
+ *     beyond fp32 rounding).
+ *   - workspace: caller-owned DEVICE scratch of at least the size the
+ *     matching *_workspace_size call returns (it may be NULL when that size
+ *     is 0).  The library never allocates device memory and never
+ *     synchronises the stream in the compute calls.
+ *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     All work is enqueued asynchronously on it; the caller keeps the
+ *     buffers alive until it completes.
+ *   - Errors: argument problems are detected on the host, before any launch,
+ *     and returned as FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED /
+ *     FA_ERR_WORKSPACE with a message in fa_last_error(); a failed launch
+ *     returns FA_ERR_CUDA.  No call silently falls back to a slower path.
+ *
+ * Thread safety: the compute calls may be issued from several host threads;
+ * fa_last_error() and fa_last_dispatch() report the calling thread's last call.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* malformed shapes, strides, pointers or types */
+    FA_ERR_UNSUPPORTED = 2, /* well-formed but outside the supported set */
+    FA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+    FA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed */
+    FA_ERR_TIMEOUT = 5      /* a kernel gave up waiting on its copy pipeline */
+} fa_status;
+
+typedef enum fa_dtype { FA_F16 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* A strided 4-D device tensor in [B, L, H, D] order (element strides). */
+typedef struct fa_tensor {
+    void *data;
+    int32_t dtype; /* fa_dtype */
+    int32_t reserved;
+    int64_t shape[4];
+    int64_t stride[4];
+} fa_tensor;
+
+/* Which kernels the calling thread's last compute call launched. */
+typedef enum fa_variant { FA_VARIANT_AUTO = 0, FA_VARIANT_MMA = 1, FA_VARIANT_SCALAR = 2 } fa_variant;
+
+typedef struct fa_dispatch_info {
+    int32_t variant;          /* fa_variant of the main kernel */
+    int32_t grid;             /* CTAs launched for the main kernel */
+    int32_t block;            /* threads per CTA of the main kernel */
+    int32_t smem_bytes;       /* dynamic shared memory per CTA */
+    int32_t tile_keys;        /* keys per pipeline stage */
+    int32_t stages;           /* pipeline depth */
+    int32_t rows_per_cta;     /* packed query rows per CTA (g * Lq packing) */
+    int32_t units;            /* (batch, kv-head, row-block) work units */
+    int32_t min_share_tiles;  /* least tiles a CTA is given */
+    int32_t combine_launched; /* 1 if the LSE combine kernel was launched */
+    int64_t work_tiles;       /* total key tiles (known on the host for fa_fwd; -1 for kvcache) */
+} fa_dispatch_info;
+
+/*
+ * fa_fwd -- forward attention over dense Q/K/V (flash_attn_func).
+ * q, k, v, o as in the conventions above (Lk taken from k->shape[1]).
+ */
+FA_API fa_status fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
+                 float *lse, int causal, float scale, int num_splits, void *workspace,
+                 size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace fa_fwd needs for these shapes on the current device. */
+FA_API fa_status fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
+                                int causal, int num_splits, size_t *bytes);
+
+/*
+ * fa_decode_kvcache -- attention of new queries against a dense KV cache
+ * (flash_attn_with_kvcache).  k_cache/v_cache are [B, Lmax, Hkv, D]; batch b
+ * attends to its first cache_seqlens[b] keys (0 <= cache_seqlens[b] <= Lmax,
+ * a DEVICE int32 array [B]; slots at and beyond cache_seqlens[b] are never
+ * used and may hold anything, NaN included).  causal/scale as above with
+ * n = cache_seqlens[b].
+ */
+FA_API fa_status fa_decode_kvcache(const fa_tensor *q, const fa_tensor *k_cache, const fa_tensor *v_cache,
+                            const int32_t *cache_seqlens, fa_tensor *o, float *lse, int num_splits,
+                            int causal, float scale, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+/* Bytes of workspace fa_decode_kvcache needs for these shapes on the current device. */
+FA_API fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache,
+                                           const fa_tensor *v_cache, int num_splits,
+                                           size_t *bytes);
+
+/*
+ * Synchronises `stream`, then reports whether any kernel of this library on
+ * the current device gave up waiting on its copy pipeline since the last
+ * check (FA_ERR_TIMEOUT) and clears that record.  FA_ERR_CUDA if the stream
+ * itself reports an error.
+ */
+FA_API fa_status fa_check_status(void *stream);
+
+/* Message of the calling thread's last failed call ("" after success). */
+FA_API const char *fa_last_error(void);
+
+/* What the calling thread's last successful compute call launched. */
+FA_API void fa_last_dispatch(fa_dispatch_info *info);
+
+/*
+ * Tuning / test hook: force the main-kernel variant for later calls of this
+ * process (FA_VARIANT_AUTO restores the library's choice).  A forced variant
+ * that does not support the call's shapes makes the call fail with
+ * FA_ERR_UNSUPPORTED.
+ */
+FA_API fa_status fa_force_variant(int variant);
+
+/*
+ * Profiling: while enabled, each compute call brackets its main kernel and
+ * its combine kernel with CUDA events on the call's stream.  Enabling
+ * clears earlier records.  fa_profile_read synchronises nothing: call it after
+ * the stream has completed; it returns the summed milliseconds and the
+ * number of timed launches of each kernel.
+ */
+FA_API fa_status fa_profile_enable(int on);
+FA_API fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double *combine_ms,
+                          int64_t *combine_launches);
+
+/*
+ * fa_schedule -- host-side copy of the work partition the kernels compute on
+ * the device (no device access; for inspection and tests).  Work is counted
+ * in key tiles of `tile_keys` keys; a unit is (batch, block of 8 packed query
+ * rows, kv head), ordered batch-major, then row block, then kv head, and owns
+ * ceil(visible keys / tile_keys) tiles.  The W tiles of all units are laid end
+ * to end and cut into ctas_used = min(num_ctas, ceil(W / min_share)) equal
+ * contiguous ranges, one per CTA.  seqlens: HOST int32 [B] (NULL: every batch
+ * has Lk keys).  For each of the first max_units units the call writes its
+ * tile count and the first and last CTA whose range touches it (-1, -1 for a
+ * unit with no tiles).  FA_ERR_INVALID_ARG for inconsistent sizes.
+ */
+FA_API fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens,
+                      int num_ctas, int min_share, int tile_keys, int64_t *work_tiles,
+                      int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta,
+                      int64_t *unit_last_cta, int64_t max_units);
+
+/* Kernels launched by this library in this process (both kinds). */
+FA_API int64_t fa_launch_count(void);
+
+/* Library version string. */
+FA_API const char *fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

@@ -1,0 +1,211 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol include/fa.h declares, rejects malformed calls on the host before
+touching a device, and its host-side work partition has the properties the
+kernels rely on."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import decode_flashattention_b200 as fa
+from decode_flashattention_b200 import FaTensor
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, TIMEOUT = range(6)
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = fa.load_library()
+    names = header_functions()
+    assert "fa_fwd" in names and "fa_decode_kvcache" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_string():
+    assert b"sm_100a" in fa.load_library().fa_version()
+
+
+def desc(shape, dtype=0, stride=None, ptr=0x10000):
+    d = FaTensor()
+    d.data = ptr
+    d.dtype = dtype
+    if stride is None:
+        stride = [int(np.prod(shape[i + 1:])) for i in range(4)]
+    for i in range(4):
+        d.shape[i] = shape[i]
+        d.stride[i] = stride[i]
+    return d
+
+
+def call_fwd(q, k, v, o, causal=0, scale=0.0, lse=None):
+    lib = fa.load_library()
+    return lib.fa_fwd(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), ctypes.byref(o) if o else None,
+                      lse, causal, scale, 0, None, 0, None)
+
+
+GOOD = dict(q=[1, 1, 8, 128], k=[1, 64, 2, 128], v=[1, 64, 2, 128], o=[1, 1, 8, 128])
+
+
+def good(name, **kw):
+    return desc(GOOD[name], **kw)
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("dtype_mismatch", INVALID), ("bad_gqa", INVALID), ("head_dim_96", UNSUPPORTED),
+    ("last_dim_strided", UNSUPPORTED), ("stride_not_16B", UNSUPPORTED), ("misaligned", UNSUPPORTED),
+    ("null_o", INVALID), ("batch_mismatch", INVALID), ("nan_scale", INVALID), ("fp32", UNSUPPORTED),
+    ("too_many_row_blocks", UNSUPPORTED), ("null_data", INVALID), ("o_shape", INVALID),
+])
+def test_host_validation(case, expect):
+    q, k, v, o = good("q"), good("k"), good("v"), good("o")
+    scale = 0.0
+    if case == "dtype_mismatch":
+        v = good("v", dtype=1)
+    elif case == "bad_gqa":
+        q = desc([1, 1, 3, 128]); o = desc([1, 1, 3, 128])
+    elif case == "head_dim_96":
+        q, k, v, o = desc([1, 1, 8, 96]), desc([1, 64, 2, 96]), desc([1, 64, 2, 96]), desc([1, 1, 8, 96])
+    elif case == "last_dim_strided":
+        k = desc([1, 64, 2, 128], stride=[64 * 2 * 256, 2 * 256, 256, 2])
+    elif case == "stride_not_16B":
+        k = desc([1, 64, 2, 128], stride=[64 * 2 * 132, 2 * 132, 132, 1])
+    elif case == "misaligned":
+        k = good("k", ptr=0x10008)
+    elif case == "null_o":
+        o = None
+    elif case == "batch_mismatch":
+        k = desc([2, 64, 2, 128])
+    elif case == "nan_scale":
+        scale = float("nan")
+    elif case == "fp32":
+        q, k, v, o = good("q", dtype=2), good("k", dtype=2), good("v", dtype=2), good("o", dtype=2)
+    elif case == "too_many_row_blocks":
+        q, o = desc([9000, 1, 8, 128]), desc([9000, 1, 8, 128])
+        k, v = desc([9000, 64, 2, 128]), desc([9000, 64, 2, 128])
+    elif case == "null_data":
+        q = good("q", ptr=0)
+    elif case == "o_shape":
+        o = desc([1, 2, 8, 128])
+    assert call_fwd(q, k, v, o, scale=scale) == expect
+    assert fa.load_library().fa_last_error()  # a message is set
+
+
+def test_kvcache_null_seqlens():
+    lib = fa.load_library()
+    q, k, v, o = good("q"), good("k"), good("v"), good("o")
+    st = lib.fa_decode_kvcache(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), None, ctypes.byref(o),
+                               None, 0, 0, 0.0, None, 0, None)
+    assert st == INVALID
+
+
+def test_workspace_query_needs_output_pointer():
+    lib = fa.load_library()
+    q, k, v = good("q"), good("k"), good("v")
+    assert lib.fa_fwd_workspace_size(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), 0, 0, None) == INVALID
+
+
+def test_force_variant_rejects_unknown():
+    assert fa.load_library().fa_force_variant(7) == INVALID
+    assert fa.load_library().fa_force_variant(0) == OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_cuda_error():
+    q, k, v, o = good("q"), good("k"), good("v"), good("o")
+    assert call_fwd(q, k, v, o) == CUDA
+
+
+def test_empty_batch_is_a_no_op():
+    q, k, v, o = desc([0, 1, 8, 128]), desc([0, 64, 2, 128]), desc([0, 64, 2, 128]), desc([0, 1, 8, 128])
+    assert call_fwd(q, k, v, o) == OK
+
+
+# ------------------------------------------------------------------ work partition
+
+def visible_tiles(n, rb, R, Lq, causal, TK=64):
+    """Independent restatement of the tiles a row block needs (bottom-right)."""
+    if n <= 0:
+        return 0
+    rows = range(rb * 8, min(rb * 8 + 8, R))
+    k = max(min(n, (r % Lq) + n - Lq + 1) if causal else n for r in rows)
+    return max(0, math.ceil(max(k, 0) / TK))
+
+
+CASES = [
+    dict(B=1, Lq=1, Hq=32, Hkv=32, Lk=4096, causal=False, seqlens=None, num_ctas=296),
+    dict(B=1, Lq=4, Hq=64, Hkv=64, Lk=3000, causal=True, seqlens=None, num_ctas=296),
+    dict(B=1, Lq=32, Hq=8, Hkv=2, Lk=128, causal=True, seqlens=None, num_ctas=296),
+    dict(B=8, Lq=8, Hq=128, Hkv=128, Lk=16384, causal=True, seqlens=None, num_ctas=296),
+    dict(B=64, Lq=1, Hq=32, Hkv=8, Lk=16384, causal=False, seqlens="rand", num_ctas=296),
+    dict(B=5, Lq=3, Hq=6, Hkv=2, Lk=100, causal=True, seqlens=[0, 1, 100, 2, 50], num_ctas=7),
+    dict(B=3, Lq=1, Hq=2, Hkv=2, Lk=10, causal=False, seqlens=[0, 0, 0], num_ctas=9),
+]
+
+
+@pytest.mark.parametrize("c", CASES, ids=range(len(CASES)))
+@pytest.mark.parametrize("min_share", [1, 2, 5])
+def test_schedule_covers_balances_and_bounds_partials(c, min_share):
+    c = dict(c)
+    if c["seqlens"] == "rand":
+        c["seqlens"] = np.random.default_rng(3).integers(1, c["Lk"] + 1, c["B"]).astype(np.int32)
+    s = fa.schedule(c["B"], c["Lq"], c["Hq"], c["Hkv"], c["Lk"], c["causal"], c["seqlens"],
+                    num_ctas=c["num_ctas"], min_share=min_share)
+    g = c["Hq"] // c["Hkv"]
+    R = g * c["Lq"]
+    RB = (R + 7) // 8
+    want = []
+    for b in range(c["B"]):
+        n = c["Lk"] if c["seqlens"] is None else int(c["seqlens"][b])
+        for rb in range(RB):
+            want += [visible_tiles(n, rb, R, c["Lq"], c["causal"])] * c["Hkv"]
+    tiles = s["unit_tiles"]
+    assert tiles.tolist() == want
+    W = int(tiles.sum())
+    assert s["work_tiles"] == W
+    P = s["ctas_used"]
+    assert P == max(1, min(c["num_ctas"], math.ceil(W / min_share)))
+    if W == 0:
+        assert np.all(s["unit_first_cta"] == -1)
+        return
+    # every CTA gets floor or ceil of W / P tiles
+    shares = [((cta + 1) * W) // P - (cta * W) // P for cta in range(P)]
+    assert max(shares) - min(shares) <= 1 and min(shares) >= 1
+    # units map to non-decreasing, contiguous CTA ranges
+    has = tiles > 0
+    first, last = s["unit_first_cta"][has], s["unit_last_cta"][has]
+    assert np.all(first <= last) and np.all(np.diff(first) >= 0) and np.all(np.diff(last) >= 0)
+    assert first[0] == 0 and last[-1] == P - 1
+    # a CTA holds at most two partial units (its first and its last segment)
+    partial_count = np.zeros(P, dtype=int)
+    for f, l in zip(first, last):
+        if f != l:
+            partial_count[f:l + 1] += 1
+    assert partial_count.max(initial=0) <= 2
+    # tiles per CTA add up: each unit's tiles land in [first, last]
+    covered = np.zeros(P, dtype=np.int64)
+    pos = 0
+    for t in tiles[has]:
+        for x in range(pos, pos + int(t)):
+            covered[(x * P) // W if False else np.searchsorted([(cc * W) // P for cc in range(P)], x, side="right") - 1] += 1
+        pos += int(t)
+    assert covered.tolist() == shares
+
+
+def test_hld_view_strides():
+    x = torch.zeros(32, 4096, 128)
+    v = fa.hld_as_blhd(x)
+    assert tuple(v.shape) == (1, 4096, 32, 128)
+    assert v.stride() == (32 * 4096 * 128, 128, 4096 * 128, 1)
