@@ -488,6 +488,8 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
 
 }  // namespace
 
+void fa::set_last_error(const char *msg) { t_err = msg ? msg : ""; }
+
 // ====================================================================== C ABI
 extern "C" {
 

@@ -22,4 +22,8 @@ bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 
+// Sets the calling thread's fa_last_error() message (for entry points that
+// live outside fa_api.cu).
+void set_last_error(const char *msg);
+
 }  // namespace fa

@@ -133,6 +133,32 @@ FA_API fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_t
                                            size_t *bytes);
 
 /*
+ * fa_decode_kvcache_noalloc -- fa_decode_kvcache for callers that cannot
+ * allocate device memory (for example a plugin inside a serving runtime that
+ * owns all device memory and forbids allocation after start-up, or a decode
+ * loop that cannot afford the implicit synchronisation cudaMalloc may cause).
+ * The pages have no counterpart to this call; it exists for such callers.
+ * Same arguments and results as fa_decode_kvcache minus the workspace: the
+ * split-KV scratch is a fixed array of fa_noalloc_scratch_bytes() bytes
+ * (8 MiB) compiled into the library, held on every GPU that loads it until
+ * the process exits.  Shapes (or num_splits) needing more scratch than that
+ * are rejected with FA_ERR_UNSUPPORTED and a message; nothing is allocated,
+ * ever.  The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current: make that first call
+ * before any stream capture.  All calls on a device share the array and it
+ * keeps the last call's contents (nothing in it needs to start at zero), so
+ * calls whose GPU work overlaps -- on different streams or from racing host
+ * threads -- race on it and must be serialised by the caller.
+ */
+FA_API fa_status fa_decode_kvcache_noalloc(const fa_tensor *q, const fa_tensor *k_cache,
+                                           const fa_tensor *v_cache, const int32_t *cache_seqlens,
+                                           fa_tensor *o, float *lse, int num_splits, int causal,
+                                           float scale, void *stream);
+
+/* Size in bytes of the fixed scratch array fa_decode_kvcache_noalloc uses. */
+FA_API size_t fa_noalloc_scratch_bytes(void);
+
+/*
  * Synchronises `stream`, then reports whether any kernel of this library on
  * the current device gave up waiting on its copy pipeline since the last
  * check (FA_ERR_TIMEOUT) and clears that record.  FA_ERR_CUDA if the stream
