@@ -268,7 +268,7 @@ def profile_read() -> dict:
             "combine_launches": cn.value}
 
 
-def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=296, min_share=2, tile_keys=64):
+def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2, tile_keys=128):
     """Host copy of the kernels' work partition (see fa_schedule in include/fa.h).
     Returns dict(work_tiles, ctas_used, unit_tiles, unit_first_cta, unit_last_cta)."""
     import numpy as np

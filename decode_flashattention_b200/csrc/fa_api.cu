@@ -195,11 +195,13 @@ struct Plan {
     fa::KernelInfo main, comb;
     int occupancy;
     int P;           // CTAs launched for the main kernel
-    int P_param;     // CTA count the schedule is computed with
+    int P_param;     // CTA count the partition is computed from
     int min_share;
     int64_t W;       // host-known total tiles (-1 for kvcache)
     bool need_combine;
-    size_t ws_o_floats;
+    bool need_workspace;
+    size_t pieces;   // partial-result slots reserved (pieces of the partition)
+    size_t ws_o_off, ws_lse_off;
     size_t ws_bytes;
     int comb_smem;
     int comb_grid;
@@ -213,34 +215,40 @@ int choose_variant(const Shapes &s) {
     return FA_VARIANT_MMA;
 }
 
-// Host copy of the device schedule for dense inputs (every batch has Lk keys):
-// returns W, and whether some unit is cut between CTAs or has no tiles.
-void host_schedule(const Shapes &s, int causal, int TK, int64_t P, int64_t min_share, int64_t *W_out,
-                   int64_t *Peff_out, bool *need_combine) {
-    std::vector<int64_t> pre(s.BR + 1, 0);
+// Host copy of the device partition for dense inputs (every batch has Lk keys):
+// returns W and the partition, and whether some unit is cut between pieces
+// or has no tiles (then the combine kernel has work).
+void host_schedule(const Shapes &s, int causal, int tile_shift, int P, int min_share, int *W_out,
+                   fa::Partition *pt_out, bool *need_combine) {
+    std::vector<int> pre(s.BR + 1, 0);
     bool empty_unit = false;
     for (int x = 0; x < s.BR; ++x) {
-        int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, TK);
+        int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, tile_shift);
         if (t == 0) empty_unit = true;
-        pre[x + 1] = pre[x] + (int64_t)s.Hkv * t;
+        pre[x + 1] = pre[x] + s.Hkv * t;
     }
-    int64_t W = pre[s.BR];
-    int64_t Peff = fa::eff_parts(W, P, min_share);
+    const int W = pre[s.BR];
+    const fa::Partition pt = fa::make_partition(W, P, min_share);
     bool split = false;
-    for (int64_t c = 1; c < Peff && !split; ++c) {
-        int64_t pos = fa::part_start(c, W, Peff);
-        // entry containing pos
-        int lo = 0, hi = s.BR - 1;
+    for (int c = 1; c < fa::num_pieces(pt) && !split && W > 0; ++c) {
+        const int pos = fa::piece_start(pt, c);
+        int lo = 0, hi = s.BR - 1;  // entry containing pos
         while (lo < hi) {
             int mid = (lo + hi + 1) / 2;
             if (pre[mid] <= pos) lo = mid; else hi = mid - 1;
         }
-        int64_t t = (pre[lo + 1] - pre[lo]) / s.Hkv;
+        const int t = (pre[lo + 1] - pre[lo]) / s.Hkv;
         if (t > 0 && (pos - pre[lo]) % t != 0) split = true;
     }
     *W_out = W;
-    *Peff_out = Peff;
+    *pt_out = pt;
     *need_combine = split || empty_unit;
+}
+
+int log2_exact(int v) {
+    int k = 0;
+    while ((1 << k) < v) ++k;
+    return k;
 }
 
 fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl) {
@@ -257,12 +265,17 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     if (!fa::get_combine_kernel(s.dtype, s.Dv, &pl->comb))
         return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.Dv);
     if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
-    pl->comb_smem = (s.BR + 1) * 8;
+    pl->comb_smem = 0;
     int comb_occ = 0;
     if ((st = prepare_fn(pl->comb.fn, pl->comb.threads, pl->comb_smem, &comb_occ))) return st;
 
     const int TK = pl->main.tile_keys;
+    const int tile_shift = log2_exact(TK);
     const int64_t units = (int64_t)s.B * s.RB * s.Hkv;
+    // every tile position must fit in 32 bits
+    const int64_t max_tiles = units * (((int64_t)s.Lk + TK - 1) / TK);
+    if (max_tiles >= (int64_t(1) << 31) - 1)
+        return fail(FA_ERR_UNSUPPORTED, "problem too large: %lld key tiles", (long long)max_tiles);
     int64_t P;
     if (num_splits > 0) {
         P = units * num_splits;
@@ -275,24 +288,29 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     if (P < 1) P = 1;
     pl->P_param = (int)P;
     if (!kvcache) {
-        int64_t W, Peff;
+        int W;
+        fa::Partition pt;
         bool need;
-        host_schedule(s, causal, TK, P, pl->min_share, &W, &Peff, &need);
+        host_schedule(s, causal, tile_shift, (int)P, pl->min_share, &W, &pt, &need);
+        if (num_splits <= 0 && W <= P) {  // small problem: one tile per CTA, as many CTAs as tiles
+            pl->min_share = 1;
+            host_schedule(s, causal, tile_shift, (int)P, pl->min_share, &W, &pt, &need);
+        }
         pl->W = W;
-        pl->P = (int)Peff;
-        pl->P_param = (int)Peff;  // same partition, no idle CTAs
+        pl->P = W > 0 ? pt.P : 0;  // W == 0: nothing to stream, the combine writes every row
         pl->need_combine = need;
-        if (W == 0) pl->P = 0;    // nothing to stream: the combine writes every row
     } else {
         pl->W = -1;
         pl->P = max_keys > 0 ? (int)P : 0;  // an empty cache: the combine writes every row
         pl->need_combine = true;
     }
-    const bool any_partial = kvcache || pl->need_combine;
-    pl->ws_o_floats = any_partial ? (size_t)pl->P_param * 2 * fa::kRowsPerCta * s.Dv : 0;
-    size_t lse_floats = any_partial ? (size_t)pl->P_param * 2 * fa::kRowsPerCta : 0;
-    size_t o_bytes = (pl->ws_o_floats * 4 + 255) & ~size_t(255);
-    pl->ws_bytes = any_partial ? o_bytes + ((lse_floats * 4 + 255) & ~size_t(255)) : 0;
+    pl->need_workspace = pl->need_combine;
+    pl->pieces = (size_t)pl->P_param;  // one piece per CTA
+    const size_t o_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta * s.Dv : 0;
+    const size_t lse_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta : 0;
+    pl->ws_o_off = 0;
+    pl->ws_lse_off = pl->ws_o_off + ((o_floats * 4 + 255) & ~size_t(255));
+    pl->ws_bytes = pl->need_workspace ? pl->ws_lse_off + ((lse_floats * 4 + 255) & ~size_t(255)) : 0;
     int64_t rows = (int64_t)s.B * s.Hq * s.Lq;
     pl->comb_grid = (int)((rows + 3) / 4);
     return FA_OK;
@@ -387,10 +405,10 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.o_sl = o->stride[1];
     p.o_sh = o->stride[2];
     p.lse = lse;
-    p.ws_o = pl.ws_bytes ? static_cast<float *>(workspace) : nullptr;
-    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                                       ((pl.ws_o_floats * 4 + 255) & ~size_t(255)))
-                           : nullptr;
+    char *wsb = static_cast<char *>(workspace);
+    p.ws_o = pl.ws_bytes ? reinterpret_cast<float *>(wsb + pl.ws_o_off) : nullptr;
+    p.ws_lse = pl.ws_bytes ? reinterpret_cast<float *>(wsb + pl.ws_lse_off) : nullptr;
+    p.W_host = pl.W >= 0 ? (int)pl.W : -1;
     p.seqlens = seqlens;
     p.status = dev->status;
     p.B = s.B;
@@ -407,6 +425,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.P = pl.P_param;
     p.min_share = pl.min_share;
     p.tile_keys = pl.main.tile_keys;
+    p.tile_shift = log2_exact(pl.main.tile_keys);
 
     bool prof = false;
     ProfRec *rec = nullptr;
@@ -436,6 +455,15 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         cfg.blockDim = dim3((unsigned)pl.main.threads);
         cfg.dynamicSmemBytes = (size_t)pl.main.smem;
         cfg.stream = stream;
+        // Programmatic dependent launch: the kernel's prologue may overlap the
+        // previous kernel in the stream; it waits for it before touching memory.
+        cudaLaunchAttribute mattr[1];
+        mattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        mattr[0].val.programmaticStreamSerializationAllowed = 1;
+        if (!prof) {
+            cfg.attrs = mattr;
+            cfg.numAttrs = 1;
+        }
         void *args[] = {&tmK, &tmV, &p};
         if (prof && (st = prof_record(&rec->e0, stream))) return st;
         cudaError_t e = cudaLaunchKernelExC(&cfg, pl.main.fn, args);
@@ -458,7 +486,6 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
             cfg.attrs = attr;
             cfg.numAttrs = 1;
         }
-        if (!launch_main) p.P = 1;
         void *args[] = {&p};
         cudaError_t e = cudaLaunchKernelExC(&cfg, pl.comb.fn, args);
         if (e != cudaSuccess) return cuda_fail(e, "launch of the combine kernel");
@@ -617,29 +644,32 @@ fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const 
                       int min_share, int tile_keys, int64_t *work_tiles, int64_t *ctas_used, int32_t *unit_tiles,
                       int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units) {
     if (B < 0 || Lq < 0 || Hq <= 0 || Hkv <= 0 || Lk < 0 || Hq % Hkv || num_ctas < 1 || min_share < 1 ||
-        tile_keys < 1 || max_units < 0)
+        tile_keys < 1 || (tile_keys & (tile_keys - 1)) || max_units < 0)
         return fail(FA_ERR_INVALID_ARG, "fa_schedule: inconsistent sizes");
     const int g = Hq / Hkv, R = g * Lq, RB = (R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
+    const int shift = log2_exact(tile_keys);
     const int64_t BR = (int64_t)B * RB;
-    std::vector<int64_t> pre(BR + 1, 0);
+    if (BR * Hkv * (((int64_t)Lk + tile_keys - 1) / tile_keys) >= (int64_t(1) << 31) - 1)
+        return fail(FA_ERR_UNSUPPORTED, "fa_schedule: problem too large");
+    std::vector<int> pre(BR + 1, 0);
     std::vector<int32_t> tx(BR, 0);
     for (int64_t x = 0; x < BR; ++x) {
         int n = fa::batch_keys(seqlens, (int)(x / RB), Lk);
-        tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, tile_keys);
-        pre[x + 1] = pre[x] + (int64_t)Hkv * tx[x];
+        tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, shift);
+        pre[x + 1] = pre[x] + Hkv * tx[x];
     }
-    const int64_t W = pre[BR];
-    const int64_t P = fa::eff_parts(W, num_ctas, min_share);
+    const int W = pre[BR];
+    const fa::Partition pt = fa::make_partition(W, num_ctas, min_share);
     if (work_tiles) *work_tiles = W;
-    if (ctas_used) *ctas_used = P;
+    if (ctas_used) *ctas_used = pt.P;
     int64_t u = 0;
     for (int64_t x = 0; x < BR && u < max_units; ++x)
         for (int h = 0; h < Hkv && u < max_units; ++h, ++u) {
-            const int64_t u0 = pre[x] + (int64_t)h * tx[x];
+            const int u0 = pre[x] + h * tx[x];
             if (unit_tiles) unit_tiles[u] = tx[x];
             const bool has = tx[x] > 0;
-            if (unit_first_cta) unit_first_cta[u] = has ? fa::part_of(u0, W, P) : -1;
-            if (unit_last_cta) unit_last_cta[u] = has ? fa::part_of(u0 + tx[x] - 1, W, P) : -1;
+            if (unit_first_cta) unit_first_cta[u] = has ? fa::piece_of(pt, u0) : -1;
+            if (unit_last_cta) unit_last_cta[u] = has ? fa::piece_of(pt, u0 + tx[x] - 1) : -1;
         }
     t_err.clear();
     return FA_OK;

@@ -1,7 +1,8 @@
 // fa_combine.cu -- log-sum-exp weighted merge of split-KV partials.
 //
-// For an output row whose unit was cut across CTAs s = first..last, each CTA
-// left a normalised partial O_s and its log2-sum-exp lse2_s.  The row's
+// For an output row whose unit was cut across pieces s = first..last of the
+// work partition, each piece left a normalised partial O_s and its
+// log2-sum-exp lse2_s.  The row's
 // result is
 //     L2 = M + log2 sum_s 2^(lse2_s - M),     M = max_s lse2_s
 //     O  = sum_s 2^(lse2_s - L2) O_s,         lse = L2 * ln 2
@@ -9,8 +10,11 @@
 // splits: CSDN "FlashAttention on Ascend CANN" post, "在线 Softmax" section;
 // split-KV partials as in the M1 split-KV decode kernel of the MXFlashAttn
 // README).  Rows whose unit has no visible key get O = 0, lse = -inf; rows
-// finished inside one CTA were already written by the main kernel and are
+// finished inside one piece were already written by the main kernel and are
 // skipped.  One warp per row; lanes cover the head dim with vector loads.
+// Each warp re-derives the work partition from the sizes (and cache lengths)
+// exactly as the split-KV kernel did: a partial lives at a fixed slot of the
+// piece that produced it, whichever CTA ran that piece.
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
@@ -18,30 +22,52 @@ namespace fa {
 
 constexpr int kCombineThreads = 128;
 
+constexpr int kPartsPerPass = 8;  // partials one warp handles per pass (one per lane)
+
 template <typename T, int DV>
 __global__ void __launch_bounds__(kCombineThreads)
     combine_kernel(const Params p) {
-    extern __shared__ long long pre[];  // BR + 1 entries
-    __shared__ long long warp_tot[kCombineThreads / 32];
-    // seqlens is an input of the whole call: it was complete before the main
-    // kernel started, so the schedule can be rebuilt before waiting on it.
-    build_prefix<kCombineThreads>(p, pre, warp_tot);
-    const long long W = pre[p.B * p.RB];
-    const long long P = eff_parts(W, p.P, p.min_share);
+    // The next kernel in the stream may start its prologue now; it still waits
+    // for this grid to finish before touching memory.
+    pdl_launch_dependents();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * (kCombineThreads / 32) + warp;
     const long long rows = (long long)p.B * p.Hq * p.Lq;
-    if (row >= rows) return;
-    const int i = (int)(row % p.Lq);
-    const int hq = (int)((row / p.Lq) % p.Hq);
-    const int b = (int)(row / ((long long)p.Lq * p.Hq));
+    const bool live = row < rows;
+    const int i = live ? (int)(row % p.Lq) : 0;
+    const int hq = live ? (int)((row / p.Lq) % p.Hq) : 0;
+    const int b = live ? (int)(row / ((long long)p.Lq * p.Hq)) : 0;
     const int r = (hq % p.g) * p.Lq + i;
     const int rb = r / kRowsPerCta, rr = r % kRowsPerCta, hkv = hq / p.g;
-    const int n = batch_keys(p.seqlens, b, p.Lk);
-    const int t = unit_tiles(n, rb, p.R, p.Lq, p.causal, p.tile_keys);
+    const int x = b * p.RB + rb;
 
+    // The partition and the partials' addresses are worked out before the
+    // wait (dense inputs need no memory for it); cache lengths only after it.
     constexpr int EPL = DV / 32;  // elements per lane
+    int t = 0, u0 = 0, cf = 0, nparts = 0;
+    long long base0 = 0;  // this lane's partial in the first pass
+    Partition pt = {0, 1};
+    auto plan = [&]() {
+        pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
+        t = entry_tiles(p, x);
+        u0 = warp_entry_begin(p, x) + hkv * t;
+        if (t > 0) {
+            cf = piece_of(pt, u0);
+            nparts = piece_of(pt, u0 + t - 1) - cf + 1;
+            const int c = cf + lane;
+            if (lane < kPartsPerPass && lane < nparts)
+                base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr;
+        }
+    };
+    if (!p.seqlens) plan();
+    // Every CTA waits for the split-KV kernel before it exits, so this grid
+    // completing implies that one completed too.
+    pdl_wait_primary();
+    if (p.seqlens) plan();
+    if (!live) return;
+    if (t > 0 && nparts == 1) return;  // finished inside one piece by the split-KV kernel
+
     T *op = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh +
             lane * EPL;
     float acc[EPL];
@@ -50,41 +76,60 @@ __global__ void __launch_bounds__(kCombineThreads)
     float lse2 = -INFINITY;
 
     if (t > 0) {
-        const long long u0 = pre[b * p.RB + rb] + (long long)hkv * t;
-        const long long u1 = u0 + t;
-        const long long cf = part_of(u0, W, P), cl = part_of(u1 - 1, W, P);
-        if (cf == cl) return;  // finished by one CTA
-        pdl_wait_primary();    // partials come from the main kernel
-        auto slot_of = [&](long long c) { return part_start(c, W, P) >= u0 ? 0 : 1; };
-        float M = -INFINITY;
-        for (long long c = cf + lane; c <= cl; c += 32)
-            M = fmaxf(M, p.ws_lse[(c * 2 + slot_of(c)) * kRowsPerCta + rr]);
+        float M = -INFINITY, L = 0.f;
+        for (int j0 = 0; j0 < nparts; j0 += kPartsPerPass) {
+            // lane j < kPartsPerPass owns partial cf + j0 + j; its lse and every
+            // lane's O slices of the pass are loaded together
+            const int c = cf + j0 + lane;
+            const bool has = lane < kPartsPerPass && j0 + lane < nparts;
+            const long long base =
+                j0 == 0 ? base0
+                        : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr : 0);
+            const int cnt = nparts - j0 < kPartsPerPass ? nparts - j0 : kPartsPerPass;
+            const float ls = has ? p.ws_lse[base] : -INFINITY;
+            float v[kPartsPerPass][EPL];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        if (M != -INFINITY) {
-            float L = 0.f;
-            for (long long c = cf + lane; c <= cl; c += 32) {
-                const float ls = p.ws_lse[(c * 2 + slot_of(c)) * kRowsPerCta + rr];
-                L += fast_exp2(ls - M);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-            lse2 = M + log2f(L);
-            for (long long c = cf; c <= cl; ++c) {
-                const long long base = (c * 2 + slot_of(c)) * kRowsPerCta + rr;
-                const float w = fast_exp2(p.ws_lse[base] - lse2);
-                const float *src = p.ws_o + base * DV + lane * EPL;
-                if constexpr (EPL == 4) {
-                    const float4 x = *reinterpret_cast<const float4 *>(src);
-                    acc[0] += w * x.x;
-                    acc[1] += w * x.y;
-                    acc[2] += w * x.z;
-                    acc[3] += w * x.w;
-                } else {
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[e] += w * src[e];
+            for (int q = 0; q < kPartsPerPass; ++q) {
+                const long long bq = __shfl_sync(0xffffffffu, base, q);
+                if (q < cnt) {
+                    const float *src = p.ws_o + bq * DV + lane * EPL;
+                    if constexpr (EPL == 4) {
+                        const float4 x4 = *reinterpret_cast<const float4 *>(src);
+                        v[q][0] = x4.x; v[q][1] = x4.y; v[q][2] = x4.z; v[q][3] = x4.w;
+                    } else {
+                        const float2 x2 = *reinterpret_cast<const float2 *>(src);
+                        v[q][0] = x2.x; v[q][1] = x2.y;
+                    }
                 }
             }
+            float mx = ls;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            const float Mn = fmaxf(M, mx);
+            if (Mn == -INFINITY) continue;
+            const float w = ls == -INFINITY ? 0.f : fast_exp2(ls - Mn);  // unnormalised weight
+            float sum = w;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            const float scale_old = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+            L = L * scale_old + sum;
+            M = Mn;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] *= scale_old;
+#pragma unroll
+            for (int q = 0; q < kPartsPerPass; ++q) {
+                const float wq = __shfl_sync(0xffffffffu, w, q);
+                if (q < cnt) {
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e) acc[e] += wq * v[q][e];
+                }
+            }
+        }
+        if (M != -INFINITY) {
+            const float inv = 1.f / L;
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] *= inv;
+            lse2 = M + log2f(L);
         }
     }
 #pragma unroll
@@ -98,7 +143,7 @@ template <typename T, int DV>
 static void fill(KernelInfo *out) {
     out->fn = reinterpret_cast<const void *>(&combine_kernel<T, DV>);
     out->threads = kCombineThreads;
-    out->smem = 0;  // the host adds (BR + 1) * 8 bytes
+    out->smem = 0;
     out->tile_keys = 0;
     out->stages = 0;
     out->variant = 0;

@@ -26,8 +26,8 @@ struct Params {
     void *o;  // [B, Lq, Hq, Dv]
     int64_t o_sb, o_sl, o_sh;
     float *lse;            // [B, Hq, Lq] or null
-    float *ws_o;           // partial outputs [P][2][8][Dv]
-    float *ws_lse;         // partial log2-sum-exp [P][2][8]
+    float *ws_o;           // partial outputs [pieces][2][8][Dv]
+    float *ws_lse;         // partial log2-sum-exp [pieces][2][8]
     const int *seqlens;    // [B] or null (then every batch has Lk keys)
     unsigned *status;      // device status word (timeouts)
     int B, Lq, Hq, Hkv, g, R, RB, Lk;
@@ -35,7 +35,9 @@ struct Params {
     float scale_log2;      // scale * log2(e)
     int P;                 // CTAs launched
     int min_share;         // least tiles per CTA
-    int tile_keys;         // keys per tile (TK)
+    int W_host;            // total tiles when known on the host (dense inputs), else -1
+    int tile_keys;         // keys per tile (TK), a power of two
+    int tile_shift;        // log2(tile_keys)
 };
 
 // ------------------------------------------------------------------ schedule
@@ -52,13 +54,12 @@ struct Params {
 __host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int Lq, int causal) {
     if (n <= 0) return 0;
     if (!causal) return n;
-    int r0 = rb * kRowsPerCta;
-    int r1 = r0 + kRowsPerCta < R ? r0 + kRowsPerCta : R;
-    int maxi = -1;
-    for (int r = r0; r < r1; ++r) {
-        int i = r % Lq;
-        maxi = i > maxi ? i : maxi;
-    }
+    // rows r0 .. r0 + cnt - 1 hold query positions i = r % Lq; the largest one
+    // is r0 % Lq + cnt - 1 unless the run wraps past Lq - 1.
+    const int r0 = rb * kRowsPerCta;
+    const int cnt = R - r0 < kRowsPerCta ? R - r0 : kRowsPerCta;
+    const int a = r0 % Lq;
+    const int maxi = (a + cnt - 1 >= Lq) ? Lq - 1 : a + cnt - 1;
     int k = maxi + n - Lq + 1;  // bottom-right: row i sees keys j <= i + n - Lq
     if (k > n) k = n;
     return k > 0 ? k : 0;
@@ -71,27 +72,56 @@ __host__ __device__ inline int batch_keys(const int *seqlens, int b, int Lk) {
     return n < 0 ? 0 : (n > Lk ? Lk : n);
 }
 
-__host__ __device__ inline int unit_tiles(int n, int rb, int R, int Lq, int causal, int TK) {
-    int k = keys_visible_to_block(n, rb, R, Lq, causal);
-    return (k + TK - 1) / TK;
+// Tiles of tile_keys = 1 << tile_shift keys covering the visible keys.
+__host__ __device__ inline int unit_tiles(int n, int rb, int R, int Lq, int causal, int tile_shift) {
+    const int k = keys_visible_to_block(n, rb, R, Lq, causal);
+    return (k + (1 << tile_shift) - 1) >> tile_shift;
 }
 
-__host__ __device__ inline int64_t eff_parts(int64_t W, int64_t P, int64_t min_share) {
-    int64_t need = (W + min_share - 1) / min_share;
-    int64_t p = P < need ? P : need;
+// Tile positions fit in 32 bits (the host rejects larger problems).
+__host__ __device__ inline int eff_parts(int W, int P, int min_share) {
+    const int need = (W + min_share - 1) / min_share;
+    const int p = P < need ? P : need;
     return p < 1 ? 1 : p;
 }
 
-__host__ __device__ inline int64_t part_start(int64_t c, int64_t W, int64_t P) { return (c * W) / P; }
+// Balanced contiguous partition of W tiles over P CTAs: the first W % P CTAs
+// take one tile more than the others.
+__host__ __device__ inline int part_start(int c, int W, int P) {
+    const int share = W / P, rem = W % P;
+    return c * share + (c < rem ? c : rem);
+}
 
 // The CTA whose range contains tile position t (0 <= t < W).
-__host__ __device__ inline int64_t part_of(int64_t t, int64_t W, int64_t P) {
-    int64_t c = (t * P) / W;
-    if (c >= P) c = P - 1;
-    while (c + 1 < P && part_start(c + 1, W, P) <= t) ++c;
-    while (c > 0 && part_start(c, W, P) > t) --c;
-    return c;
+__host__ __device__ inline int part_of(int t, int W, int P) {
+    const int share = W / P, rem = W % P;
+    const int big = (share + 1) * rem;
+    return t < big ? t / (share + 1) : rem + (t - big) / share;
 }
+
+// The work partition: W tiles over P = eff_parts(...) CTAs, CTA c taking the
+// contiguous piece [part_start(c), part_start(c + 1)).  A piece leaves up to
+// two partial results (slot 0: the unit it starts in, slot 1: the unit it ends
+// in) for units it shares with other pieces; a unit inside one piece is
+// finished directly.  (A dynamic tail -- CTAs claiming the last quarter of the
+// tiles from a counter -- evened out when CTAs finish but did not move the
+// last one, since the kernel is bound by the total DRAM bandwidth, and cost
+// more than it saved.)
+struct Partition {
+    int W, P;
+};
+
+__host__ __device__ inline Partition make_partition(int W, int P_param, int min_share) {
+    Partition q;
+    q.W = W;
+    q.P = eff_parts(W, P_param, min_share);
+    return q;
+}
+
+__host__ __device__ inline int piece_of(const Partition &q, int t) { return part_of(t, q.W, q.P); }
+__host__ __device__ inline int piece_start(const Partition &q, int id) { return part_start(id, q.W, q.P); }
+__host__ __device__ inline int piece_end(const Partition &q, int id) { return part_start(id + 1, q.W, q.P); }
+__host__ __device__ inline int num_pieces(const Partition &q) { return q.P; }
 
 // ------------------------------------------------------------------ PTX wrappers
 #if defined(__CUDACC__)
@@ -252,6 +282,35 @@ __device__ __forceinline__ void pdl_wait_primary() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Sync of the consumer warps through an mbarrier (one arrival per warp), with
+// the same bounded wait as the pipeline: a warp that gave up never leaves the
+// others blocked.  `phase` is the caller's running parity.
+__device__ __forceinline__ bool consumer_sync_bounded(uint32_t bar, uint32_t &phase, volatile int *abort,
+                                                      unsigned *status, uint64_t limit_ns) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, phase, abort, status, limit_ns);
+    phase ^= 1u;
+    return __all_sync(0xffffffffu, ok);
+}
+
+// 16-byte global -> shared copy on the LSU async path (cp.async); src_bytes = 0
+// fills the 16 bytes with zeros without reading global memory.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+// The mbarrier's current phase also waits for this thread's earlier cp.async
+// copies (the pending count is raised now and lowered when they land).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void consumer_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
 }
@@ -283,79 +342,104 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16 *dst, co
     *reinterpret_cast<uint4 *>(dst) = u;
 }
 
-// Exclusive prefix over the (batch, row-block) entries: pre[x] = Hkv * (tiles
-// of entries before x), pre[BR] = W.  Runs on the whole CTA (NT
-// threads); pre must hold BR + 1 int64 in shared memory, warp_tot NT / 32.
-template <int NT>
-__device__ __forceinline__ void build_prefix(const Params &p, long long *pre, long long *warp_tot) {
-    const int BR = p.B * p.RB;
-    const int tid = threadIdx.x;
-    const int per = (BR + NT - 1) / NT;
-    const int lo = tid * per;
-    const int hi = lo + per < BR ? lo + per : BR;
-    long long local = 0;
-    for (int x = lo; x < hi; ++x) {
-        int b = x / p.RB, rb = x % p.RB;
-        int n = batch_keys(p.seqlens, b, p.Lk);
-        local += unit_tiles(n, rb, p.R, p.Lq, p.causal, p.tile_keys);
-    }
-    // inclusive warp scan
-    const int lane = tid & 31, warp = tid >> 5;
-    long long incl = local;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        long long y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    long long base = 0;
-    for (int w = 0; w < warp; ++w) base += warp_tot[w];
-    long long run = base + incl - local;  // exclusive prefix of this thread's chunk
-    for (int x = lo; x < hi; ++x) {
-        int b = x / p.RB, rb = x % p.RB;
-        int n = batch_keys(p.seqlens, b, p.Lk);
-        pre[x] = run * p.Hkv;
-        run += unit_tiles(n, rb, p.R, p.Lq, p.causal, p.tile_keys);
-    }
-    if (tid == NT - 1) pre[BR] = run * p.Hkv;
-    __syncthreads();
+// ------------------------------------------------------------------ warp-level schedule
+// Every warp of a CTA derives the same schedule on its own, in registers, so
+// the copy pipeline can start without a block-wide prefix in shared memory.
+// Entries x = b * RB + rb are visited in chunks of 32 (one per lane).
+
+__device__ __forceinline__ int entry_tiles(const Params &p, int x) {
+    const int b = x / p.RB, rb = x - b * p.RB;
+    return unit_tiles(batch_keys(p.seqlens, b, p.Lk), rb, p.R, p.Lq, p.causal, p.tile_shift);
 }
 
-// Largest x in [0, BR) with pre[x] <= t (t < pre[BR]); that entry has tiles.
-__device__ __forceinline__ int find_entry(const long long *pre, int BR, long long t) {
-    int lo = 0, hi = BR - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= t) lo = mid; else hi = mid - 1;
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+    return v;
+}
+
+// Tiles of all units of entries [x0, x1), counted Hkv times (one per kv head).
+__device__ __forceinline__ int warp_entry_tiles(const Params &p, int x0, int x1) {
+    const int lane = threadIdx.x & 31;
+    int acc = 0;
+    for (int x = x0 + lane; x < x1; x += 32) acc += entry_tiles(p, x);
+    return warp_sum(acc) * p.Hkv;
+}
+
+// Total tiles W.  Dense inputs (no seqlens): every batch has the same units.
+__device__ __forceinline__ int warp_total_tiles(const Params &p) {
+    if (p.W_host >= 0) return p.W_host;
+    if (!p.seqlens) return warp_entry_tiles(p, 0, p.RB) * p.B;
+    return warp_entry_tiles(p, 0, p.B * p.RB);
+}
+
+// First tile position of entry x's units.
+__device__ __forceinline__ int warp_entry_begin(const Params &p, int x) {
+    if (!p.seqlens) {
+        const int b = x / p.RB;
+        return warp_entry_tiles(p, 0, p.RB) * b + warp_entry_tiles(p, b * p.RB, x);
     }
-    return lo;
+    return warp_entry_tiles(p, 0, x);
+}
+
+// Entry x holding tile position t (0 <= t < W); *x_begin receives the first
+// position of x's units.
+__device__ __forceinline__ int warp_locate(const Params &p, int t, int *x_begin) {
+    const int lane = threadIdx.x & 31;
+    int x_lo = 0, x_hi = p.B * p.RB, run = 0;
+    if (!p.seqlens) {  // jump straight to the batch: all batches weigh the same
+        const int per_batch = warp_entry_tiles(p, 0, p.RB);
+        const int b = t / per_batch;
+        x_lo = b * p.RB;
+        x_hi = x_lo + p.RB;
+        run = per_batch * b;
+    }
+    for (int c0 = x_lo; c0 < x_hi; c0 += 32) {
+        const int x = c0 + lane;
+        const int tt = x < x_hi ? entry_tiles(p, x) * p.Hkv : 0;
+        int incl = tt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const int excl = run + incl - tt;
+        const unsigned hit = __ballot_sync(0xffffffffu, tt > 0 && excl <= t && t < excl + tt);
+        if (hit) {
+            const int src = __ffs(hit) - 1;
+            *x_begin = __shfl_sync(0xffffffffu, excl, src);
+            return c0 + src;
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    *x_begin = run;  // not reached for t < W
+    return x_hi - 1;
 }
 
 // Walks the segments of one CTA's tile range [start, end): each segment is a
 // run of tiles of one unit.  Producer and consumers step identical copies.
 struct SegmentWalker {
-    int x, hkv;        // current (b*RB + rb) entry and kv head
-    long long u0;      // first tile position of the current unit
-    int t;             // tiles of the current unit
-    long long pos, start, end;
+    int x, hkv;   // current (b*RB + rb) entry and kv head
+    int u0;       // first tile position of the current unit
+    int t;        // tiles of the current unit
+    int pos, start, end;
 
-    __device__ __forceinline__ void init(const Params &p, const long long *pre, long long s,
-                                         long long e) {
+    // Must be called by all 32 lanes of a warp (uses warp collectives).
+    __device__ __forceinline__ void init(const Params &p, int s, int e) {
         start = s;
         end = e;
         pos = s;
-        const int BR = p.B * p.RB;
-        x = find_entry(pre, BR, s);
-        t = (int)((pre[x + 1] - pre[x]) / p.Hkv);
-        hkv = (int)((s - pre[x]) / t);
-        u0 = pre[x] + (long long)hkv * t;
+        int xb = 0;
+        x = warp_locate(p, s, &xb);
+        t = entry_tiles(p, x);
+        hkv = (s - xb) / t;
+        u0 = xb + hkv * t;
     }
     __device__ __forceinline__ bool done() const { return pos >= end; }
     __device__ __forceinline__ int b(const Params &p) const { return x / p.RB; }
     __device__ __forceinline__ int rb(const Params &p) const { return x % p.RB; }
-    __device__ __forceinline__ long long seg_end() const {
-        long long ue = u0 + t;
+    __device__ __forceinline__ int seg_end() const {
+        const int ue = u0 + t;
         return ue < end ? ue : end;
     }
     // Move past the current segment.
@@ -370,8 +454,7 @@ struct SegmentWalker {
         for (;;) {
             ++x;
             if (x >= BR) { t = 1; return; }  // unreachable while pos < end
-            int n = batch_keys(p.seqlens, x / p.RB, p.Lk);
-            t = unit_tiles(n, x % p.RB, p.R, p.Lq, p.causal, p.tile_keys);
+            t = entry_tiles(p, x);
             if (t > 0) return;
         }
     }

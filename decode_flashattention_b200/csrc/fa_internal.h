@@ -19,6 +19,7 @@ struct KernelInfo {
 bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 // LSE-weighted combine of split partials.
 bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
+
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 

@@ -1,57 +1,79 @@
 // fa_splitkv_mma.cu -- split-KV decode / small-Q attention, tensor-core variant.
 //
-// One CTA streams a contiguous range of key tiles (see the schedule in
-// fa_common.cuh) for one or more (batch, kv-head, 8-row block) units:
+// One CTA per SM.  Its producer warp walks the CTA's piece of the key-tile
+// space (the Partition in fa_common.cuh) and feeds a ring of STAGES
+// shared-memory stages: per tile it issues TMA loads of K and V (128 keys x 64
+// elements per box, 128-byte swizzle, no multicast); at the first tile of a
+// unit's segment it also copies that unit's 8 packed query rows into the
+// stage's Q slot with cp.async, tracked by the same barrier; and it publishes
+// the tile's coordinates in the stage header.  (K-outer blocking with the next
+// tiles prefetched while the current one is consumed: "SmallQ FlashAttention
+// for Ascend 910B", section "算法要点"; the CSDN "FlashAttention on Ascend
+// CANN" post, section on pipelining HBM prefetch with compute.)
 //
-//   warp 4 (producer): one lane issues TMA tile loads of K and V (64 keys x
-//       64 elements per box, 128-byte swizzle, no multicast) into a ring of
-//       STAGES shared-memory stages, each guarded by a full/empty mbarrier pair
-//       (K-outer blocking with prefetch of the next tiles while the current one
-//       is consumed: "SmallQ FlashAttention for Ascend 910B", section "算法要点",
-//       and the CSDN "FlashAttention on Ascend CANN" post, section on
-//       pipelining HBM prefetch with compute);
-//   warps 0-3 (consumers): each takes 16 of the 64 keys of a tile and computes
-//       S^T = K Q^T with mma.sync m16n8k16 (keys are the M operand, the 8
-//       packed query rows are N, fp32 accumulation), masks, runs the online
-//       softmax in base 2 (running max m and sum l in fp32, previous
-//       accumulator rescaled by 2^(m_old - m_new) whenever the max grows:
-//       "昇腾CANN上的FlashAttention工程实战", tiling + online softmax section),
-//       turns P into the B operand with movmatrix, and accumulates
-//       O^T += V^T P^T with a second m16n8k16 (head dim as M).
-//   At the end of a unit's segment the four warps merge their (m, l, O) in
-//   shared memory and write either the final O / lse (unit finished by this
-//   CTA) or a normalised partial O and its log2-sum-exp (unit shared with
-//   other CTAs; merged by the combine kernel).
+// The four consumer warps take 32 of the 128 keys of each tile (two 16-key
+// blocks): S^T = K Q^T with mma.sync m16n8k16 (keys as M, packed query rows as
+// N, fp32 accumulation), masking, the base-2 online softmax (running max m and
+// sum l in fp32; the accumulator is rescaled by 2^(m_old - m_new) when the max
+// grows: "昇腾CANN上的FlashAttention工程实战", tiling + online softmax section),
+// P turned into the B operand with movmatrix, and O^T += V^T P^T with a second
+// m16n8k16 (head dim as M).  At the last tile of a segment the warps merge
+// their (m, l, O) through shared memory and write the final O / lse (unit
+// finished inside this piece) or a normalised partial and its log2-sum-exp
+// (unit shared with other pieces; merged by the combine kernel).
+//
+// Launched with programmatic dependent launch: barrier set-up, tensor-map
+// prefetch and (for dense K/V) the schedule run before the kernel waits for
+// the previous kernel in the stream; nothing in global memory is touched
+// before that wait.  Every wait is bounded (see mbar_wait).
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
 namespace fa {
 
+// Stage header written by the producer, read by every consumer warp.
+struct StageMeta {
+    int b, rb, hkv, tile;  // unit and key tile (keys tile * TK ...)
+    int flags, piece, slot, pad;
+};
+constexpr int kMetaFirst = 1;  // first tile of a segment: Q is in the stage, reset state
+constexpr int kMetaLast = 2;   // last tile of a segment: run the epilogue
+constexpr int kMetaWhole = 4;  // the segment is the whole unit: write O / lse
+constexpr int kMetaDone = 8;   // no more work
+constexpr int kMetaFinal = 16; // the CTA's last tile
+
+constexpr int KB = 2;  // 16-key blocks per consumer warp per tile
+
 template <int DQK, int DV, int STAGES>
 struct MmaCfg {
-    static constexpr int TK = 64;  // keys per tile: 4 consumer warps x 16
+    static constexpr int KEYS_PER_WARP = 16 * KB;
+    static constexpr int TK = KEYS_PER_WARP * kConsumerWarps;  // keys per tile
     static constexpr int KBOX = DQK / 64;
     static constexpr int VBOX = DV / 64;
-    static constexpr int BOX_BYTES = TK * 128;  // 64 keys x 64 elements x 2 bytes
-    static constexpr int STAGE_BYTES = (KBOX + VBOX) * BOX_BYTES;
-    static constexpr int RED_STRIDE = DV + 4;  // padded row: conflict-free scatter
-    static constexpr int RED_BYTES = 2 * kRowsPerCta * RED_STRIDE * 4;
-    static constexpr int OFF_RED = STAGES * STAGE_BYTES;
+    static constexpr int BOX_BYTES = TK * 128;  // TK keys x 64 elements x 2 bytes
+    static constexpr int STAGE_BYTES = (KBOX + VBOX) * BOX_BYTES;  // K and V of one tile
+    static constexpr int Q_STRIDE = DQK + 8;    // padded Q row (elements): conflict-free fragment loads
+    static constexpr int Q_BYTES = kRowsPerCta * Q_STRIDE * 2;
+    static constexpr int RED_STRIDE = DV + 4;   // padded row: conflict-free scatter
+    static constexpr int RED_BYTES = kConsumerWarps * kRowsPerCta * RED_STRIDE * 4;
+    static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+    static constexpr int OFF_RED = OFF_Q + STAGES * Q_BYTES;
     static constexpr int OFF_M = OFF_RED + RED_BYTES;
     static constexpr int OFF_L = OFF_M + kConsumerWarps * kRowsPerCta * 4;
-    static constexpr int OFF_BAR = OFF_L + kConsumerWarps * kRowsPerCta * 4;
-    static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
-    static constexpr int SMEM_USED = OFF_MISC + 16 + 8 * 8;
+    static constexpr int OFF_META = OFF_L + kConsumerWarps * kRowsPerCta * 4;
+    static constexpr int OFF_BAR = OFF_META + STAGES * (int)sizeof(StageMeta);
+    static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 1) * 8;
+    static constexpr int SMEM_USED = OFF_MISC + 16;
     static constexpr int SMEM = SMEM_USED + 1024;  // slack to align the base to 1024 B
     static_assert(DQK % 64 == 0 && DV % 64 == 0, "head dims are multiples of 64");
-    static_assert(STAGES * STAGE_BYTES >= (kMaxPrefixEntries + 1) * 8,
-                  "the stage area also holds the schedule prefix");
+    static_assert(OFF_RED % 16 == 0 && OFF_BAR % 8 == 0, "aligned regions");
+    static_assert(SMEM <= 232448, "fits the 227 KB per-CTA shared memory limit");
 };
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
 template <typename T, int DQK, int DV, int STAGES>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     splitkv_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
     using C = MmaCfg<DQK, DV, STAGES>;
@@ -59,28 +81,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-    // Let the combine kernel's CTAs be scheduled as soon as every CTA of this
-    // grid is running; the combine waits for this grid's memory before reading.
-    pdl_launch_dependents();
-
     float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
     float *sm_m = reinterpret_cast<float *>(smem + C::OFF_M);
     float *sm_l = reinterpret_cast<float *>(smem + C::OFF_L);
+    StageMeta *meta = reinterpret_cast<StageMeta *>(smem + C::OFF_META);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC);
-    long long *warp_tot = reinterpret_cast<long long *>(smem + C::OFF_MISC + 16);
-    long long *pre = reinterpret_cast<long long *>(smem);  // stage area, before any TMA
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t smem_base = smem_u32(smem);
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    const uint32_t ep_bar = smem_u32(&bars[2 * STAGES]);
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), kConsumerWarps);
         }
+        mbar_init(ep_bar, kConsumerWarps);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -88,150 +107,236 @@ __global__ void __launch_bounds__(kThreads, 2)
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
     }
-    build_prefix<kThreads>(p, pre, warp_tot);  // ends with __syncthreads
-    const long long W = pre[p.B * p.RB];
-    const long long P = eff_parts(W, p.P, p.min_share);
-    if (W == 0 || (long long)blockIdx.x >= P) return;  // uniform across the CTA
-    const long long r_start = part_start(blockIdx.x, W, P);
-    const long long r_end = part_start(blockIdx.x + 1, W, P);
-    SegmentWalker wk;
-    wk.init(p, pre, r_start, r_end);
-    __syncthreads();  // the prefix is dead from here on: the stages may be filled
+    __syncthreads();  // barriers initialised
 
     if (warp == kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        if (lane != 0) return;
+        // ============================================================ producer warp
+        // Dense inputs: the schedule needs only the kernel's parameters, so it
+        // is worked out before the wait and overlaps the previous kernel; cache
+        // lengths and the pool header are read only after the wait.
+        Partition pt = {0, 1};
+        SegmentWalker wk;
+        bool active = false;
+        const int cta = blockIdx.x;
+        auto plan = [&]() {
+            pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
+            active = pt.W > 0 && cta < pt.P;
+            if (active) wk.init(p, piece_start(pt, cta), piece_end(pt, cta));
+        };
+        if (!p.seqlens) plan();
+        pdl_wait_primary();
+        // The combine kernel's CTAs may be scheduled now (they wait for this
+        // grid to complete before reading anything it writes).
+        pdl_launch_dependents();
+        if (p.seqlens) plan();
+
+        const T *__restrict__ qg = reinterpret_cast<const T *>(p.q);
         const uint64_t policy = l2_policy_evict_first();
         int it = 0;
-        bool stop = false;
-        for (; !wk.done() && !stop; wk.advance(p)) {
-            const int b = wk.b(p), hkv = wk.hkv;
-            const long long t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
-            for (long long tt = t0; tt < t1; ++tt, ++it) {
+        bool stop = !active;
+        const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
+        for (; active && !wk.done() && !stop; wk.advance(p)) {
+            const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
+            const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
+            const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
+            const int slot = (wk.pos == lo) ? 0 : 1;
+            for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
                 const int s = it % STAGES, use = it / STAGES;
-                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) {
+                const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's control flow uniform
                     stop = true;
                     break;
                 }
                 const uint32_t kdst = smem_base + s * C::STAGE_BYTES;
                 const uint32_t vdst = kdst + C::KBOX * C::BOX_BYTES;
-                const int j = (int)(tt * C::TK);
-                mbar_arrive_expect_tx(full_bar(s), C::STAGE_BYTES);
+                // (one piece per CTA: the piece's last tile is the CTA's last tile)
+                const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
+                                  (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
+                if (lane == 0) {
+                    mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+                    const int j = tt * C::TK;
 #pragma unroll
-                for (int c = 0; c < C::KBOX; ++c)
-                    tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, j, hkv, b, policy);
+                    for (int c = 0; c < C::KBOX; ++c)
+                        tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, j, hkv, b, policy);
 #pragma unroll
-                for (int c = 0; c < C::VBOX; ++c)
-                    tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, j, hkv, b, policy);
+                    for (int c = 0; c < C::VBOX; ++c)
+                        tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, j, hkv, b, policy);
+                    StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
+                    meta[s] = m;
+                }
+                if (flags & kMetaFirst) {
+                    // the unit's 8 packed query rows (rows past g*Lq are zero), copied
+                    // asynchronously and counted on the same stage barrier
+                    const uint32_t qs = smem_base + C::OFF_Q + s * C::Q_BYTES;
+                    for (int idx = lane; idx < kRowsPerCta * (DQK / 8); idx += 32) {
+                        const int r = idx / (DQK / 8), c = idx % (DQK / 8);
+                        const int rq = rb * kRowsPerCta + r;
+                        const T *src = qg;
+                        uint32_t nbytes = 0;
+                        if (rq < p.R) {
+                            const int hq = hkv * p.g + rq / p.Lq, i = rq % p.Lq;
+                            src = qg + b * p.q_sb + (long long)i * p.q_sl + (long long)hq * p.q_sh + c * 8;
+                            nbytes = 16;
+                        }
+                        cp_async_16(qs + (r * C::Q_STRIDE + c * 8) * 2, src, nbytes);
+                    }
+                    cp_async_mbar_arrive(full_bar(s));
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full_bar(s));
             }
         }
+        // end-of-work marker in the next stage (its previous load was consumed:
+        // the empty barrier says so)
+        const int s_done = it % STAGES;
+        bool done_sent = false;
+        {
+            const int use = it / STAGES;
+            bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = __all_sync(0xffffffffu, ok);
+            if (lane == 0) {
+                StageMeta m = {0, 0, 0, 0, kMetaDone, 0, 0, 0};
+                meta[s_done] = m;
+            }
+            __syncwarp();
+            if (lane == 0 && ok) mbar_arrive(full_bar(s_done));
+            done_sent = ok;
+        }
         // Never leave the CTA with copies in flight: wait (bounded, whatever
-        // the abort state) for the last load issued into each stage.
-        const int issued = it;
-        for (int s = 0; s < STAGES && s < issued; ++s) {
-            const int last_use = (issued - 1 - s) / STAGES;
-            volatile int no_abort = 0;
-            mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, kWaitLimitNs / 8);
+        // the abort state) for the last load issued into each stage.  The
+        // marker's stage needs no wait once the marker went out.
+        if (lane == 0) {
+            for (int s = 0; s < STAGES && s < it; ++s) {
+                if (s == s_done && done_sent) continue;
+                const int last_use = (it - 1 - s) / STAGES;
+                volatile int no_abort = 0;
+                mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, kWaitLimitNs / 8);
+            }
         }
         return;
     }
 
-    // ---------------------------------------------------------------- consumers
-    const T *__restrict__ qg = reinterpret_cast<const T *>(p.q);
+    // ================================================================ consumer warps
+    pdl_wait_primary();  // outputs and workspace are written below
     T *__restrict__ og = reinterpret_cast<T *>(p.o);
-    const int kw = warp * 16;             // this warp's keys within a tile
-    const int r_lo = 2 * (lane & 3);      // accumulator rows of this lane: r_lo, r_lo + 1
-    const int ct = tid;                   // 0..127 epilogue thread index
-    constexpr int EPT = DV / 16;          // epilogue elements per thread
-    int it = 0;
+    const int kw = warp * C::KEYS_PER_WARP;  // this warp's first key within a tile
+    const int r_lo = 2 * (lane & 3);         // accumulator rows of this lane: r_lo, r_lo + 1
+    uint32_t ep_phase = 0;
 
-    for (; !wk.done(); wk.advance(p)) {
-        const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
-        const int n = batch_keys(p.seqlens, b, p.Lk);
-        const long long t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
-        const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
-        const int slot = (wk.pos == wk.start) ? 0 : 1;
-
-        // Q as the B operand: lane holds row (lane >> 2), dims 2*(lane & 3) + {0, 1} (+8).
-        uint32_t qf[DQK / 16][2];
-        {
-            const int rq = rb * kRowsPerCta + (lane >> 2);
-            if (rq < p.R) {
-                const int hq = hkv * p.g + rq / p.Lq, i = rq % p.Lq;
-                const T *qp = qg + b * p.q_sb + (long long)i * p.q_sl + (long long)hq * p.q_sh + 2 * (lane & 3);
+    // Per-lane ldmatrix offsets inside a stage (the 128-byte swizzle XORs the
+    // 16-byte chunk index with key & 7, and key & 7 == lane & 7 here).
+    uint32_t koff[DQK / 16], voff[DV / 16];
+    {
+        const int sw = lane & 7;
+        const int kkey = (lane & 7) + ((lane >> 3) & 1) * 8;  // A = K block: matrices (k0-7|k8-15) x (d lo|hi)
 #pragma unroll
-                for (int kk = 0; kk < DQK / 16; ++kk) {
-                    qf[kk][0] = *reinterpret_cast<const uint32_t *>(qp + kk * 16);
-                    qf[kk][1] = *reinterpret_cast<const uint32_t *>(qp + kk * 16 + 8);
+        for (int kk = 0; kk < DQK / 16; ++kk) {
+            const int d = kk * 16 + ((lane >> 4) & 1) * 8;
+            koff[kk] = (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4) + kkey * 128;
+        }
+        const int vkey = (lane & 7) + ((lane >> 4) & 1) * 8;  // A = V^T block: (d lo|hi) x (k0-7|k8-15)
+#pragma unroll
+        for (int t = 0; t < DV / 16; ++t) {
+            const int d = t * 16 + ((lane >> 3) & 1) * 8;
+            voff[t] = (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4) + vkey * 128;
+        }
+    }
+
+    uint32_t qf[DQK / 16][2];
+    int lim[2] = {0, 0};
+    int n = 0;
+    float m[2] = {-INFINITY, -INFINITY};
+    float l[2] = {0.f, 0.f};
+    float acc[DV / 16][4];
+
+    for (int it = 0;; ++it) {
+        const int s = it % STAGES, use = it / STAGES;
+        const bool ok = mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
+        if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;
+        const StageMeta md = meta[s];
+        if (md.flags & kMetaDone) break;
+        const uint32_t kbase = smem_base + s * C::STAGE_BYTES + kw * 128;
+        const uint32_t vbase = kbase + C::KBOX * C::BOX_BYTES;
+
+        if (md.flags & kMetaFirst) {
+            // Q as the B operand: lane holds row (lane >> 2), dims 2*(lane & 3) + {0, 1} (+8).
+            const uint32_t qrow =
+                smem_base + C::OFF_Q + s * C::Q_BYTES + ((lane >> 2) * C::Q_STRIDE + 2 * (lane & 3)) * 2;
+#pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][0]) : "r"(qrow + kk * 32));
+                asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][1]) : "r"(qrow + kk * 32 + 16));
+            }
+            n = batch_keys(p.seqlens, md.b, p.Lk);
+            // last visible key of this lane's two accumulator rows (bottom-right causal)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int r = md.rb * kRowsPerCta + r_lo + e;
+                int lm = n - 1;
+                if (p.causal && r < p.R) {
+                    const int c = r % p.Lq + n - p.Lq;
+                    lm = c < lm ? c : lm;
                 }
-            } else {
+                lim[e] = lm;
+            }
+            m[0] = m[1] = -INFINITY;
+            l[0] = l[1] = 0.f;
 #pragma unroll
-                for (int kk = 0; kk < DQK / 16; ++kk) qf[kk][0] = qf[kk][1] = 0u;
+            for (int t = 0; t < DV / 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+        }
+        const int jbase = md.tile * C::TK + kw;
+
+        // ---- S^T (16 keys x 8 rows per block) = K Q^T, two independent chains per block
+        float sc[KB][4], sd[KB][4];
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[kb][e] = sd[kb][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < DQK / 16; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4(kbase + kb * 16 * 128 + koff[kk], a0, a1, a2, a3);
+                if (kk & 1) Mma<T>::run(sd[kb], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+                else Mma<T>::run(sc[kb], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
             }
         }
-        // Last visible key of this lane's two accumulator rows (bottom-right causal).
-        int lim[2];
+        // ---- mask + online softmax (base 2)
+        float sv[KB][4];
+        float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int r = rb * kRowsPerCta + r_lo + e;
-            int l = n - 1;
-            if (p.causal && r < p.R) {
-                const int c = r % p.Lq + n - p.Lq;
-                l = c < l ? c : l;
-            }
-            lim[e] = l;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int j0 = jbase + kb * 16 + (lane >> 2), j1 = j0 + 8;
+            sv[kb][0] = j0 <= lim[0] ? (sc[kb][0] + sd[kb][0]) * p.scale_log2 : -INFINITY;
+            sv[kb][1] = j0 <= lim[1] ? (sc[kb][1] + sd[kb][1]) * p.scale_log2 : -INFINITY;
+            sv[kb][2] = j1 <= lim[0] ? (sc[kb][2] + sd[kb][2]) * p.scale_log2 : -INFINITY;
+            sv[kb][3] = j1 <= lim[1] ? (sc[kb][3] + sd[kb][3]) * p.scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(sv[kb][0], sv[kb][2]));
+            mx1 = fmaxf(mx1, fmaxf(sv[kb][1], sv[kb][3]));
         }
-
-        float m[2] = {-INFINITY, -INFINITY};
-        float l[2] = {0.f, 0.f};
-        float acc[DV / 16][4];
 #pragma unroll
-        for (int t = 0; t < DV / 16; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-
-        for (long long tt = t0; tt < t1; ++tt, ++it) {
-            const int s = it % STAGES, use = it / STAGES;
-            mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
-            const uint32_t kbase = smem_base + s * C::STAGE_BYTES;
-            const uint32_t vbase = kbase + C::KBOX * C::BOX_BYTES;
-            const int jtile = (int)(tt * C::TK);
-
-            // ---- S^T (16 keys x 8 rows) = K Q^T
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
-            {
-                const int key = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const uint32_t row = kbase + key * 128;
-                const int sw = key & 7;
+        for (int off = 4; off < 32; off <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+        const float base0 = mn0 == -INFINITY ? 0.f : mn0;
+        const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+        uint32_t pb[KB][2];
+        float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
-                for (int kk = 0; kk < DQK / 16; ++kk) {
-                    const int d = kk * 16 + ((lane >> 4) & 1) * 8;
-                    const uint32_t addr = row + (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(addr, a0, a1, a2, a3);
-                    Mma<T>::run(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-                }
-            }
-            // ---- mask + online softmax (base 2)
-            const int j0 = jtile + kw + (lane >> 2), j1 = j0 + 8;
-            float s0 = j0 <= lim[0] ? sc[0] * p.scale_log2 : -INFINITY;
-            float s1 = j0 <= lim[1] ? sc[1] * p.scale_log2 : -INFINITY;
-            float s2 = j1 <= lim[0] ? sc[2] * p.scale_log2 : -INFINITY;
-            float s3 = j1 <= lim[1] ? sc[3] * p.scale_log2 : -INFINITY;
-            float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-            }
-            const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-            const float base0 = mn0 == -INFINITY ? 0.f : mn0;
-            const float base1 = mn1 == -INFINITY ? 0.f : mn1;
+        for (int kb = 0; kb < KB; ++kb) {
+            const float p0 = fast_exp2(sv[kb][0] - base0), p2 = fast_exp2(sv[kb][2] - base0);
+            const float p1 = fast_exp2(sv[kb][1] - base1), p3 = fast_exp2(sv[kb][3] - base1);
+            ps0 += p0 + p2;
+            ps1 += p1 + p3;
+            pb[kb][0] = movmatrix_trans(Mma<T>::pack(p0, p1));  // keys 0-7 of the block
+            pb[kb][1] = movmatrix_trans(Mma<T>::pack(p2, p3));  // keys 8-15
+        }
+        // rescale what was accumulated so far only when a row's max moved
+        if (__any_sync(0xffffffffu, mn0 != m[0] || mn1 != m[1])) {
             const float al0 = fast_exp2(m[0] - base0), al1 = fast_exp2(m[1] - base1);
-            const float p0 = fast_exp2(s0 - base0), p2 = fast_exp2(s2 - base0);
-            const float p1 = fast_exp2(s1 - base1), p3 = fast_exp2(s3 - base1);
-            l[0] = l[0] * al0 + (p0 + p2);
-            l[1] = l[1] * al1 + (p1 + p3);
-            m[0] = mn0;
-            m[1] = mn1;
+            l[0] *= al0;
+            l[1] *= al1;
 #pragma unroll
             for (int t = 0; t < DV / 16; ++t) {
                 acc[t][0] *= al0;
@@ -239,40 +344,39 @@ __global__ void __launch_bounds__(kThreads, 2)
                 acc[t][2] *= al0;
                 acc[t][3] *= al1;
             }
-            const uint32_t pb0 = movmatrix_trans(Mma<T>::pack(p0, p1));  // keys 0-7
-            const uint32_t pb1 = movmatrix_trans(Mma<T>::pack(p2, p3));  // keys 8-15
-
-            // ---- cache slots at or beyond this batch's length may hold
-            // anything (NaN included): zero those V rows so 0 * V stays 0.
-            if (p.seqlens && jtile + C::TK > n) {
-                for (int idx = lane; idx < 16 * C::VBOX * 8; idx += 32) {
-                    const int key = kw + idx / (C::VBOX * 8);
-                    const int rem = idx % (C::VBOX * 8);
-                    if (jtile + key >= n) {
-                        const uint32_t a = vbase + (rem >> 3) * C::BOX_BYTES + key * 128 + (rem & 7) * 16;
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
-                    }
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-            }
-            // ---- O^T (DV x 8 rows) += V^T P^T
-            {
-                const int key = kw + (lane & 7) + ((lane >> 4) & 1) * 8;
-                const uint32_t row = vbase + key * 128;
-                const int sw = key & 7;
-#pragma unroll
-                for (int t = 0; t < DV / 16; ++t) {
-                    const int d = t * 16 + ((lane >> 3) & 1) * 8;
-                    const uint32_t addr = row + (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4);
-                    uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4_trans(addr, a0, a1, a2, a3);
-                    Mma<T>::run(acc[t], a0, a1, a2, a3, pb0, pb1);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(s));
         }
+        l[0] += ps0;
+        l[1] += ps1;
+        m[0] = mn0;
+        m[1] = mn1;
+
+        // ---- cache slots at or beyond this batch's length may hold anything
+        // (NaN included): zero those V rows so 0 * V stays 0.
+        if (p.seqlens && jbase + C::KEYS_PER_WARP > n) {
+            for (int idx = lane; idx < C::KEYS_PER_WARP * C::VBOX * 8; idx += 32) {
+                const int key = idx / (C::VBOX * 8);
+                const int rem = idx % (C::VBOX * 8);
+                if (jbase + key >= n) {
+                    const uint32_t a = vbase + (rem >> 3) * C::BOX_BYTES + key * 128 + (rem & 7) * 16;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        // ---- O^T (DV x 8 rows) += V^T P^T
+#pragma unroll
+        for (int t = 0; t < DV / 16; ++t) {
+#pragma unroll
+            for (int kb = 0; kb < KB; ++kb) {
+                uint32_t a0, a1, a2, a3;
+                ldmatrix_x4_trans(vbase + kb * 16 * 128 + voff[t], a0, a1, a2, a3);
+                Mma<T>::run(acc[t], a0, a1, a2, a3, pb[kb][0], pb[kb][1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));  // the stage (K, V, Q) is free again
+        if (!(md.flags & kMetaLast)) continue;
 
         // ------------------------------------------------------------ epilogue
         // full l of this warp's rows (sum over the 8 lanes sharing lane & 3)
@@ -287,96 +391,81 @@ __global__ void __launch_bounds__(kThreads, 2)
             sm_l[warp * kRowsPerCta + r_lo] = l[0];
             sm_l[warp * kRowsPerCta + r_lo + 1] = l[1];
         }
-        consumer_sync();
-        // per-warp weight 2^(m_w - M) / L for this lane's two rows
-        float f[2];
+        {
+            float *buf = red + warp * kRowsPerCta * C::RED_STRIDE;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int r = r_lo + e;
+            for (int t = 0; t < DV / 16; ++t) {
+                const int d = t * 16 + (lane >> 2);
+                buf[r_lo * C::RED_STRIDE + d] = acc[t][0];
+                buf[(r_lo + 1) * C::RED_STRIDE + d] = acc[t][1];
+                buf[r_lo * C::RED_STRIDE + d + 8] = acc[t][2];
+                buf[(r_lo + 1) * C::RED_STRIDE + d + 8] = acc[t][3];
+            }
+        }
+        if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
+        {
+            // thread -> (row, 8 consecutive dims); weights 2^(m_w - M) of the warps' partials
+            constexpr int EPT = DV * kRowsPerCta / (32 * kConsumerWarps);
+            constexpr int TPR = DV / EPT;
+            const int r = tid / TPR;
+            const int d0 = (tid % TPR) * EPT;
             float M = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kRowsPerCta + r]);
+            float wt[kConsumerWarps];
             float L = 0.f;
-            if (M != -INFINITY) {
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = sm_m[w * kRowsPerCta + r];
-                    if (mw != -INFINITY) L += sm_l[w * kRowsPerCta + r] * fast_exp2(mw - M);
-                }
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = sm_m[w * kRowsPerCta + r];
+                wt[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+                L += wt[w] * sm_l[w * kRowsPerCta + r];
             }
-            f[e] = (L > 0.f && m[e] != -INFINITY) ? fast_exp2(m[e] - M) / L : 0.f;
-        }
-        // tree merge of the four warps' scaled accumulators through 2 buffers
-        auto scatter = [&](float *buf) {
-#pragma unroll
-            for (int t = 0; t < DV / 16; ++t) {
-                const int d = t * 16 + (lane >> 2);
-                buf[r_lo * C::RED_STRIDE + d] = acc[t][0] * f[0];
-                buf[(r_lo + 1) * C::RED_STRIDE + d] = acc[t][1] * f[1];
-                buf[r_lo * C::RED_STRIDE + d + 8] = acc[t][2] * f[0];
-                buf[(r_lo + 1) * C::RED_STRIDE + d + 8] = acc[t][3] * f[1];
-            }
-        };
-        float *buf_w = red + (warp & 1) * kRowsPerCta * C::RED_STRIDE;
-        if (warp >= 2) scatter(buf_w);
-        consumer_sync();
-        if (warp < 2) {
-#pragma unroll
-            for (int t = 0; t < DV / 16; ++t) {
-                const int d = t * 16 + (lane >> 2);
-                acc[t][0] = acc[t][0] * f[0] + buf_w[r_lo * C::RED_STRIDE + d];
-                acc[t][1] = acc[t][1] * f[1] + buf_w[(r_lo + 1) * C::RED_STRIDE + d];
-                acc[t][2] = acc[t][2] * f[0] + buf_w[r_lo * C::RED_STRIDE + d + 8];
-                acc[t][3] = acc[t][3] * f[1] + buf_w[(r_lo + 1) * C::RED_STRIDE + d + 8];
-            }
-        }
-        consumer_sync();
-        if (warp < 2) {
-            f[0] = f[1] = 1.f;
-            scatter(buf_w);
-        }
-        consumer_sync();
-        {
-            const int r = ct / 16;
-            const int d0 = (ct % 16) * EPT;
+            const float inv = L > 0.f ? 1.f / L : 0.f;
             float v[EPT];
 #pragma unroll
-            for (int e = 0; e < EPT; ++e)
-                v[e] = red[r * C::RED_STRIDE + d0 + e] + red[(kRowsPerCta + r) * C::RED_STRIDE + d0 + e];
-            float M = -INFINITY, L = 0.f;
+            for (int e = 0; e < EPT; ++e) v[e] = 0.f;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm_m[w * kRowsPerCta + r]);
-            if (M != -INFINITY) {
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float *src = red + (w * kRowsPerCta + r) * C::RED_STRIDE + d0;
 #pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = sm_m[w * kRowsPerCta + r];
-                    if (mw != -INFINITY) L += sm_l[w * kRowsPerCta + r] * fast_exp2(mw - M);
+                for (int e = 0; e < EPT; e += 4) {
+                    const float4 x = *reinterpret_cast<const float4 *>(src + e);
+                    v[e] += wt[w] * x.x;
+                    v[e + 1] += wt[w] * x.y;
+                    v[e + 2] += wt[w] * x.z;
+                    v[e + 3] += wt[w] * x.w;
                 }
             }
-            const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
-            const int rr = rb * kRowsPerCta + r;
-            if (whole) {
-                if (rr < p.R) {
-                    const int hq = hkv * p.g + rr / p.Lq, i = rr % p.Lq;
-                    T *op = og + b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
 #pragma unroll
-                    for (int e = 0; e < EPT; e += 2) {
-                        const uint32_t w2 = Mma<T>::pack(v[e], v[e + 1]);
-                        *reinterpret_cast<uint32_t *>(op + e) = w2;
+            for (int e = 0; e < EPT; ++e) v[e] *= inv;
+            const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
+            const int rr = md.rb * kRowsPerCta + r;
+            if (md.flags & kMetaWhole) {
+                if (rr < p.R) {
+                    const int hq = md.hkv * p.g + rr / p.Lq, i = rr % p.Lq;
+                    T *op = og + md.b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
+                    if constexpr (EPT == 8) {
+                        store_row8<T>(op, v);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < EPT; e += 2)
+                            *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(v[e], v[e + 1]);
                     }
-                    if (p.lse && (ct % 16) == 0)
-                        p.lse[((long long)b * p.Hq + hq) * p.Lq + i] = lse2 * 0.69314718055994531f;
+                    if (p.lse && (tid % TPR) == 0)
+                        p.lse[((long long)md.b * p.Hq + hq) * p.Lq + i] = lse2 * 0.69314718055994531f;
                 }
             } else {
-                float *wo = p.ws_o + (((long long)blockIdx.x * 2 + slot) * kRowsPerCta + r) * DV + d0;
+                const long long base = ((long long)md.piece * 2 + md.slot) * kRowsPerCta + r;
+                float *wo = p.ws_o + base * DV + d0;
 #pragma unroll
                 for (int e = 0; e < EPT; e += 4)
                     *reinterpret_cast<float4 *>(wo + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                if ((ct % 16) == 0)
-                    p.ws_lse[((long long)blockIdx.x * 2 + slot) * kRowsPerCta + r] = lse2;
+                if ((tid % TPR) == 0) p.ws_lse[base] = lse2;
             }
         }
-        consumer_sync();  // red / sm_m / sm_l are reused by the next segment
+        // red / sm_m / sm_l are reused by the next segment, if there is one
+        if (md.flags & kMetaFinal) break;
+        if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
     }
 }
 
@@ -395,11 +484,11 @@ static void fill(KernelInfo *out, int variant) {
 bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out) {
     constexpr int kMma = 1;
     if (dtype == 0) {
-        if (dqk == 64 && dv == 64) { fill<__half, 64, 64, 5>(out, kMma); return true; }
+        if (dqk == 64 && dv == 64) { fill<__half, 64, 64, 6>(out, kMma); return true; }
         if (dqk == 128 && dv == 128) { fill<__half, 128, 128, 3>(out, kMma); return true; }
         if (dqk == 192 && dv == 128) { fill<__half, 192, 128, 2>(out, kMma); return true; }
     } else if (dtype == 1) {
-        if (dqk == 64 && dv == 64) { fill<__nv_bfloat16, 64, 64, 5>(out, kMma); return true; }
+        if (dqk == 64 && dv == 64) { fill<__nv_bfloat16, 64, 64, 6>(out, kMma); return true; }
         if (dqk == 128 && dv == 128) { fill<__nv_bfloat16, 128, 128, 3>(out, kMma); return true; }
         if (dqk == 192 && dv == 128) { fill<__nv_bfloat16, 192, 128, 2>(out, kMma); return true; }
     }

@@ -36,8 +36,10 @@
  *     beyond fp32 rounding).
  *   - workspace: caller-owned DEVICE scratch of at least the size the
  *     matching *_workspace_size call returns (it may be NULL when that size
- *     is 0).  The library never allocates device memory and never
- *     synchronises the stream in the compute calls.
+ *     is 0), 256-byte aligned; nothing in it needs initialising.  Calls that
+ *     share a workspace must not overlap in time.  The library never
+ *     allocates device memory and never synchronises the stream in the
+ *     compute calls.
  *   - stream: a cudaStream_t passed as void* (NULL = legacy default stream).
  *     All work is enqueued asynchronously on it; the caller keeps the
  *     buffers alive until it completes.
@@ -194,19 +196,21 @@ FA_API fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double
 /*
  * fa_schedule -- host-side copy of the work partition the kernels compute on
  * the device (no device access; for inspection and tests).  Work is counted
- * in key tiles of `tile_keys` keys; a unit is (batch, block of 8 packed query
- * rows, kv head), ordered batch-major, then row block, then kv head, and owns
- * ceil(visible keys / tile_keys) tiles.  The W tiles of all units are laid end
- * to end and cut into ctas_used = min(num_ctas, ceil(W / min_share)) equal
- * contiguous ranges, one per CTA.  seqlens: HOST int32 [B] (NULL: every batch
- * has Lk keys).  For each of the first max_units units the call writes its
- * tile count and the first and last CTA whose range touches it (-1, -1 for a
- * unit with no tiles).  FA_ERR_INVALID_ARG for inconsistent sizes.
+ * in key tiles of `tile_keys` keys (a power of two); a unit is (batch, block
+ * of 8 packed query rows, kv head), ordered batch-major, then row block, then
+ * kv head, and owns ceil(visible keys / tile_keys) tiles.  The W tiles of all
+ * units are laid end to end and cut into ctas_used = min(num_ctas,
+ * ceil(W / min_share)) contiguous pieces, one per CTA, whose sizes differ by
+ * at most one tile (the first W mod ctas_used pieces are the longer ones).
+ * seqlens: HOST int32 [B] (NULL: every batch has Lk keys).  For each of the
+ * first max_units units the call writes its tile count and the first and last
+ * CTA whose piece holds its tiles (-1, -1 for a unit with no tiles).
+ * FA_ERR_INVALID_ARG for inconsistent sizes.
  */
 FA_API fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens,
-                      int num_ctas, int min_share, int tile_keys, int64_t *work_tiles,
-                      int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta,
-                      int64_t *unit_last_cta, int64_t max_units);
+                             int num_ctas, int min_share, int tile_keys, int64_t *work_tiles,
+                             int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta,
+                             int64_t *unit_last_cta, int64_t max_units);
 
 /* Kernels launched by this library in this process (both kinds). */
 FA_API int64_t fa_launch_count(void);

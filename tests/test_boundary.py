@@ -135,7 +135,7 @@ def test_empty_batch_is_a_no_op():
 
 # ------------------------------------------------------------------ work partition
 
-def visible_tiles(n, rb, R, Lq, causal, TK=64):
+def visible_tiles(n, rb, R, Lq, causal, TK=128):
     """Independent restatement of the tiles a row block needs (bottom-right)."""
     if n <= 0:
         return 0
@@ -152,6 +152,7 @@ CASES = [
     dict(B=64, Lq=1, Hq=32, Hkv=8, Lk=16384, causal=False, seqlens="rand", num_ctas=296),
     dict(B=5, Lq=3, Hq=6, Hkv=2, Lk=100, causal=True, seqlens=[0, 1, 100, 2, 50], num_ctas=7),
     dict(B=3, Lq=1, Hq=2, Hkv=2, Lk=10, causal=False, seqlens=[0, 0, 0], num_ctas=9),
+    dict(B=2, Lq=1, Hq=4, Hkv=4, Lk=70000, causal=False, seqlens=None, num_ctas=11),
 ]
 
 
@@ -162,7 +163,7 @@ def test_schedule_covers_balances_and_bounds_partials(c, min_share):
     if c["seqlens"] == "rand":
         c["seqlens"] = np.random.default_rng(3).integers(1, c["Lk"] + 1, c["B"]).astype(np.int32)
     s = fa.schedule(c["B"], c["Lq"], c["Hq"], c["Hkv"], c["Lk"], c["causal"], c["seqlens"],
-                    num_ctas=c["num_ctas"], min_share=min_share)
+                    num_ctas=c["num_ctas"], min_share=min_share, tile_keys=128)
     g = c["Hq"] // c["Hkv"]
     R = g * c["Lq"]
     RB = (R + 7) // 8
@@ -180,28 +181,28 @@ def test_schedule_covers_balances_and_bounds_partials(c, min_share):
     if W == 0:
         assert np.all(s["unit_first_cta"] == -1)
         return
-    # every CTA gets floor or ceil of W / P tiles
-    shares = [((cta + 1) * W) // P - (cta * W) // P for cta in range(P)]
-    assert max(shares) - min(shares) <= 1 and min(shares) >= 1
-    # units map to non-decreasing, contiguous CTA ranges
+    # P contiguous pieces; the first W % P are one tile longer
+    share, rem = divmod(W, P)
+    starts = [cc * share + min(cc, rem) for cc in range(P)] + [W]
+    sizes = np.diff(starts)
+    assert np.all(sizes >= 1) and max(sizes) - min(sizes) <= 1
+    # each unit's first/last CTA is the one whose piece holds its first/last tile
     has = tiles > 0
     first, last = s["unit_first_cta"][has], s["unit_last_cta"][has]
-    assert np.all(first <= last) and np.all(np.diff(first) >= 0) and np.all(np.diff(last) >= 0)
+    pos = 0
+    for t, f, l in zip(tiles[has], first, last):
+        assert starts[f] <= pos < starts[f + 1]
+        assert starts[l] <= pos + int(t) - 1 < starts[l + 1]
+        pos += int(t)
+    assert pos == W
+    assert np.all(np.diff(first) >= 0) and np.all(np.diff(last) >= 0)
     assert first[0] == 0 and last[-1] == P - 1
-    # a CTA holds at most two partial units (its first and its last segment)
+    # a piece holds at most two partial units (its first and its last segment)
     partial_count = np.zeros(P, dtype=int)
     for f, l in zip(first, last):
         if f != l:
             partial_count[f:l + 1] += 1
     assert partial_count.max(initial=0) <= 2
-    # tiles per CTA add up: each unit's tiles land in [first, last]
-    covered = np.zeros(P, dtype=np.int64)
-    pos = 0
-    for t in tiles[has]:
-        for x in range(pos, pos + int(t)):
-            covered[(x * P) // W if False else np.searchsorted([(cc * W) // P for cc in range(P)], x, side="right") - 1] += 1
-        pos += int(t)
-    assert covered.tolist() == shares
 
 
 def test_hld_view_strides():
