@@ -368,8 +368,14 @@ bool g_prof_on = false;
 std::vector<ProfRec> g_prof;
 size_t g_prof_used = 0;
 
+// While the stream is being captured into a CUDA graph the events become
+// event-record nodes of the graph, so every replay re-times the kernels.
 fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
-    cudaError_t e = cudaEventRecord(*ev, stream);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    e = cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(*ev, stream, cudaEventRecordExternal)
+                                            : cudaEventRecord(*ev, stream);
     return e == cudaSuccess ? FA_OK : cuda_fail(e, "cudaEventRecord");
 }
 
@@ -612,7 +618,7 @@ fa_status fa_force_variant(int variant) {
 fa_status fa_profile_enable(int on) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     g_prof_on = on != 0;
-    g_prof_used = 0;
+    if (g_prof_on) g_prof_used = 0;
     return FA_OK;
 }
 

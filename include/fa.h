@@ -184,9 +184,13 @@ FA_API fa_status fa_force_variant(int variant);
 
 /*
  * Profiling: while enabled, each compute call brackets its main kernel and
- * its combine kernel with CUDA events on the call's stream.  Enabling
- * clears earlier records.  fa_profile_read synchronises nothing: call it after
- * the stream has completed; it returns the summed milliseconds and the
+ * its combine kernel with CUDA events on the call's stream (and launches them
+ * without programmatic overlap, so each event pair times one kernel alone).
+ * Enabling clears earlier records; disabling keeps them for fa_profile_read.
+ * Calls captured into a CUDA graph record their events as event-record nodes,
+ * so each replay of the graph writes that call's record again.
+ * fa_profile_read synchronises nothing: call it after the stream (or the
+ * graph's replay) has completed; it returns the summed milliseconds and the
  * number of timed launches of each kernel.
  */
 FA_API fa_status fa_profile_enable(int on);
