@@ -333,27 +333,18 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, world, device)
     fa.check_status()
 
-    # --- pass B: each kernel's own duration: the library brackets its launches
-    # with CUDA events on the call's stream; replayed from a graph like pass A
-    # (the events sit between the kernels, so this pass has no launch overlap) --
-    Kb = int(min(K, 1000))
-    fa.profile_enable(True)  # eager first: creates the event records outside any capture
+    # --- pass B: each kernel's own duration.  The library brackets its launches
+    # with CUDA events on the call's stream (and launches them without
+    # programmatic overlap, so each event pair times one kernel alone).  A
+    # spin kernel ahead of the calls lets the host queue them all before the
+    # first runs, so no host launch gap falls between an event and its kernel.
+    Kb = int(min(K, 200))
+    fa.profile_enable(True)
+    torch.cuda._sleep(int(40e6))  # about 20 ms of device time
     for i in range(Kb):
         step(i)
     torch.cuda.synchronize()
     prof = fa.profile_read()
-    if use_graph:
-        fa.profile_enable(True)  # reuses the records for the captured calls
-        g_prof = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_prof):
-            for i in range(Kb):
-                step(i)
-        fa.profile_enable(False)
-        for _ in range(2):  # the second replay is the one read
-            g_prof.replay()
-        torch.cuda.synchronize()
-        prof = fa.profile_read()
-        del g_prof
     fa.profile_enable(False)
     fa.check_status()
 

@@ -109,6 +109,13 @@ fa_status prepare_fn(const void *fn, int threads, int smem, int *occupancy) {
         }
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(max dynamic smem)");
+    // Every kernel of the library asks for the same (largest) shared-memory
+    // carve-out: an SM changes its L1 / shared split only when it is idle, so
+    // kernels with different carve-outs could not share an SM, which is what
+    // lets the combine kernel and the next call's split-KV kernel start while
+    // the kernel before them is still finishing.
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(shared memory carve-out)");
     int occ = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");

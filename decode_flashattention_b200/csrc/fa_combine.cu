@@ -52,6 +52,8 @@ __global__ void __launch_bounds__(kCombineThreads)
         pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
         t = entry_tiles(p, x);
         u0 = warp_entry_begin(p, x) + hkv * t;
+        nparts = 0;
+        base0 = 0;
         if (t > 0) {
             cf = piece_of(pt, u0);
             nparts = piece_of(pt, u0 + t - 1) - cf + 1;
@@ -61,82 +63,100 @@ __global__ void __launch_bounds__(kCombineThreads)
         }
     };
     if (!p.seqlens) plan();
-    // Every CTA waits for the split-KV kernel before it exits, so this grid
-    // completing implies that one completed too.
-    pdl_wait_primary();
-    if (p.seqlens) plan();
-    if (!live) return;
-    if (t > 0 && nparts == 1) return;  // finished inside one piece by the split-KV kernel
 
-    T *op = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh +
-            lane * EPL;
-    float acc[EPL];
+    // Two passes over the same code: a warm-up pass before the wait for the
+    // split-KV kernel, which merges eight copies of a shared-memory row into a
+    // shared-memory sink (its result is discarded), so that the instructions
+    // are cached when the real pass runs; then the real pass.
+    __shared__ __align__(16) float sink[DV + 4];
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const bool warm = pass == 0;
+        if (!warm) {
+            // Every CTA waits for the split-KV kernel before it exits, so this
+            // grid completing implies that one completed too.
+            pdl_wait_primary();
+            if (p.seqlens) plan();
+            if (!live) return;
+            if (t > 0 && nparts == 1) return;  // finished inside one piece by the split-KV kernel
+        }
+        const int tu = warm ? 1 : t, np = warm ? kPartsPerPass : nparts;
+        const long long b0 = warm ? 0 : base0;
+        const float *ws_o = warm ? sink : p.ws_o;
+        const float *ws_lse = warm ? sink : p.ws_lse;
+        T *op = warm ? reinterpret_cast<T *>(sink)
+                     : reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh +
+                           lane * EPL;
+        float *lse_out = warm ? sink : (p.lse ? p.lse + ((long long)b * p.Hq + hq) * p.Lq + i : nullptr);
+        const int lane_off = warm ? 0 : lane * EPL;
+        float acc[EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-    float lse2 = -INFINITY;
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        float lse2 = -INFINITY;
 
-    if (t > 0) {
-        float M = -INFINITY, L = 0.f;
-        for (int j0 = 0; j0 < nparts; j0 += kPartsPerPass) {
-            // lane j < kPartsPerPass owns partial cf + j0 + j; its lse and every
-            // lane's O slices of the pass are loaded together
-            const int c = cf + j0 + lane;
-            const bool has = lane < kPartsPerPass && j0 + lane < nparts;
-            const long long base =
-                j0 == 0 ? base0
-                        : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr : 0);
-            const int cnt = nparts - j0 < kPartsPerPass ? nparts - j0 : kPartsPerPass;
-            const float ls = has ? p.ws_lse[base] : -INFINITY;
-            float v[kPartsPerPass][EPL];
+        if (tu > 0) {
+            float M = -INFINITY, L = 0.f;
+            for (int j0 = 0; j0 < np; j0 += kPartsPerPass) {
+                // lane j < kPartsPerPass owns partial cf + j0 + j; its lse and every
+                // lane's O slices of the pass are loaded together
+                const int c = cf + j0 + lane;
+                const bool has = lane < kPartsPerPass && j0 + lane < np;
+                const long long base =
+                    j0 == 0 ? b0
+                            : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr : 0);
+                const int cnt = np - j0 < kPartsPerPass ? np - j0 : kPartsPerPass;
+                const float ls = has ? ws_lse[base] : -INFINITY;
+                float v[kPartsPerPass][EPL];
 #pragma unroll
-            for (int q = 0; q < kPartsPerPass; ++q) {
-                const long long bq = __shfl_sync(0xffffffffu, base, q);
-                if (q < cnt) {
-                    const float *src = p.ws_o + bq * DV + lane * EPL;
-                    if constexpr (EPL == 4) {
-                        const float4 x4 = *reinterpret_cast<const float4 *>(src);
-                        v[q][0] = x4.x; v[q][1] = x4.y; v[q][2] = x4.z; v[q][3] = x4.w;
-                    } else {
-                        const float2 x2 = *reinterpret_cast<const float2 *>(src);
-                        v[q][0] = x2.x; v[q][1] = x2.y;
+                for (int q = 0; q < kPartsPerPass; ++q) {
+                    const long long bq = __shfl_sync(0xffffffffu, base, q);
+                    if (q < cnt) {
+                        const float *src = ws_o + bq * DV + lane_off;
+                        if constexpr (EPL == 4) {
+                            const float4 x4 = *reinterpret_cast<const float4 *>(src);
+                            v[q][0] = x4.x; v[q][1] = x4.y; v[q][2] = x4.z; v[q][3] = x4.w;
+                        } else {
+                            const float2 x2 = *reinterpret_cast<const float2 *>(src);
+                            v[q][0] = x2.x; v[q][1] = x2.y;
+                        }
+                    }
+                }
+                float mx = ls;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float Mn = fmaxf(M, mx);
+                if (Mn == -INFINITY) continue;
+                const float w = ls == -INFINITY ? 0.f : fast_exp2(ls - Mn);  // unnormalised weight
+                float sum = w;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                const float scale_old = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+                L = L * scale_old + sum;
+                M = Mn;
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) acc[e] *= scale_old;
+#pragma unroll
+                for (int q = 0; q < kPartsPerPass; ++q) {
+                    const float wq = __shfl_sync(0xffffffffu, w, q);
+                    if (q < cnt) {
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e) acc[e] += wq * v[q][e];
                     }
                 }
             }
-            float mx = ls;
+            if (M != -INFINITY) {
+                const float inv = 1.f / L;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float Mn = fmaxf(M, mx);
-            if (Mn == -INFINITY) continue;
-            const float w = ls == -INFINITY ? 0.f : fast_exp2(ls - Mn);  // unnormalised weight
-            float sum = w;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            const float scale_old = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
-            L = L * scale_old + sum;
-            M = Mn;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] *= scale_old;
-#pragma unroll
-            for (int q = 0; q < kPartsPerPass; ++q) {
-                const float wq = __shfl_sync(0xffffffffu, w, q);
-                if (q < cnt) {
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e) acc[e] += wq * v[q][e];
-                }
+                for (int e = 0; e < EPL; ++e) acc[e] *= inv;
+                lse2 = M + log2f(L);
             }
         }
-        if (M != -INFINITY) {
-            const float inv = 1.f / L;
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] *= inv;
-            lse2 = M + log2f(L);
-        }
+        for (int e = 0; e < EPL; e += 2)
+            *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(acc[e], acc[e + 1]);
+        if (lse_out && lane == 0) *lse_out = lse2 == -INFINITY ? -INFINITY : lse2 * 0.69314718055994531f;
+        __syncwarp();
     }
-#pragma unroll
-    for (int e = 0; e < EPL; e += 2)
-        *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(acc[e], acc[e + 1]);
-    if (p.lse && lane == 0)
-        p.lse[((long long)b * p.Hq + hq) * p.Lq + i] = lse2 == -INFINITY ? -INFINITY : lse2 * 0.69314718055994531f;
 }
 
 template <typename T, int DV>

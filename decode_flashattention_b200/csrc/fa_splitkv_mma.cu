@@ -63,7 +63,8 @@ struct MmaCfg {
     static constexpr int OFF_META = OFF_L + kConsumerWarps * kRowsPerCta * 4;
     static constexpr int OFF_BAR = OFF_META + STAGES * (int)sizeof(StageMeta);
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 1) * 8;
-    static constexpr int SMEM_USED = OFF_MISC + 16;
+    static constexpr int OFF_SCRATCH = (OFF_MISC + 16 + 15) & ~15;  // sink of the warm-up pass's stores
+    static constexpr int SMEM_USED = OFF_SCRATCH + 64;
     static constexpr int SMEM = SMEM_USED + 1024;  // slack to align the base to 1024 B
     static_assert(DQK % 64 == 0 && DV % 64 == 0, "head dims are multiples of 64");
     static_assert(OFF_RED % 16 == 0 && OFF_BAR % 8 == 0, "aligned regions");
@@ -217,8 +218,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ================================================================ consumer warps
-    pdl_wait_primary();  // outputs and workspace are written below
+    // The loop below starts with two warm-up passes (it = -2, -1) that run
+    // before the wait for the previous kernel: the tile body and the epilogue
+    // (its partial-output and its final-output form) execute once on a stage
+    // that holds no data yet, with every store sent to a shared-memory sink.
+    // Their results are discarded (the first real tile resets the state).  They
+    // bring the code into the instruction caches while nothing else is waiting
+    // on these warps; otherwise the first epilogue of a CTA can stall for
+    // microseconds on instruction fetches queued behind the K/V stream.
     T *__restrict__ og = reinterpret_cast<T *>(p.o);
+    void *const sink = smem + C::OFF_SCRATCH;
     const int kw = warp * C::KEYS_PER_WARP;  // this warp's first key within a tile
     const int r_lo = 2 * (lane & 3);         // accumulator rows of this lane: r_lo, r_lo + 1
     uint32_t ep_phase = 0;
@@ -249,11 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l[2] = {0.f, 0.f};
     float acc[DV / 16][4];
 
-    for (int it = 0;; ++it) {
-        const int s = it % STAGES, use = it / STAGES;
-        const bool ok = mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
+    for (int it = -2;; ++it) {
+        const bool warm = it < 0;
+        if (it == 0) pdl_wait_primary();  // outputs and workspace are written below
+        const int s = warm ? 0 : it % STAGES, use = warm ? 0 : it / STAGES;
+        const bool ok = warm || mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
         if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;
-        const StageMeta md = meta[s];
+        StageMeta md = {0, 0, 0, 0, kMetaFirst | kMetaLast | (it == -1 ? kMetaWhole : 0), 0, 0, 0};
+        if (!warm) md = meta[s];
         if (md.flags & kMetaDone) break;
         const uint32_t kbase = smem_base + s * C::STAGE_BYTES + kw * 128;
         const uint32_t vbase = kbase + C::KBOX * C::BOX_BYTES;
@@ -267,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][0]) : "r"(qrow + kk * 32));
                 asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][1]) : "r"(qrow + kk * 32 + 16));
             }
-            n = batch_keys(p.seqlens, md.b, p.Lk);
+            n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk);
             // last visible key of this lane's two accumulator rows (bottom-right causal)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -375,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(s));  // the stage (K, V, Q) is free again
+        if (lane == 0 && !warm) mbar_arrive(empty_bar(s));  // the stage (K, V, Q) is free again
         if (!(md.flags & kMetaLast)) continue;
 
         // ------------------------------------------------------------ epilogue
@@ -443,7 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (md.flags & kMetaWhole) {
                 if (rr < p.R) {
                     const int hq = md.hkv * p.g + rr / p.Lq, i = rr % p.Lq;
-                    T *op = og + md.b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
+                    T *op = warm ? static_cast<T *>(sink)
+                                 : og + md.b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
                     if constexpr (EPT == 8) {
                         store_row8<T>(op, v);
                     } else {
@@ -452,15 +465,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(v[e], v[e + 1]);
                     }
                     if (p.lse && (tid % TPR) == 0)
-                        p.lse[((long long)md.b * p.Hq + hq) * p.Lq + i] = lse2 * 0.69314718055994531f;
+                        *(warm ? static_cast<float *>(sink) : p.lse + ((long long)md.b * p.Hq + hq) * p.Lq + i) =
+                            lse2 * 0.69314718055994531f;
                 }
             } else {
                 const long long base = ((long long)md.piece * 2 + md.slot) * kRowsPerCta + r;
-                float *wo = p.ws_o + base * DV + d0;
+                float *wo = warm ? static_cast<float *>(sink) : p.ws_o + base * DV + d0;
 #pragma unroll
                 for (int e = 0; e < EPT; e += 4)
-                    *reinterpret_cast<float4 *>(wo + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                if ((tid % TPR) == 0) p.ws_lse[base] = lse2;
+                    *reinterpret_cast<float4 *>(wo + (warm ? 0 : e)) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                if ((tid % TPR) == 0) *(warm ? static_cast<float *>(sink) : p.ws_lse + base) = lse2;
             }
         }
         // red / sm_m / sm_l are reused by the next segment, if there is one
