@@ -358,9 +358,20 @@ fa_status encode_kv_map(const fa_tensor *t, int TK, CUtensorMap *map, const char
     cuuint32_t box[4] = {64, (cuuint32_t)TK, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMapDataType dt = t->dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // L2 promotion: fetch whole 256-byte (or 128-byte) lines only when every
+    // head row starts on such a line and fills it, so a promoted fetch never
+    // pulls in bytes of a neighbouring row (a 192-element row is 384 bytes).
+    auto rows_fill = [&](uint64_t line) {
+        if (reinterpret_cast<uintptr_t>(t->data) % line || (uint64_t)(t->shape[3] * elt) % line) return false;
+        for (int i = 0; i < 3; ++i)
+            if (dims[i + 1] > 1 && strides[i] % line) return false;
+        return true;
+    };
+    const CUtensorMapL2promotion promo = rows_fill(256)   ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+                                         : rows_fill(128) ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                                          : CU_TENSOR_MAP_L2_PROMOTION_NONE;
     CUresult r = fn(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FA_ERR_UNSUPPORTED, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
     return FA_OK;
 }
