@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of graph replays")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound of the oracle CPU sample")
+    ap.add_argument("--variant", choices=["auto", "mma", "scalar"], default="auto",
+                    help="force the split-KV kernel's variant (tensor-core or fp32 FMA)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (a reduced case, e.g. for an ncu capture)")
     return ap.parse_args()
@@ -253,6 +255,7 @@ def run_ours(args):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fa.load_library()
+    fa.force_variant({"auto": fa.VARIANT_AUTO, "mma": fa.VARIANT_MMA, "scalar": fa.VARIANT_SCALAR}[args.variant])
     name = args.workload or wl.DEFAULT_BENCH
     w = workload_of(args)
     q0, k0, v0, sl0 = wl.make_inputs(w, device, seed=w.seed + 1000 * rank)
@@ -444,7 +447,7 @@ def run_ours(args):
             "workload": name, "description": w.description, "call": w.call, "layout": w.layout,
             "batch_override": args.batch or None,
             "B": w.B, "Lq": w.Lq, "Hq": w.Hq, "Hkv": w.Hkv, "Lk": w.Lk, "Dqk": w.Dqk, "Dv": w.Dv,
-            "causal": w.causal, "num_splits": args.num_splits or "auto",
+            "causal": w.causal, "num_splits": args.num_splits or "auto", "variant": args.variant,
             "kv_bytes_per_step": bytes_per_step,
             "l2": f"inputs rotate over {n_copies} copies ({n_copies * per_copy / 1e6:.0f} MB > 4x L2)",
             "launch": "cuda_graph_replay" if use_graph else "eager",

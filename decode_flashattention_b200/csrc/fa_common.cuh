@@ -267,6 +267,26 @@ struct Mma<__nv_bfloat16> {
     }
 };
 
+// 16-bit element(s) to fp32 (exact).
+template <typename T>
+struct Cvt;
+
+template <>
+struct Cvt<__half> {
+    __device__ __forceinline__ static float f1(__half x) { return __half2float(x); }
+    __device__ __forceinline__ static float2 f2(uint32_t x) {
+        return __half22float2(*reinterpret_cast<const __half2 *>(&x));
+    }
+};
+
+template <>
+struct Cvt<__nv_bfloat16> {
+    __device__ __forceinline__ static float f1(__nv_bfloat16 x) { return __bfloat162float(x); }
+    __device__ __forceinline__ static float2 f2(uint32_t x) {
+        return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x));
+    }
+};
+
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32): 2^-inf = +0.
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;

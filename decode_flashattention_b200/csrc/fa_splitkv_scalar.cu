@@ -1,9 +1,32 @@
-// fa_splitkv_scalar.cu -- split-KV attention with fp32 FMA dot products for a
-// single packed query row (placeholder registry until the kernel lands).
-#include "fa_internal.h"
+// fa_splitkv_scalar.cu -- the split-KV kernel's fp32 FMA variant for a single
+// packed query row: instances and registry (the kernel itself is in
+// fa_splitkv.cuh).
+#include "fa_splitkv.cuh"
 
 namespace fa {
 
-bool get_scalar_kernel(int, int, int, KernelInfo *) { return false; }
+template <typename T, int DQK, int DV, int STAGES>
+static void fill(KernelInfo *out) {
+    using C = SplitCfg<DQK, DV, STAGES, true>;
+    out->fn = reinterpret_cast<const void *>(&splitkv_kernel<T, DQK, DV, STAGES, true>);
+    out->threads = kThreads;
+    out->smem = C::SMEM;
+    out->tile_keys = C::TK;
+    out->stages = STAGES;
+    out->variant = 2;  // FA_VARIANT_SCALAR
+}
+
+bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out) {
+    if (dtype == 0) {
+        if (dqk == 64 && dv == 64) { fill<__half, 64, 64, 6>(out); return true; }
+        if (dqk == 128 && dv == 128) { fill<__half, 128, 128, 3>(out); return true; }
+        if (dqk == 192 && dv == 128) { fill<__half, 192, 128, 2>(out); return true; }
+    } else if (dtype == 1) {
+        if (dqk == 64 && dv == 64) { fill<__nv_bfloat16, 64, 64, 6>(out); return true; }
+        if (dqk == 128 && dv == 128) { fill<__nv_bfloat16, 128, 128, 3>(out); return true; }
+        if (dqk == 192 && dv == 128) { fill<__nv_bfloat16, 192, 128, 2>(out); return true; }
+    }
+    return false;
+}
 
 }  // namespace fa

@@ -176,8 +176,16 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
 
 /*
  * Tuning / test hook: force the main-kernel variant for later calls of this
- * process (FA_VARIANT_AUTO restores the library's choice).  A forced variant
- * that does not support the call's shapes makes the call fail with
+ * process (FA_VARIANT_AUTO restores the library's choice).
+ *   FA_VARIANT_MMA     tensor cores (mma.sync m16n8k16, keys as the 16-row
+ *                      side, up to 8 packed query rows as the 8-column side);
+ *   FA_VARIANT_SCALAR  fp32 FMA dot products, one packed query row only
+ *                      (g * Lq == 1), the "scalar fp32 dot product" form of
+ *                      "SmallQ FlashAttention for Ascend 910B", section
+ *                      "算法要点".
+ * The library's own choice is FA_VARIANT_MMA for every shape: measured on
+ * B200 it is faster than the FMA variant even for one packed row.  A forced
+ * variant that does not support the call's shapes makes the call fail with
  * FA_ERR_UNSUPPORTED.
  */
 FA_API fa_status fa_force_variant(int variant);

@@ -258,3 +258,47 @@ def test_errors_raise_without_launching():
         with pytest.raises((fa.FaError, ValueError)):
             fa.fa_fwd(q, k, k, num_splits=4, workspace=torch.empty(16, dtype=torch.uint8, device=DEV))
     assert fa.launch_count() == n0
+
+
+# ------------------------------------------------------------------ both variants on one packed row
+
+ONE_ROW = [(kv, d, dt) for kv in (1, 127, 129, 3000) for d in ((64, 64), (128, 128), (192, 128))
+           for dt in (torch.float16, torch.bfloat16) if (kv + d[0] + (dt == torch.float16)) % 2 == 0 or kv == 3000]
+
+
+@pytest.mark.parametrize("variant", ["mma", "scalar"])
+@pytest.mark.parametrize("kv,d,dt", ONE_ROW, ids=[f"kv{a}-d{b[0]}_{b[1]}-{str(c)[6:]}" for a, b, c in ONE_ROW])
+def test_one_row_both_variants(variant, kv, d, dt):
+    """g * Lq == 1: the fp32 FMA variant and the tensor-core variant must both
+    match the oracle (the library picks one of them by itself)."""
+    fa.force_variant(fa.VARIANT_MMA if variant == "mma" else fa.VARIANT_SCALAR)
+    w = wl.Workload("onerow", "fwd", "blhd", dt, B=3, Lq=1, Hq=4, Hkv=4, Lk=kv, Dqk=d[0], Dv=d[1],
+                    causal=bool(kv % 2), seed=500 + kv)
+    _, disp = check_full(w)
+    assert disp["variant"] == (fa.VARIANT_MMA if variant == "mma" else fa.VARIANT_SCALAR)
+
+
+@pytest.mark.parametrize("variant", ["mma", "scalar"])
+@pytest.mark.parametrize("num_splits", [0, 1, 3, 50])
+def test_one_row_kvcache_poisoned_tails(variant, num_splits):
+    """Cache slots past each length hold NaN; lengths include 0, 1 and tile edges."""
+    fa.force_variant(fa.VARIANT_MMA if variant == "mma" else fa.VARIANT_SCALAR)
+    w = wl.Workload("onerow_kv", "kvcache", "blhd", torch.bfloat16, B=6, Lq=1, Hq=3, Hkv=3, Lk=700,
+                    Dqk=128, Dv=128, causal=False, seed=610)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    sl = torch.tensor([0, 1, 127, 128, 129, 700], dtype=torch.int32)
+    for b in range(w.B):
+        k[b, int(sl[b]):] = float("nan")
+        v[b, int(sl[b]):] = float("nan")
+    o, lse = run_workload(w, q, k, v, sl, num_splits=num_splits)
+    ro, rl = oracle_full(q, k, v, False, seqlens=sl)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, w.dtype, w.name)
+
+
+def test_scalar_variant_refuses_packed_rows():
+    fa.force_variant(fa.VARIANT_SCALAR)
+    w = wl.Workload("rows2", "fwd", "blhd", torch.float16, B=1, Lq=2, Hq=2, Hkv=2, Lk=64, Dqk=128, Dv=128,
+                    causal=False, seed=1)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    with pytest.raises(fa.FaError, match="one packed row"):
+        fa.fa_fwd(q, k, v)
