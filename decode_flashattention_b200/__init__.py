@@ -26,7 +26,8 @@ import os
 import torch
 
 __all__ = [
-    "FaError", "fa_fwd", "fa_decode_kvcache", "flash_attn_func", "flash_attn_with_kvcache",
+    "FaError", "fa_fwd", "fa_decode_kvcache", "fa_decode_kvcache_paged", "paged_workspace_size",
+    "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
     "last_dispatch", "force_variant", "profile_enable", "profile_read", "launch_count",
     "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR",
@@ -80,6 +81,8 @@ def load_library():
         "fa_fwd_workspace_size": (i32, [T, T, T, i32, i32, P(sz)]),
         "fa_decode_kvcache": (i32, [T, T, T, vp, T, vp, i32, i32, f32, vp, sz, vp]),
         "fa_decode_kvcache_workspace_size": (i32, [T, T, T, i32, P(sz)]),
+        "fa_decode_kvcache_paged": (i32, [T, T, T, vp, ctypes.c_int64, i32, vp, T, vp, i32, i32, f32, vp, sz, vp]),
+        "fa_decode_kvcache_paged_workspace_size": (i32, [T, T, T, i32, i32, P(sz)]),
         "fa_check_status": (i32, [vp]),
         "fa_last_error": (ctypes.c_char_p, []),
         "fa_last_dispatch": (None, [P(FaDispatchInfo)]),
@@ -225,15 +228,62 @@ def fa_decode_kvcache(q, k_cache, v_cache, cache_seqlens, causal=False, scale=No
     return out, lse
 
 
+def paged_workspace_size(q, k_pages, v_pages, max_blocks_per_seq, num_splits=0) -> int:
+    lib = load_library()
+    n = ctypes.c_size_t(0)
+    with torch.cuda.device(q.device):
+        _check(lib.fa_decode_kvcache_paged_workspace_size(_desc(q, "q"), _desc(k_pages, "k_pages"),
+                                                          _desc(v_pages, "v_pages"), int(max_blocks_per_seq),
+                                                          int(num_splits), ctypes.byref(n)))
+    return n.value
+
+
+def fa_decode_kvcache_paged(q, k_pages, v_pages, block_table, cache_seqlens, causal=False, scale=None,
+                            num_splits=0, out=None, lse=None, workspace=None, return_lse=True):
+    """Attention of q [B, Lq, Hq, Dqk] against a paged cache: k_pages / v_pages
+    [num_blocks, page, Hkv, D], block_table CUDA int32 [B, max_blocks_per_seq]
+    (row stride free, unit column stride), cache_seqlens CUDA int32 [B]; key j
+    of batch b is row j % page of block block_table[b, j // page]."""
+    lib = load_library()
+    dev = _cuda_inputs(q, k_pages, v_pages, block_table, cache_seqlens)
+    if cache_seqlens.dtype != torch.int32 or cache_seqlens.dim() != 1 or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous int32 [B] tensor")
+    if cache_seqlens.shape[0] != q.shape[0]:
+        raise ValueError("cache_seqlens must have B entries")
+    if (block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != q.shape[0]
+            or block_table.stride(1) != 1):
+        raise ValueError("block_table must be an int32 [B, max_blocks_per_seq] tensor with unit column stride")
+    out, lse = _outputs(q, v_pages.shape[3], out, lse, return_lse)
+    mb = block_table.shape[1]
+    with torch.cuda.device(dev):
+        nbytes = paged_workspace_size(q, k_pages, v_pages, mb, num_splits)
+        ws, ws_bytes = _workspace(nbytes, dev, workspace)
+        _check(lib.fa_decode_kvcache_paged(
+            _desc(q, "q"), _desc(k_pages, "k_pages"), _desc(v_pages, "v_pages"),
+            ctypes.c_void_p(block_table.data_ptr()), int(block_table.stride(0)), int(mb),
+            ctypes.c_void_p(cache_seqlens.data_ptr()), _desc(out, "o"),
+            ctypes.c_void_p(lse.data_ptr() if lse is not None else None), int(num_splits), int(bool(causal)),
+            float(scale or 0.0), ctypes.c_void_p(ws.data_ptr() if ws is not None else None), ws_bytes,
+            _stream_ptr(q)))
+    return out, lse
+
+
 def flash_attn_func(q, k, v, causal=False, softmax_scale=None, return_lse=False):
     o, lse = fa_fwd(q, k, v, causal=causal, scale=softmax_scale, return_lse=return_lse)
     return (o, lse) if return_lse else o
 
 
 def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, causal=False, softmax_scale=None,
-                            num_splits=0, return_softmax_lse=False):
-    o, lse = fa_decode_kvcache(q, k_cache, v_cache, cache_seqlens, causal=causal, scale=softmax_scale,
-                               num_splits=num_splits, return_lse=return_softmax_lse)
+                            num_splits=0, return_softmax_lse=False, block_table=None):
+    """Dense cache ([B, Lmax, Hkv, D]) or, with block_table, a paged one
+    ([num_blocks, page, Hkv, D])."""
+    if block_table is None:
+        o, lse = fa_decode_kvcache(q, k_cache, v_cache, cache_seqlens, causal=causal, scale=softmax_scale,
+                                   num_splits=num_splits, return_lse=return_softmax_lse)
+    else:
+        o, lse = fa_decode_kvcache_paged(q, k_cache, v_cache, block_table, cache_seqlens, causal=causal,
+                                         scale=softmax_scale, num_splits=num_splits,
+                                         return_lse=return_softmax_lse)
     return (o, lse) if return_softmax_lse else o
 
 

@@ -14,6 +14,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -156,8 +157,18 @@ struct Shapes {
     int B, Lq, Hq, Lk, Hkv, Dqk, Dv, g, R, RB, BR;
 };
 
+// Paged K/V: K and V are [num_blocks, page, Hkv, D]; batch b's key j is row
+// j % page of block block_table[b * bt_stride + j / page].
+struct Paging {
+    const int32_t *block_table;
+    int64_t bt_stride;
+    int max_pages;
+    int page;
+    int num_blocks;
+};
+
 fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *o,
-                       Shapes *s) {
+                       Shapes *s, const Paging *pg = nullptr) {
     fa_status st;
     if ((st = check_tensor(q, "q")) || (st = check_tensor(k, "k")) || (st = check_tensor(v, "v")))
         return st;
@@ -172,11 +183,30 @@ fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
     s->Lk = (int)k->shape[1];
     s->Hkv = (int)k->shape[2];
     s->Dv = (int)v->shape[3];
-    if (k->shape[0] != s->B || v->shape[0] != s->B)
+    if (pg) {
+        // k, v: [num_blocks, page, Hkv, D]; the key capacity of a batch is
+        // max_pages * page
+        if (v->shape[0] != k->shape[0])
+            return fail(FA_ERR_INVALID_ARG, "k_pages and v_pages must have the same number of blocks");
+        if (k->shape[0] < 1 || k->shape[0] > INT32_MAX - 1)
+            return fail(FA_ERR_INVALID_ARG, "num_blocks must be in [1, 2^31 - 2]");
+        const int64_t page = k->shape[1];
+        if (page < 16 || page > (1 << 20) || (page & (page - 1)))
+            return fail(FA_ERR_UNSUPPORTED, "page size %lld: a power of two from 16 to 2^20 is required",
+                        (long long)page);
+        if (pg->max_pages < 1) return fail(FA_ERR_INVALID_ARG, "max_blocks_per_seq must be positive");
+        if (pg->bt_stride < pg->max_pages)
+            return fail(FA_ERR_INVALID_ARG, "block_table_stride (%lld) < max_blocks_per_seq (%d)",
+                        (long long)pg->bt_stride, pg->max_pages);
+        if ((int64_t)pg->max_pages * page > INT32_MAX / 2)
+            return fail(FA_ERR_UNSUPPORTED, "max_blocks_per_seq * page too large");
+        s->Lk = (int)((int64_t)pg->max_pages * page);
+    } else if (k->shape[0] != s->B || v->shape[0] != s->B) {
         return fail(FA_ERR_INVALID_ARG, "batch mismatch: q %d, k %lld, v %lld", s->B, (long long)k->shape[0],
                     (long long)v->shape[0]);
+    }
     if (k->shape[3] != s->Dqk) return fail(FA_ERR_INVALID_ARG, "k head dim %lld != q head dim %d", (long long)k->shape[3], s->Dqk);
-    if (v->shape[1] != s->Lk || v->shape[2] != s->Hkv)
+    if (v->shape[1] != k->shape[1] || v->shape[2] != s->Hkv)
         return fail(FA_ERR_INVALID_ARG, "v must be [B, Lk, Hkv, Dv] matching k");
     if (o && (o->shape[0] != s->B || o->shape[1] != s->Lq || o->shape[2] != s->Hq || o->shape[3] != s->Dv))
         return fail(FA_ERR_INVALID_ARG, "o must be [B, Lq, Hq, Dv]");
@@ -343,7 +373,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [B, L, H, D] tensor as a 4-D TMA map {D, L, H, B}; box = 64 elements x TK
 // rows of one head of one batch, 128-byte swizzle, zero fill out of bounds.
-fa_status encode_kv_map(const fa_tensor *t, int TK, CUtensorMap *map, const char *name) {
+fa_status encode_kv_map(const fa_tensor *t, int box_rows, CUtensorMap *map, const char *name) {
     auto fn = encode_fn();
     if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const int64_t elt = 2;
@@ -358,7 +388,7 @@ fa_status encode_kv_map(const fa_tensor *t, int TK, CUtensorMap *map, const char
         if (st[i] % 8) st[i] = (st[i] + 7) / 8 * 8;
     }
     cuuint64_t strides[3] = {(cuuint64_t)(st[0] * elt), (cuuint64_t)(st[1] * elt), (cuuint64_t)(st[2] * elt)};
-    cuuint32_t box[4] = {64, (cuuint32_t)TK, 1, 1};
+    cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUtensorMapDataType dt = t->dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     // L2 promotion: fetch whole 256-byte (or 128-byte) lines only when every
@@ -403,7 +433,7 @@ fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
 // ------------------------------------------------------------ the call
 fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
               const int32_t *seqlens, float *lse, int causal, float scale, int num_splits, void *workspace,
-              size_t workspace_bytes, cudaStream_t stream) {
+              size_t workspace_bytes, cudaStream_t stream, const Paging *pg = nullptr) {
     if (s.B == 0 || s.Lq == 0) {
         t_disp = {};
         return FA_OK;
@@ -453,6 +483,13 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.min_share = pl.min_share;
     p.tile_keys = pl.main.tile_keys;
     p.tile_shift = log2_exact(pl.main.tile_keys);
+    if (pg) {
+        p.block_table = pg->block_table;
+        p.bt_stride = pg->bt_stride;
+        p.max_pages = pg->max_pages;
+        p.page_shift = log2_exact((int)k->shape[1]);
+        p.num_blocks = (int)k->shape[0];
+    }
 
     bool prof = false;
     ProfRec *rec = nullptr;
@@ -475,8 +512,9 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     const bool launch_main = pl.P > 0;
     if (launch_main) {
         CUtensorMap tmK, tmV;
-        if ((st = encode_kv_map(k, pl.main.tile_keys, &tmK, "k"))) return st;
-        if ((st = encode_kv_map(v, pl.main.tile_keys, &tmV, "v"))) return st;
+        const int box_rows = pg ? (int)std::min<int64_t>(k->shape[1], pl.main.tile_keys) : pl.main.tile_keys;
+        if ((st = encode_kv_map(k, box_rows, &tmK, "k"))) return st;
+        if ((st = encode_kv_map(v, box_rows, &tmV, "v"))) return st;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)pl.P);
         cfg.blockDim = dim3((unsigned)pl.main.threads);
@@ -594,6 +632,42 @@ fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *
     if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes: null pointer");
     Shapes s;
     fa_status st = check_shapes(q, k_cache, v_cache, nullptr, &s);
+    if (st) return st;
+    if (s.B == 0 || s.Lq == 0) {
+        *bytes = 0;
+        return FA_OK;
+    }
+    Plan pl;
+    if ((st = make_plan(s, 0, num_splits, true, s.Lk, &pl))) return st;
+    *bytes = pl.ws_bytes;
+    return FA_OK;
+}
+
+fa_status fa_decode_kvcache_paged(const fa_tensor *q, const fa_tensor *k_pages, const fa_tensor *v_pages,
+                                  const int32_t *block_table, int64_t block_table_stride, int max_blocks_per_seq,
+                                  const int32_t *cache_seqlens, fa_tensor *o, float *lse, int num_splits, int causal,
+                                  float scale, void *workspace, size_t workspace_bytes, void *stream) {
+    const Paging pg = {block_table, block_table_stride, max_blocks_per_seq, 0, 0};
+    Shapes s;
+    fa_status st = check_shapes(q, k_pages, v_pages, o, &s, &pg);
+    if (st) return st;
+    if (!o) return fail(FA_ERR_INVALID_ARG, "o: null descriptor");
+    if (s.B > 0 && !cache_seqlens) return fail(FA_ERR_INVALID_ARG, "cache_seqlens: null pointer");
+    if (s.B > 0 && !block_table) return fail(FA_ERR_INVALID_ARG, "block_table: null pointer");
+    if ((reinterpret_cast<uintptr_t>(cache_seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
+        return fail(FA_ERR_INVALID_ARG, "cache_seqlens and block_table must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+    return run(s, q, k_pages, v_pages, o, cache_seqlens, lse, causal, scale, num_splits, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream), &pg);
+}
+
+fa_status fa_decode_kvcache_paged_workspace_size(const fa_tensor *q, const fa_tensor *k_pages,
+                                                 const fa_tensor *v_pages, int max_blocks_per_seq, int num_splits,
+                                                 size_t *bytes) {
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes: null pointer");
+    const Paging pg = {nullptr, max_blocks_per_seq, max_blocks_per_seq, 0, 0};
+    Shapes s;
+    fa_status st = check_shapes(q, k_pages, v_pages, nullptr, &s, &pg);
     if (st) return st;
     if (s.B == 0 || s.Lq == 0) {
         *bytes = 0;

@@ -38,6 +38,14 @@ struct Params {
     int W_host;            // total tiles when known on the host (dense inputs), else -1
     int tile_keys;         // keys per tile (TK), a power of two
     int tile_shift;        // log2(tile_keys)
+    // Paged K/V (block_table non-null): K and V are [num_blocks, page, Hkv, D]
+    // and key j of batch b lives in block block_table[b * bt_stride + j / page]
+    // at row j % page.
+    const int *block_table;
+    int64_t bt_stride;
+    int max_pages;         // block-table entries per batch
+    int page_shift;        // log2(page)
+    int num_blocks;
 };
 
 // ------------------------------------------------------------------ schedule

@@ -58,6 +58,8 @@ template <int DQK, int DV, int STAGES, bool FMA>
 struct SplitCfg {
     static constexpr int KEYS_PER_WARP = 16 * KB;
     static constexpr int TK = KEYS_PER_WARP * kConsumerWarps;  // keys per tile
+    static constexpr int TK_SHIFT = 7;
+    static_assert((1 << TK_SHIFT) == TK, "TK is 2^TK_SHIFT");
     static constexpr int KBOX = DQK / 64;
     static constexpr int VBOX = DV / 64;
     static constexpr int BOX_BYTES = TK * 128;  // TK keys x 64 elements x 2 bytes
@@ -165,15 +167,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // (one piece per CTA: the piece's last tile is the CTA's last tile)
                 const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
                                   (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
+                const int j = tt * C::TK;
+                if (!p.block_table) {
+                    if (lane == 0) {
+                        mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+#pragma unroll
+                        for (int c = 0; c < C::KBOX; ++c)
+                            tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, j, hkv, b, policy);
+#pragma unroll
+                        for (int c = 0; c < C::VBOX; ++c)
+                            tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, j, hkv, b, policy);
+                    }
+                } else {
+                    // Paged K/V: the tile is gathered page by page.  A page of at
+                    // least TK keys gives one box of TK rows; a smaller page gives
+                    // TK / page boxes of `page` rows, stacked in the stage exactly
+                    // where one TK-row box would put them (a box of 8 or more rows
+                    // starts on a 1024-byte swizzle period).  The lanes share the
+                    // boxes; a page past the table or an invalid block number
+                    // reads as zeros (out-of-range coordinates).
+                    if (lane == 0) mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+                    __syncwarp();
+                    const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
+                    const int nsub = C::TK >> sub_shift;
+                    for (int idx = lane; idx < (C::KBOX + C::VBOX) * nsub; idx += 32) {
+                        const int c = idx / nsub, sub = idx - c * nsub;
+                        const int key = j + (sub << sub_shift);
+                        const int page = key >> p.page_shift;
+                        int blk = p.num_blocks;
+                        if (page < p.max_pages) {
+                            const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
+                            if (e >= 0 && e < p.num_blocks) blk = e;
+                        }
+                        const int row = key & ((1 << p.page_shift) - 1);
+                        const uint32_t off = (uint32_t)(sub << sub_shift) * 128u;
+                        if (c < C::KBOX)
+                            tma_load_4d(kdst + c * C::BOX_BYTES + off, &tmK, full_bar(s), c * 64, row, hkv, blk, policy);
+                        else
+                            tma_load_4d(vdst + (c - C::KBOX) * C::BOX_BYTES + off, &tmV, full_bar(s), (c - C::KBOX) * 64,
+                                        row, hkv, blk, policy);
+                    }
+                }
                 if (lane == 0) {
-                    mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
-                    const int j = tt * C::TK;
-#pragma unroll
-                    for (int c = 0; c < C::KBOX; ++c)
-                        tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, j, hkv, b, policy);
-#pragma unroll
-                    for (int c = 0; c < C::VBOX; ++c)
-                        tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, j, hkv, b, policy);
                     StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
                     meta[s] = m;
                 }

@@ -36,6 +36,7 @@ class Workload:
     seqlen_lo: int = 0        # kvcache: lengths uniform in [seqlen_lo, seqlen_hi]
     seqlen_hi: int = 0
     description: str = ""
+    page: int = 0             # "paged": keys per cache block
 
     @property
     def g(self) -> int:
@@ -64,6 +65,16 @@ WORKLOADS = {
         Dqk=192, Dv=128, causal=True, seed=1005,
         description="MLA-shaped small-Q bf16 B8 qLen8 H128 Dqk192 Dv128 kvLen16384, causal"),
 }
+
+# Paged variants of the batched decode (not one of the five pages' shapes: the
+# same GQA decode over a block-table cache, vLLM's usual 16-key pages and
+# FlashAttention's 256-key pages).
+for _pg in (16, 256):
+    WORKLOADS[f"gqa_paged{_pg}_bf16"] = Workload(
+        f"gqa_paged{_pg}_bf16", "paged", "blhd", torch.bfloat16, B=64, Lq=1, Hq=32, Hkv=8, Lk=16384,
+        Dqk=128, Dv=128, causal=False, seed=1004, seqlen_lo=1, seqlen_hi=16384, page=_pg,
+        description=f"batched GQA decode, paged cache ({_pg}-key blocks, shuffled) bf16 B64 Hq32 Hkv8 "
+                    f"D128, seqlens U[1,16384]")
 
 # the workload the bench reports by default (single-row decode over a 4K context)
 DEFAULT_BENCH = "decode_hld_fp16"
@@ -106,8 +117,50 @@ def make_inputs(w: Workload, device="cuda", seed: int | None = None, **over):
         q = _randn((w.B, w.Lq, w.Hq, w.Dqk), gen, dev, w.dtype)
         k = _randn((w.B, w.Lk, w.Hkv, w.Dqk), gen, dev, w.dtype)
         v = _randn((w.B, w.Lk, w.Hkv, w.Dv), gen, dev, w.dtype)
+    if w.call == "paged":
+        raise ValueError("paged workloads are drawn by make_paged_inputs")
     seqlens = draw_seqlens(w, seed) if w.call == "kvcache" else None
     return q, k, v, seqlens
+
+
+def make_paged_inputs(w: Workload, device="cuda", seed: int | None = None, poison: bool = False, **over):
+    """Draw (q, k_pages, v_pages, block_table, seqlens) for a paged workload.
+
+    Each batch gets ceil(seqlens[b] / page) blocks from one pool of
+    sum_b ceil(seqlens[b] / page) + 8 blocks, assigned in a seeded random
+    order; table entries past a batch's blocks are -1.  K/V values are
+    i.i.d. N(0, 1) like the dense workloads; with poison=True the pool's
+    rows that no key addresses hold NaN.  block_table is an int32 device
+    tensor [B, ceil(Lk / page)], seqlens an int32 CPU tensor."""
+    if over:
+        w = dataclasses.replace(w, **over)
+    if w.page <= 0:
+        raise ValueError("not a paged workload")
+    seed = w.seed if seed is None else seed
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    sl = draw_seqlens(w, seed)
+    mb = -(-w.Lk // w.page)
+    used = [-(-int(n) // w.page) for n in sl]
+    nb = sum(used) + 8
+    order = torch.randperm(nb, generator=torch.Generator().manual_seed(seed + 1))
+    table = torch.full((w.B, mb), -1, dtype=torch.int32)
+    pos = 0
+    for b in range(w.B):
+        table[b, :used[b]] = order[pos:pos + used[b]].to(torch.int32)
+        pos += used[b]
+    q = _randn((w.B, w.Lq, w.Hq, w.Dqk), gen, dev, w.dtype)
+    kp = _randn((nb, w.page, w.Hkv, w.Dqk), gen, dev, w.dtype)
+    vp = _randn((nb, w.page, w.Hkv, w.Dv), gen, dev, w.dtype)
+    if poison:
+        live = torch.zeros(nb, w.page, dtype=torch.bool)
+        for b in range(w.B):
+            for j0 in range(0, int(sl[b]), w.page):
+                live[int(table[b, j0 // w.page]), :min(w.page, int(sl[b]) - j0)] = True
+        dead = (~live).to(dev)
+        kp[dead] = float("nan")
+        vp[dead] = float("nan")
+    return q, kp, vp, table.to(dev), sl
 
 
 def empty_output(w: Workload, q: torch.Tensor) -> torch.Tensor:
@@ -121,7 +174,7 @@ def kv_bytes(w: Workload, seqlens=None) -> int:
     """Algorithmic K/V bytes of one call: every key row a batch attends to
     (cache_seqlens[b] rows, or Lk) is read once for K (Dqk) and once for V (Dv)."""
     elt = 2
-    if w.call == "kvcache":
+    if w.call in ("kvcache", "paged"):
         total = int(torch.as_tensor(seqlens).to(torch.int64).sum())
     else:
         total = w.B * w.Lk

@@ -135,6 +135,40 @@ FA_API fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_t
                                            size_t *bytes);
 
 /*
+ * fa_decode_kvcache_paged -- fa_decode_kvcache over a paged K/V cache.
+ *
+ * The M1 kernel of the MXFlashAttn README is a "split-KV paged decode"
+ * kernel, and the README's capability table ("能力矩阵", the dense / varlen /
+ * paged KV cache row) lists paged KV caches as implemented.  The pages do not
+ * spell out the page layout; this call takes the FlashAttention block-table
+ * convention that the README's flash_attn_with_kvcache interface implies:
+ *   k_pages  [num_blocks, page, Hkv, Dqk], v_pages [num_blocks, page, Hkv, Dv]
+ *            (fa_tensor, shape[0] = num_blocks, shape[1] = page: a power of
+ *            two from 16 to 2^20; last dim contiguous, 16-byte aligned);
+ *   block_table  DEVICE int32, batch b's entries at
+ *            block_table[b * block_table_stride + i], i < max_blocks_per_seq;
+ *   key j of batch b (j < cache_seqlens[b]) is row j % page of block
+ *   block_table[b * block_table_stride + j / page].
+ * Everything else (q, o, lse, causal, scale, num_splits, workspace, stream)
+ * is as for fa_decode_kvcache; cache_seqlens[b] is clamped to
+ * [0, max_blocks_per_seq * page].  Blocks may be shared or in any order.
+ * Table entries for pages past a batch's length are never used for values
+ * (they may hold anything); an entry outside [0, num_blocks) inside the
+ * length reads as zeros.  The caller owns every buffer; nothing is allocated
+ * and nothing is synchronised.
+ */
+FA_API fa_status fa_decode_kvcache_paged(const fa_tensor *q, const fa_tensor *k_pages, const fa_tensor *v_pages,
+                                         const int32_t *block_table, int64_t block_table_stride,
+                                         int max_blocks_per_seq, const int32_t *cache_seqlens, fa_tensor *o,
+                                         float *lse, int num_splits, int causal, float scale, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace fa_decode_kvcache_paged needs for these shapes on the current device. */
+FA_API fa_status fa_decode_kvcache_paged_workspace_size(const fa_tensor *q, const fa_tensor *k_pages,
+                                                        const fa_tensor *v_pages, int max_blocks_per_seq,
+                                                        int num_splits, size_t *bytes);
+
+/*
  * fa_decode_kvcache_noalloc -- fa_decode_kvcache for callers that cannot
  * allocate device memory (for example a plugin inside a serving runtime that
  * owns all device memory and forbids allocation after start-up, or a decode

@@ -168,3 +168,44 @@ def attention(q, k, v, *, causal: bool = False, scale: float | None = None, seql
         o = o.reshape(B, Hq, Lq, Dv).transpose(0, 2, 1, 3).copy()
         lse = lse.reshape(B, Hq, Lq)
     return o, lse
+
+
+def gather_pages(pages, block_table, seqlens):
+    """Paged cache -> dense cache.
+
+    pages: CPU torch tensor [num_blocks, page, H, D]; block_table: int array
+    [B, max_blocks]; seqlens: int [B].  Returns a dense [B, max_blocks * page,
+    H, D] tensor (same dtype, values copied unchanged) whose row j of batch b
+    (j < seqlens[b]) is row j % page of block block_table[b, j // page] -- the
+    block-table addressing of a paged K/V cache (FlashAttention's
+    ``block_table`` convention, which the MXFlashAttn README's
+    ``flash_attn_with_kvcache`` interface follows).  Rows at or past
+    seqlens[b] are zero and never visible to the definition.
+    """
+    import torch  # a container and an index-copy primitive only
+
+    bt = np.asarray(block_table, dtype=np.int64)
+    sl = np.asarray(seqlens, dtype=np.int64).reshape(-1)
+    nb, page, H, D = (int(s) for s in pages.shape)
+    B, mb = bt.shape
+    out = torch.zeros((B, mb * page, H, D), dtype=pages.dtype)
+    for b in range(B):
+        n = int(min(max(sl[b], 0), mb * page))
+        if n == 0:
+            continue
+        j = np.arange(n)
+        blk = bt[b, j // page]
+        if (blk < 0).any() or (blk >= nb).any():
+            raise ValueError("block_table entry outside [0, num_blocks) within a sequence")
+        out[b, :n] = pages[torch.from_numpy(blk), torch.from_numpy(j % page)]
+    return out
+
+
+def attention_paged(q, k_pages, v_pages, block_table, seqlens, *, causal: bool = False,
+                    scale: float | None = None, rows=None, nthreads: int | None = None):
+    """The definition over a paged K/V cache: gather_pages, then ``attention``
+    with the cache lengths (keys past seqlens[b] are not present)."""
+    k = gather_pages(k_pages, block_table, seqlens)
+    v = gather_pages(v_pages, block_table, seqlens)
+    sl = np.minimum(np.asarray(seqlens, dtype=np.int64).reshape(-1), k.shape[1]).clip(min=0)
+    return attention(q, k, v, causal=causal, scale=scale, seqlens=sl, rows=rows, nthreads=nthreads)
