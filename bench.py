@@ -208,15 +208,25 @@ def recorded_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
-def cpu_baseline(w, q, k, v, seqlens, seconds: float):
+def cpu_baseline(w, ins, seqlens, seconds: float):
     """The fp64 oracle as it stands, on this host's cores, over a bounded
-    sample of the workload's rows; throughput scaled to the same metric."""
+    sample of the workload's rows; throughput scaled to the same metric.
+    ins: (q, k, v) or, for a paged cache, (q, k_pages, v_pages, block_table);
+    a paged cache is gathered into its dense form once, untimed, and the
+    definition is timed on it."""
     import numpy as np
 
     import oracle
     from decode_flashattention_b200 import workloads as wl
 
     oracle.build()
+    q = ins[0]
+    if w.call == "paged":
+        bt = ins[3].cpu().numpy()
+        k = oracle.gather_pages(ins[1].cpu(), bt, seqlens.numpy())
+        v = oracle.gather_pages(ins[2].cpu(), bt, seqlens.numpy())
+    else:
+        k, v = ins[1], ins[2]
     cores = os.cpu_count() or 1
     rows_total = w.B * w.Hq * w.Lq
     qc, kc, vc = q.cpu(), None, None
@@ -258,31 +268,42 @@ def run_ours(args):
     fa.force_variant({"auto": fa.VARIANT_AUTO, "mma": fa.VARIANT_MMA, "scalar": fa.VARIANT_SCALAR}[args.variant])
     name = args.workload or wl.DEFAULT_BENCH
     w = workload_of(args)
-    q0, k0, v0, sl0 = wl.make_inputs(w, device, seed=w.seed + 1000 * rank)
-    per_copy = wl.kv_bytes(w, sl0) + q0.numel() * 2
+    def draw(seed):
+        # (inputs of one call, cache lengths): dense q, k, v or paged q, k_pages, v_pages, block_table
+        if w.call == "paged":
+            q, kp, vp, bt, sl = wl.make_paged_inputs(w, device, seed=seed)
+            return (q, kp, vp, bt), sl
+        q, k, v, sl = wl.make_inputs(w, device, seed=seed)
+        return (q, k, v), sl
+
+    ins0, sl0 = draw(w.seed + 1000 * rank)
+    q0 = ins0[0]
+    per_copy = sum(t.numel() * t.element_size() for t in ins0)
     n_copies = max(1, math.ceil(4 * L2_BYTES / max(per_copy, 1)))
-    copies = [(q0, k0, v0)]
-    for c in range(1, n_copies):
-        q, k, v, _ = wl.make_inputs(w, device, seed=w.seed + 1000 * rank + c)
-        copies.append((q, k, v))
+    copies = [ins0] + [draw(w.seed + 1000 * rank + c)[0] for c in range(1, n_copies)]
     sl_dev = sl0.to(device) if sl0 is not None else None
     outs = [wl.empty_output(w, q0) for _ in range(n_copies)]
     lses = [torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device) for _ in range(n_copies)]
-    if w.call == "kvcache":
-        ws_bytes = fa.kvcache_workspace_size(q0, k0, v0, args.num_splits)
+    if w.call == "paged":
+        ws_bytes = fa.paged_workspace_size(q0, ins0[1], ins0[2], ins0[3].shape[1], args.num_splits)
+    elif w.call == "kvcache":
+        ws_bytes = fa.kvcache_workspace_size(*ins0, args.num_splits)
     else:
-        ws_bytes = fa.fwd_workspace_size(q0, k0, v0, w.causal, args.num_splits)
+        ws_bytes = fa.fwd_workspace_size(*ins0, w.causal, args.num_splits)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
     bytes_per_step = wl.kv_bytes(w, sl0)
 
-    def step(i):
-        q, k, v = copies[i % n_copies]
-        o, l = outs[i % n_copies], lses[i % n_copies]
+    def call(ins, sl, o, l):
+        if w.call == "paged":
+            return fa.fa_decode_kvcache_paged(*ins, sl, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
+                                              workspace=ws)
         if w.call == "kvcache":
-            fa.fa_decode_kvcache(q, k, v, sl_dev, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
-                                 workspace=ws)
-        else:
-            fa.fa_fwd(q, k, v, causal=w.causal, num_splits=args.num_splits, out=o, lse=l, workspace=ws)
+            return fa.fa_decode_kvcache(*ins, sl, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
+                                        workspace=ws)
+        return fa.fa_fwd(*ins, causal=w.causal, num_splits=args.num_splits, out=o, lse=l, workspace=ws)
+
+    def step(i):
+        call(copies[i % n_copies], sl_dev, outs[i % n_copies], lses[i % n_copies])
 
     stream = torch.cuda.current_stream(device)
     for i in range(max(args.warmup, 3)):
@@ -368,30 +389,22 @@ def run_ours(args):
     fa.check_status()
 
     # --- e2e: through the public API from pinned host buffers -------------------------
-    hq = q0.cpu().pin_memory()
-    hk = k0.cpu().pin_memory()
-    hv = v0.cpu().pin_memory()
+    hins = [t.cpu().pin_memory() for t in ins0]
     hsl = sl0.pin_memory() if sl0 is not None else None
     ho = torch.empty(outs[0].shape, dtype=w.dtype).pin_memory()
     hl = torch.empty(lses[0].shape, dtype=torch.float32).pin_memory()
-    dq, dk, dv = torch.empty_like(q0), torch.empty_like(k0), torch.empty_like(v0)
+    dins = [torch.empty_like(t) for t in ins0]
     dsl = torch.empty_like(sl_dev) if sl_dev is not None else None
-    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + (hsl.numel() * 4 if hsl is not None else 0)
+    h2d = sum(t.numel() * t.element_size() for t in hins) + (hsl.numel() * 4 if hsl is not None else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
     E = max(1, args.e2e_steps)
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
+        for d, h in zip(dins, hins):
+            d.copy_(h, non_blocking=True)
         if dsl is not None:
             dsl.copy_(hsl, non_blocking=True)
-        if w.call == "kvcache":
-            o, l = fa.fa_decode_kvcache(dq, dk, dv, dsl, causal=w.causal, num_splits=args.num_splits,
-                                        out=outs[0], lse=lses[0], workspace=ws)
-        else:
-            o, l = fa.fa_fwd(dq, dk, dv, causal=w.causal, num_splits=args.num_splits, out=outs[0],
-                             lse=lses[0], workspace=ws)
+        o, l = call(dins, dsl, outs[0], lses[0])
         ho.copy_(o, non_blocking=True)
         hl.copy_(l, non_blocking=True)
 
@@ -476,7 +489,7 @@ def run_ours(args):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
-    res["cpu_baseline"] = cpu_baseline(w, q0, k0, v0, sl0, args.cpu_seconds) if world == 1 else None
+    res["cpu_baseline"] = cpu_baseline(w, ins0, sl0, args.cpu_seconds) if world == 1 else None
     print(json.dumps(res), flush=True)
 
 
@@ -492,15 +505,20 @@ def run_reference(args):
 
     name = args.workload or wl.DEFAULT_BENCH
     w = workload_of(args)
-    q, k, v, sl = wl.make_inputs(w, "cpu")
+    if w.call == "paged":
+        q, kp, vp, bt, sl = wl.make_paged_inputs(w, "cpu")
+        ins = (q, kp, vp, bt)
+    else:
+        q, k, v, sl = wl.make_inputs(w, "cpu")
+        ins = (q, k, v)
     W = max(args.warmup, 3)
     K = args.steps if args.steps > 0 else 3
     per_step = max(1.0, min(args.cpu_seconds, 60.0 / max(K + W, 1)))
     for _ in range(min(W, 1)):
-        cpu_baseline(w, q, k, v, sl, per_step / 4)
+        cpu_baseline(w, ins, sl, per_step / 4)
     vals, secs = [], 0.0
     for _ in range(K):
-        r = cpu_baseline(w, q, k, v, sl, per_step)
+        r = cpu_baseline(w, ins, sl, per_step)
         vals.append(r["value"])
         secs += r["seconds"]
     value = sum(vals) / len(vals)

@@ -83,6 +83,9 @@ struct SplitCfg {
     static_assert(DQK % 64 == 0 && DV % 64 == 0, "head dims are multiples of 64");
     static_assert(OFF_QF % 16 == 0 && OFF_RED % 16 == 0 && OFF_BAR % 8 == 0, "aligned regions");
     static_assert(SMEM <= 232448, "fits the 227 KB per-CTA shared memory limit");
+    // paged K/V: pages of >= 16 keys give at most TK / 16 boxes per column
+    // chunk; the producer's lanes loop over them
+    static_assert((KBOX + VBOX) * (TK / 16) <= 64, "paged boxes per tile: at most two per lane");
 };
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
