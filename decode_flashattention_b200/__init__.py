@@ -27,6 +27,7 @@ import torch
 
 __all__ = [
     "FaError", "fa_fwd", "fa_decode_kvcache", "fa_decode_kvcache_paged", "paged_workspace_size",
+    "fa_decode_kvcache_append",
     "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
     "last_dispatch", "force_variant", "profile_enable", "profile_read", "launch_count",
@@ -83,6 +84,8 @@ def load_library():
         "fa_decode_kvcache_workspace_size": (i32, [T, T, T, i32, P(sz)]),
         "fa_decode_kvcache_paged": (i32, [T, T, T, vp, ctypes.c_int64, i32, vp, T, vp, i32, i32, f32, vp, sz, vp]),
         "fa_decode_kvcache_paged_workspace_size": (i32, [T, T, T, i32, i32, P(sz)]),
+        "fa_decode_kvcache_append": (i32, [T, T, T, T, T, vp, ctypes.c_int64, i32, vp, T, vp, i32, i32, f32, vp,
+                                           sz, vp]),
         "fa_check_status": (i32, [vp]),
         "fa_last_error": (ctypes.c_char_p, []),
         "fa_last_dispatch": (None, [P(FaDispatchInfo)]),
@@ -268,16 +271,59 @@ def fa_decode_kvcache_paged(q, k_pages, v_pages, block_table, cache_seqlens, cau
     return out, lse
 
 
+def fa_decode_kvcache_append(q, k_new, v_new, k_cache, v_cache, cache_seqlens, block_table=None, causal=False,
+                             scale=None, num_splits=0, out=None, lse=None, workspace=None, return_lse=True):
+    """Write k_new / v_new [B, Lnew, Hkv, D] into the cache at positions
+    cache_seqlens[b] + t (dense k_cache [B, Lmax, Hkv, D], or paged
+    [num_blocks, page, Hkv, D] with block_table), then attend over
+    cache_seqlens[b] + Lnew keys.  cache_seqlens is not modified."""
+    lib = load_library()
+    dev = _cuda_inputs(q, k_new, v_new, k_cache, v_cache, cache_seqlens)
+    if cache_seqlens.dtype != torch.int32 or cache_seqlens.dim() != 1 or not cache_seqlens.is_contiguous():
+        raise ValueError("cache_seqlens must be a contiguous int32 [B] tensor")
+    if cache_seqlens.shape[0] != q.shape[0]:
+        raise ValueError("cache_seqlens must have B entries")
+    if block_table is not None:
+        if (block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != q.shape[0]
+                or block_table.stride(1) != 1 or block_table.device != dev):
+            raise ValueError("block_table must be a CUDA int32 [B, max_blocks_per_seq] tensor, unit column stride")
+        mb, bts, btp = block_table.shape[1], block_table.stride(0), block_table.data_ptr()
+    else:
+        mb, bts, btp = 0, 0, None
+    out, lse = _outputs(q, v_cache.shape[3], out, lse, return_lse)
+    with torch.cuda.device(dev):
+        if block_table is not None:
+            nbytes = paged_workspace_size(q, k_cache, v_cache, mb, num_splits)
+        else:
+            nbytes = kvcache_workspace_size(q, k_cache, v_cache, num_splits)
+        ws, ws_bytes = _workspace(nbytes, dev, workspace)
+        _check(lib.fa_decode_kvcache_append(
+            _desc(q, "q"), _desc(k_new, "k_new"), _desc(v_new, "v_new"), _desc(k_cache, "k_cache"),
+            _desc(v_cache, "v_cache"), ctypes.c_void_p(btp), int(bts), int(mb),
+            ctypes.c_void_p(cache_seqlens.data_ptr()), _desc(out, "o"),
+            ctypes.c_void_p(lse.data_ptr() if lse is not None else None), int(num_splits), int(bool(causal)),
+            float(scale or 0.0), ctypes.c_void_p(ws.data_ptr() if ws is not None else None), ws_bytes,
+            _stream_ptr(q)))
+    return out, lse
+
+
 def flash_attn_func(q, k, v, causal=False, softmax_scale=None, return_lse=False):
     o, lse = fa_fwd(q, k, v, causal=causal, scale=softmax_scale, return_lse=return_lse)
     return (o, lse) if return_lse else o
 
 
 def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, causal=False, softmax_scale=None,
-                            num_splits=0, return_softmax_lse=False, block_table=None):
+                            num_splits=0, return_softmax_lse=False, block_table=None, k=None, v=None):
     """Dense cache ([B, Lmax, Hkv, D]) or, with block_table, a paged one
-    ([num_blocks, page, Hkv, D])."""
-    if block_table is None:
+    ([num_blocks, page, Hkv, D]); with k / v ([B, Lnew, Hkv, D]) those tokens
+    are appended to the cache first."""
+    if k is not None or v is not None:
+        if k is None or v is None:
+            raise ValueError("k and v are appended together")
+        o, lse = fa_decode_kvcache_append(q, k, v, k_cache, v_cache, cache_seqlens, block_table=block_table,
+                                          causal=causal, scale=softmax_scale, num_splits=num_splits,
+                                          return_lse=return_softmax_lse)
+    elif block_table is None:
         o, lse = fa_decode_kvcache(q, k_cache, v_cache, cache_seqlens, causal=causal, scale=softmax_scale,
                                    num_splits=num_splits, return_lse=return_softmax_lse)
     else:

@@ -433,7 +433,8 @@ fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
 // ------------------------------------------------------------ the call
 fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
               const int32_t *seqlens, float *lse, int causal, float scale, int num_splits, void *workspace,
-              size_t workspace_bytes, cudaStream_t stream, const Paging *pg = nullptr) {
+              size_t workspace_bytes, cudaStream_t stream, const Paging *pg = nullptr,
+              const fa::AppendParams *ap = nullptr) {
     if (s.B == 0 || s.Lq == 0) {
         t_disp = {};
         return FA_OK;
@@ -489,6 +490,32 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         p.max_pages = pg->max_pages;
         p.page_shift = log2_exact((int)k->shape[1]);
         p.num_blocks = (int)k->shape[0];
+    }
+
+    if (ap) {
+        // KV append first: the split-KV kernel then sees seqlens[b] + Lnew keys
+        p.seqlen_add = ap->Lnew;
+        fa::KernelInfo ak;
+        fa::append_kernel_info(&ak);
+        int occ = 0;
+        if ((st = prepare_fn(ak.fn, ak.threads, 0, &occ))) return st;
+        const long long rows = (long long)ap->B * ap->Lnew * ap->Hkv;
+        if (rows > 0) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)((rows + ak.threads / 32 - 1) / (ak.threads / 32)));
+            cfg.blockDim = dim3((unsigned)ak.threads);
+            cfg.stream = stream;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            at[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            fa::AppendParams a = *ap;
+            void *args[] = {&a};
+            cudaError_t e = cudaLaunchKernelExC(&cfg, ak.fn, args);
+            if (e != cudaSuccess) return cuda_fail(e, "launch of the KV append kernel");
+            g_launches.fetch_add(1);
+        }
     }
 
     bool prof = false;
@@ -677,6 +704,55 @@ fa_status fa_decode_kvcache_paged_workspace_size(const fa_tensor *q, const fa_te
     if ((st = make_plan(s, 0, num_splits, true, s.Lk, &pl))) return st;
     *bytes = pl.ws_bytes;
     return FA_OK;
+}
+
+fa_status fa_decode_kvcache_append(const fa_tensor *q, const fa_tensor *k_new, const fa_tensor *v_new,
+                                   fa_tensor *k_cache, fa_tensor *v_cache, const int32_t *block_table,
+                                   int64_t block_table_stride, int max_blocks_per_seq, const int32_t *cache_seqlens,
+                                   fa_tensor *o, float *lse, int num_splits, int causal, float scale, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    const Paging pg = {block_table, block_table_stride, max_blocks_per_seq, 0, 0};
+    Shapes s;
+    fa_status st = check_shapes(q, k_cache, v_cache, o, &s, block_table ? &pg : nullptr);
+    if (st) return st;
+    if (!o) return fail(FA_ERR_INVALID_ARG, "o: null descriptor");
+    if (s.B > 0 && !cache_seqlens) return fail(FA_ERR_INVALID_ARG, "cache_seqlens: null pointer");
+    if ((reinterpret_cast<uintptr_t>(cache_seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
+        return fail(FA_ERR_INVALID_ARG, "cache_seqlens and block_table must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+    if ((st = check_tensor(k_new, "k_new")) || (st = check_tensor(v_new, "v_new"))) return st;
+    if (k_new->dtype != q->dtype || v_new->dtype != q->dtype)
+        return fail(FA_ERR_INVALID_ARG, "k_new and v_new must have q's element type");
+    const int64_t Lnew = k_new->shape[1];
+    if (k_new->shape[0] != s.B || k_new->shape[2] != s.Hkv || k_new->shape[3] != s.Dqk || v_new->shape[0] != s.B ||
+        v_new->shape[1] != Lnew || v_new->shape[2] != s.Hkv || v_new->shape[3] != s.Dv)
+        return fail(FA_ERR_INVALID_ARG, "k_new / v_new must be [B, Lnew, Hkv, Dqk] / [B, Lnew, Hkv, Dv]");
+    if (Lnew > INT32_MAX / 4) return fail(FA_ERR_UNSUPPORTED, "Lnew too large");
+    fa::AppendParams a = {};
+    a.k_new = k_new->data;
+    a.v_new = v_new->data;
+    for (int i = 0; i < 3; ++i) {
+        a.kn[i] = k_new->stride[i];
+        a.vn[i] = v_new->stride[i];
+        a.kc[i] = k_cache->stride[i];
+        a.vc[i] = v_cache->stride[i];
+    }
+    a.k_cache = k_cache->data;
+    a.v_cache = v_cache->data;
+    a.seqlens = cache_seqlens;
+    a.block_table = block_table;
+    a.bt_stride = block_table_stride;
+    a.max_pages = max_blocks_per_seq;
+    a.page_shift = block_table ? log2_exact((int)k_cache->shape[1]) : 0;
+    a.num_blocks = block_table ? (int)k_cache->shape[0] : 0;
+    a.B = s.B;
+    a.Lnew = (int)Lnew;
+    a.Hkv = s.Hkv;
+    a.Dqk = s.Dqk;
+    a.Dv = s.Dv;
+    a.capacity = s.Lk;
+    return run(s, q, k_cache, v_cache, o, cache_seqlens, lse, causal, scale, num_splits, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream), block_table ? &pg : nullptr, &a);
 }
 
 fa_status fa_check_status(void *stream) {

@@ -46,6 +46,7 @@ struct Params {
     int max_pages;         // block-table entries per batch
     int page_shift;        // log2(page)
     int num_blocks;
+    int seqlen_add;        // tokens appended to every cache by this call (added to seqlens[b])
 };
 
 // ------------------------------------------------------------------ schedule
@@ -74,10 +75,12 @@ __host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int L
 }
 
 // Keys present for batch b: cache_seqlens[b] clamped to [0, Lk], or Lk.
-__host__ __device__ inline int batch_keys(const int *seqlens, int b, int Lk) {
+// Keys present for batch b: Lk for dense inputs, else cache_seqlens[b] plus
+// the tokens appended by this call, clamped to [0, Lk].
+__host__ __device__ inline int batch_keys(const int *seqlens, int b, int Lk, int add = 0) {
     if (!seqlens) return Lk;
-    int n = seqlens[b];
-    return n < 0 ? 0 : (n > Lk ? Lk : n);
+    const long long n = (long long)seqlens[b] + add;
+    return n < 0 ? 0 : (n > Lk ? Lk : (int)n);
 }
 
 // Tiles of tile_keys = 1 << tile_shift keys covering the visible keys.
@@ -377,7 +380,7 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16 *dst, co
 
 __device__ __forceinline__ int entry_tiles(const Params &p, int x) {
     const int b = x / p.RB, rb = x - b * p.RB;
-    return unit_tiles(batch_keys(p.seqlens, b, p.Lk), rb, p.R, p.Lq, p.causal, p.tile_shift);
+    return unit_tiles(batch_keys(p.seqlens, b, p.Lk, p.seqlen_add), rb, p.R, p.Lq, p.causal, p.tile_shift);
 }
 
 __device__ __forceinline__ int warp_sum(int v) {

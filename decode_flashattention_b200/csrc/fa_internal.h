@@ -23,6 +23,24 @@ bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 
+// KV append (fa_append.cu): new K / V rows [B, Lnew, Hkv, D] into a dense
+// cache [B, Lmax, Hkv, D] or a paged one [num_blocks, page, Hkv, D] at
+// positions cache_seqlens[b] + t.  Strides in elements ({batch or block, row,
+// head}); the last dim is contiguous.
+struct AppendParams {
+    const void *k_new, *v_new;
+    int64_t kn[3], vn[3];
+    void *k_cache, *v_cache;
+    int64_t kc[3], vc[3];
+    const int *seqlens;
+    const int *block_table;  // null for a dense cache
+    int64_t bt_stride;
+    int max_pages, page_shift, num_blocks;
+    int B, Lnew, Hkv, Dqk, Dv;
+    long long capacity;      // keys a batch's cache can hold
+};
+void append_kernel_info(KernelInfo *out);
+
 // Sets the calling thread's fa_last_error() message (for entry points that
 // live outside fa_api.cu).
 void set_last_error(const char *msg);

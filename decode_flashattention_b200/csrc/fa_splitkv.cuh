@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const T *qs = reinterpret_cast<const T *>(smem + C::OFF_Q + s * C::Q_BYTES);
                 for (int d = lane; d < DQK; d += 32) qf32[d] = Cvt<T>::f1(qs[d]);
                 __syncwarp();
-                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk);
+                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk, p.seqlen_add);
                 m = -INFINITY;
                 l = 0.f;
 #pragma unroll
@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][0]) : "r"(qrow + kk * 32));
                     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][1]) : "r"(qrow + kk * 32 + 16));
                 }
-                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk);
+                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk, p.seqlen_add);
                 // last visible key of this lane's two accumulator rows (bottom-right causal)
     #pragma unroll
                 for (int e = 0; e < 2; ++e) {

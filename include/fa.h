@@ -169,6 +169,33 @@ FA_API fa_status fa_decode_kvcache_paged_workspace_size(const fa_tensor *q, cons
                                                         int num_splits, size_t *bytes);
 
 /*
+ * fa_decode_kvcache_append -- append new tokens' K / V to the cache, then
+ * attend (the order of flash_attn_with_kvcache with new k / v, the interface
+ * the MXFlashAttn README follows; its capability table lists paged KV append
+ * among the verified cases).
+ *   k_new [B, Lnew, Hkv, Dqk], v_new [B, Lnew, Hkv, Dv]: DEVICE, q's type.
+ *   k_cache / v_cache: dense [B, Lmax, Hkv, D] when block_table is NULL,
+ *   else paged [num_blocks, page, Hkv, D] with block_table /
+ *   block_table_stride / max_blocks_per_seq as for fa_decode_kvcache_paged.
+ *   Token t of batch b is written to cache position cache_seqlens[b] + t
+ *   (dense row, or row pos % page of block block_table[b, pos / page]); a
+ *   position at or past the capacity, or an invalid block number, is not
+ *   written.  The attention then sees cache_seqlens[b] + Lnew keys (clamped
+ *   to the capacity); cache_seqlens itself is not modified.  With causal,
+ *   query i (of Lq, normally Lq = Lnew) sees keys j <= i + n - Lq.
+ * Everything else is as for fa_decode_kvcache; the workspace is the size
+ * fa_decode_kvcache_workspace_size (dense) or
+ * fa_decode_kvcache_paged_workspace_size (paged) returns.  The copy runs as
+ * its own small kernel ahead of the attention kernels, on the same stream.
+ */
+FA_API fa_status fa_decode_kvcache_append(const fa_tensor *q, const fa_tensor *k_new, const fa_tensor *v_new,
+                                          fa_tensor *k_cache, fa_tensor *v_cache, const int32_t *block_table,
+                                          int64_t block_table_stride, int max_blocks_per_seq,
+                                          const int32_t *cache_seqlens, fa_tensor *o, float *lse, int num_splits,
+                                          int causal, float scale, void *workspace, size_t workspace_bytes,
+                                          void *stream);
+
+/*
  * fa_decode_kvcache_noalloc -- fa_decode_kvcache for callers that cannot
  * allocate device memory (for example a plugin inside a serving runtime that
  * owns all device memory and forbids allocation after start-up, or a decode

@@ -209,3 +209,36 @@ def attention_paged(q, k_pages, v_pages, block_table, seqlens, *, causal: bool =
     v = gather_pages(v_pages, block_table, seqlens)
     sl = np.minimum(np.asarray(seqlens, dtype=np.int64).reshape(-1), k.shape[1]).clip(min=0)
     return attention(q, k, v, causal=causal, scale=scale, seqlens=sl, rows=rows, nthreads=nthreads)
+
+
+def append_kv(k_cache, v_cache, k_new, v_new, seqlens, block_table=None):
+    """KV append, written out: returns copies of the caches with token t of
+    batch b written at position pos = seqlens[b] + t -- dense row pos of
+    [B, Lmax, H, D], or (block_table given) row pos % page of block
+    block_table[b, pos // page] of [num_blocks, page, H, D].  A position
+    outside [0, capacity) or a block number outside [0, num_blocks) is not
+    written.  CPU torch tensors in, values copied unchanged."""
+    kc, vc = k_cache.clone(), v_cache.clone()
+    sl = np.asarray(seqlens, dtype=np.int64).reshape(-1)
+    B, Lnew = int(k_new.shape[0]), int(k_new.shape[1])
+    if block_table is None:
+        cap = int(kc.shape[1])
+    else:
+        bt = np.asarray(block_table, dtype=np.int64)
+        page = int(kc.shape[1])
+        cap = bt.shape[1] * page
+    for b in range(B):
+        for t in range(Lnew):
+            pos = int(sl[b]) + t
+            if pos < 0 or pos >= cap:
+                continue
+            if block_table is None:
+                kc[b, pos] = k_new[b, t]
+                vc[b, pos] = v_new[b, t]
+            else:
+                blk = int(bt[b, pos // page])
+                if blk < 0 or blk >= kc.shape[0]:
+                    continue
+                kc[blk, pos % page] = k_new[b, t]
+                vc[blk, pos % page] = v_new[b, t]
+    return kc, vc
