@@ -212,9 +212,10 @@ fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
         return fail(FA_ERR_INVALID_ARG, "o must be [B, Lq, Hq, Dv]");
     if (s->Hkv <= 0 || s->Hq <= 0) return fail(FA_ERR_INVALID_ARG, "head counts must be positive");
     if (s->Hq % s->Hkv) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", s->Hq, s->Hkv);
-    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128)))
-        return fail(FA_ERR_UNSUPPORTED, "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128)}", s->Dqk,
-                    s->Dv);
+    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128) ||
+          (s->Dqk == 256 && s->Dv == 256)))
+        return fail(FA_ERR_UNSUPPORTED,
+                    "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128), (256,256)}", s->Dqk, s->Dv);
     s->g = s->Hq / s->Hkv;
     int64_t R = (int64_t)s->g * s->Lq;
     if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * Lq too large");

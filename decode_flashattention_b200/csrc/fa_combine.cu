@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     // The partition and the partials' addresses are worked out before the
     // wait (dense inputs need no memory for it); cache lengths only after it.
     constexpr int EPL = DV / 32;  // elements per lane
+    constexpr int PPP = DV >= 256 ? 4 : kPartsPerPass;  // partials per pass (fewer for wide rows: registers)
     int t = 0, u0 = 0, cf = 0, nparts = 0;
     long long base0 = 0;  // this lane's partial in the first pass
     Partition pt = {0, 1};
@@ -58,7 +59,7 @@ __global__ void __launch_bounds__(kCombineThreads)
             cf = piece_of(pt, u0);
             nparts = piece_of(pt, u0 + t - 1) - cf + 1;
             const int c = cf + lane;
-            if (lane < kPartsPerPass && lane < nparts)
+            if (lane < PPP && lane < nparts)
                 base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr;
         }
     };
@@ -80,7 +81,7 @@ __global__ void __launch_bounds__(kCombineThreads)
             if (!live) return;
             if (t > 0 && nparts == 1) return;  // finished inside one piece by the split-KV kernel
         }
-        const int tu = warm ? 1 : t, np = warm ? kPartsPerPass : nparts;
+        const int tu = warm ? 1 : t, np = warm ? PPP : nparts;
         const long long b0 = warm ? 0 : base0;
         const float *ws_o = warm ? sink : p.ws_o;
         const float *ws_lse = warm ? sink : p.ws_lse;
@@ -96,25 +97,28 @@ __global__ void __launch_bounds__(kCombineThreads)
 
         if (tu > 0) {
             float M = -INFINITY, L = 0.f;
-            for (int j0 = 0; j0 < np; j0 += kPartsPerPass) {
-                // lane j < kPartsPerPass owns partial cf + j0 + j; its lse and every
+            for (int j0 = 0; j0 < np; j0 += PPP) {
+                // lane j < PPP owns partial cf + j0 + j; its lse and every
                 // lane's O slices of the pass are loaded together
                 const int c = cf + j0 + lane;
-                const bool has = lane < kPartsPerPass && j0 + lane < np;
+                const bool has = lane < PPP && j0 + lane < np;
                 const long long base =
                     j0 == 0 ? b0
                             : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr : 0);
-                const int cnt = np - j0 < kPartsPerPass ? np - j0 : kPartsPerPass;
+                const int cnt = np - j0 < PPP ? np - j0 : PPP;
                 const float ls = has ? ws_lse[base] : -INFINITY;
-                float v[kPartsPerPass][EPL];
+                float v[PPP][EPL];
 #pragma unroll
-                for (int q = 0; q < kPartsPerPass; ++q) {
+                for (int q = 0; q < PPP; ++q) {
                     const long long bq = __shfl_sync(0xffffffffu, base, q);
                     if (q < cnt) {
                         const float *src = ws_o + bq * DV + lane_off;
-                        if constexpr (EPL == 4) {
-                            const float4 x4 = *reinterpret_cast<const float4 *>(src);
-                            v[q][0] = x4.x; v[q][1] = x4.y; v[q][2] = x4.z; v[q][3] = x4.w;
+                        if constexpr (EPL % 4 == 0) {
+#pragma unroll
+                            for (int e = 0; e < EPL; e += 4) {
+                                const float4 x4 = *reinterpret_cast<const float4 *>(src + e);
+                                v[q][e] = x4.x; v[q][e + 1] = x4.y; v[q][e + 2] = x4.z; v[q][e + 3] = x4.w;
+                            }
                         } else {
                             const float2 x2 = *reinterpret_cast<const float2 *>(src);
                             v[q][0] = x2.x; v[q][1] = x2.y;
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 #pragma unroll
                 for (int e = 0; e < EPL; ++e) acc[e] *= scale_old;
 #pragma unroll
-                for (int q = 0; q < kPartsPerPass; ++q) {
+                for (int q = 0; q < PPP; ++q) {
                     const float wq = __shfl_sync(0xffffffffu, w, q);
                     if (q < cnt) {
 #pragma unroll
@@ -173,9 +177,11 @@ bool get_combine_kernel(int dtype, int dv, KernelInfo *out) {
     if (dtype == 0) {
         if (dv == 64) { fill<__half, 64>(out); return true; }
         if (dv == 128) { fill<__half, 128>(out); return true; }
+        if (dv == 256) { fill<__half, 256>(out); return true; }
     } else if (dtype == 1) {
         if (dv == 64) { fill<__nv_bfloat16, 64>(out); return true; }
         if (dv == 128) { fill<__nv_bfloat16, 128>(out); return true; }
+        if (dv == 256) { fill<__nv_bfloat16, 256>(out); return true; }
     }
     return false;
 }

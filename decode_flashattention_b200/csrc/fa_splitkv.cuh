@@ -52,13 +52,14 @@ constexpr int kMetaWhole = 4;  // the segment is the whole unit: write O / lse
 constexpr int kMetaDone = 8;   // no more work
 constexpr int kMetaFinal = 16; // the CTA's last tile
 
-constexpr int KB = 2;  // 16-key blocks per consumer warp per tile
 
-template <int DQK, int DV, int STAGES, bool FMA>
+// KB: 16-key blocks per consumer warp per tile (2: 128-key tiles; 1: 64-key
+// tiles, for head dims whose 128-key stage would not leave room for a ring).
+template <int DQK, int DV, int STAGES, bool FMA, int KB = 2>
 struct SplitCfg {
     static constexpr int KEYS_PER_WARP = 16 * KB;
     static constexpr int TK = KEYS_PER_WARP * kConsumerWarps;  // keys per tile
-    static constexpr int TK_SHIFT = 7;
+    static constexpr int TK_SHIFT = KB == 2 ? 7 : 6;
     static_assert((1 << TK_SHIFT) == TK, "TK is 2^TK_SHIFT");
     static constexpr int KBOX = DQK / 64;
     static constexpr int VBOX = DV / 64;
@@ -90,11 +91,12 @@ struct SplitCfg {
 
 constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
-template <typename T, int DQK, int DV, int STAGES, bool FMA>
+template <typename T, int DQK, int DV, int STAGES, bool FMA, int KB = 2>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_kernel(const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
-    using C = SplitCfg<DQK, DV, STAGES, FMA>;
+    using C = SplitCfg<DQK, DV, STAGES, FMA, KB>;
+    static_assert(!FMA || KB == 2, "the FMA consumer gives each lane one of 32 keys per warp");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -346,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int hq = md.hkv * p.g + rr / p.Lq, i = rr % p.Lq;
                 T *op = warm ? static_cast<T *>(sink)
                              : og + md.b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
-                if constexpr (EPT == 8) {
-                    store_row8<T>(op, v);
+                if constexpr (EPT % 8 == 0) {
+#pragma unroll
+                    for (int e = 0; e < EPT; e += 8) store_row8<T>(op + e, v + e);
                 } else {
 #pragma unroll
                     for (int e = 0; e < EPT; e += 2)

@@ -76,6 +76,12 @@ for _pg in (16, 256):
         description=f"batched GQA decode, paged cache ({_pg}-key blocks, shuffled) bf16 B64 Hq32 Hkv8 "
                     f"D128, seqlens U[1,16384]")
 
+# Head dim 256 (the SmallQ README's validation shapes include hd 256): GQA 4
+# decode over an 8K context.
+WORKLOADS["gqa_decode_hd256_bf16"] = Workload(
+    "gqa_decode_hd256_bf16", "fwd", "blhd", torch.bfloat16, B=8, Lq=1, Hq=16, Hkv=4, Lk=8192, Dqk=256, Dv=256,
+    causal=False, seed=1006, description="GQA decode bf16 B8 Hq16 Hkv4 D256 kvLen8192, non-causal")
+
 # the workload the bench reports by default (single-row decode over a 4K context)
 DEFAULT_BENCH = "decode_hld_fp16"
 

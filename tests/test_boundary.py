@@ -210,3 +210,57 @@ def test_hld_view_strides():
     v = fa.hld_as_blhd(x)
     assert tuple(v.shape) == (1, 4096, 32, 128)
     assert v.stride() == (32 * 4096 * 128, 128, 4096 * 128, 1)
+
+
+# ------------------------------------------------------------------ paged cache and KV append (host checks)
+
+def call_paged(q, kp, vp, bt=0x20000, bt_stride=4, max_blocks=4, sl=0x30000, o=None):
+    lib = fa.load_library()
+    o = o or good("o")
+    return lib.fa_decode_kvcache_paged(ctypes.byref(q), ctypes.byref(kp), ctypes.byref(vp), ctypes.c_void_p(bt),
+                                       bt_stride, max_blocks, ctypes.c_void_p(sl), ctypes.byref(o), None, 0, 0,
+                                       0.0, None, 0, None)
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("page_12", UNSUPPORTED), ("page_8", UNSUPPORTED), ("stride_lt_blocks", INVALID), ("null_table", INVALID),
+    ("null_seqlens", INVALID), ("blocks_mismatch", INVALID), ("misaligned_table", INVALID),
+])
+def test_paged_host_validation(case, expect):
+    q = good("q")
+    kp, vp = desc([10, 16, 2, 128]), desc([10, 16, 2, 128])
+    kw = {}
+    if case == "page_12":
+        kp, vp = desc([10, 12, 2, 128]), desc([10, 12, 2, 128])
+    elif case == "page_8":
+        kp, vp = desc([10, 8, 2, 128]), desc([10, 8, 2, 128])
+    elif case == "stride_lt_blocks":
+        kw = dict(bt_stride=2, max_blocks=4)
+    elif case == "null_table":
+        kw = dict(bt=0)
+    elif case == "null_seqlens":
+        kw = dict(sl=0)
+    elif case == "blocks_mismatch":
+        vp = desc([11, 16, 2, 128])
+    elif case == "misaligned_table":
+        kw = dict(bt=0x20002)
+    assert call_paged(q, kp, vp, **kw) == expect
+    assert fa.load_library().fa_last_error()
+
+
+@pytest.mark.parametrize("case", ["shape", "dtype", "heads"])
+def test_append_host_validation(case):
+    lib = fa.load_library()
+    q, k, v, o = good("q"), good("k"), good("v"), good("o")
+    kn, vn = desc([1, 1, 2, 128]), desc([1, 1, 2, 128])
+    if case == "shape":
+        vn = desc([1, 2, 2, 128])
+    elif case == "dtype":
+        kn = desc([1, 1, 2, 128], dtype=1)
+    elif case == "heads":
+        kn, vn = desc([1, 1, 4, 128]), desc([1, 1, 4, 128])
+    st = lib.fa_decode_kvcache_append(ctypes.byref(q), ctypes.byref(kn), ctypes.byref(vn), ctypes.byref(k),
+                                      ctypes.byref(v), None, 0, 0, ctypes.c_void_p(0x30000), ctypes.byref(o), None,
+                                      0, 0, 0.0, None, 0, None)
+    assert st == INVALID
+    assert fa.load_library().fa_last_error()
