@@ -27,7 +27,7 @@ import torch
 
 __all__ = [
     "FaError", "fa_fwd", "fa_decode_kvcache", "fa_decode_kvcache_paged", "paged_workspace_size",
-    "fa_decode_kvcache_append",
+    "fa_decode_kvcache_append", "fa_fwd_varlen", "flash_attn_varlen_func",
     "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
     "last_dispatch", "force_variant", "profile_enable", "profile_read", "launch_count",
@@ -84,6 +84,8 @@ def load_library():
         "fa_decode_kvcache_workspace_size": (i32, [T, T, T, i32, P(sz)]),
         "fa_decode_kvcache_paged": (i32, [T, T, T, vp, ctypes.c_int64, i32, vp, T, vp, i32, i32, f32, vp, sz, vp]),
         "fa_decode_kvcache_paged_workspace_size": (i32, [T, T, T, i32, i32, P(sz)]),
+        "fa_fwd_varlen": (i32, [T, T, T, vp, vp, i32, i32, i32, T, vp, i32, f32, i32, vp, sz, vp]),
+        "fa_fwd_varlen_workspace_size": (i32, [T, T, T, i32, i32, i32, i32, P(sz)]),
         "fa_decode_kvcache_append": (i32, [T, T, T, T, T, vp, ctypes.c_int64, i32, vp, T, vp, i32, i32, f32, vp,
                                            sz, vp]),
         "fa_check_status": (i32, [vp]),
@@ -305,6 +307,53 @@ def fa_decode_kvcache_append(q, k_new, v_new, k_cache, v_cache, cache_seqlens, b
             float(scale or 0.0), ctypes.c_void_p(ws.data_ptr() if ws is not None else None), ws_bytes,
             _stream_ptr(q)))
     return out, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False, scale=None,
+                  num_splits=0, out=None, lse=None, workspace=None, return_lse=True):
+    """Attention within packed variable-length sequences: q [total_q, Hq, Dqk],
+    k [total_k, Hkv, Dqk], v [total_k, Hkv, Dv] (3-D, or 4-D with a leading 1),
+    cu_seqlens_q / cu_seqlens_k CUDA int32 [batch + 1].  Returns
+    (o [total_q, Hq, Dv] in q's rank, lse [Hq, total_q])."""
+    lib = load_library()
+    dev = _cuda_inputs(q, k, v, cu_seqlens_q, cu_seqlens_k)
+    for name, cu in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if cu.dtype != torch.int32 or cu.dim() != 1 or not cu.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 [batch + 1] tensor")
+    if cu_seqlens_k.shape[0] != cu_seqlens_q.shape[0]:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    batch = cu_seqlens_q.shape[0] - 1
+    squeeze = q.dim() == 3
+    q4, k4, v4 = (t.unsqueeze(0) if t.dim() == 3 else t for t in (q, k, v))
+    total_q, Hq = q4.shape[1], q4.shape[2]
+    if out is None:
+        out = torch.empty((1, total_q, Hq, v4.shape[3]), dtype=q.dtype, device=dev)
+    o4 = out.unsqueeze(0) if out.dim() == 3 else out
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=dev)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or tuple(lse.shape) != (Hq, total_q)):
+        raise ValueError("lse must be a contiguous float32 [Hq, total_q] tensor")
+    with torch.cuda.device(dev):
+        n = ctypes.c_size_t(0)
+        _check(lib.fa_fwd_varlen_workspace_size(_desc(q4, "q"), _desc(k4, "k"), _desc(v4, "v"), int(batch),
+                                                int(max_seqlen_q), int(max_seqlen_k), int(num_splits),
+                                                ctypes.byref(n)))
+        ws, ws_bytes = _workspace(n.value, dev, workspace)
+        _check(lib.fa_fwd_varlen(
+            _desc(q4, "q"), _desc(k4, "k"), _desc(v4, "v"), ctypes.c_void_p(cu_seqlens_q.data_ptr()),
+            ctypes.c_void_p(cu_seqlens_k.data_ptr()), int(batch), int(max_seqlen_q), int(max_seqlen_k),
+            _desc(o4, "o"), ctypes.c_void_p(lse.data_ptr() if lse is not None else None), int(bool(causal)),
+            float(scale or 0.0), int(num_splits), ctypes.c_void_p(ws.data_ptr() if ws is not None else None),
+            ws_bytes, _stream_ptr(q)))
+    return (o4[0] if squeeze and out.dim() == 4 else out), lse
+
+
+def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                           softmax_scale=None, return_attn_probs=False):
+    o, lse = fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=causal,
+                           scale=softmax_scale, return_lse=return_attn_probs)
+    return (o, lse) if return_attn_probs else o
 
 
 def flash_attn_func(q, k, v, causal=False, softmax_scale=None, return_lse=False):

@@ -159,6 +159,14 @@ struct Shapes {
 
 // Paged K/V: K and V are [num_blocks, page, Hkv, D]; batch b's key j is row
 // j % page of block block_table[b * bt_stride + j / page].
+// Packed variable-length inputs: q / o [1, total_q, H, D], k / v
+// [1, total_k, Hkv, D]; sequence b owns query tokens [cu_q[b], cu_q[b + 1])
+// and key tokens [cu_k[b], cu_k[b + 1]).
+struct Varlen {
+    const int32_t *cu_q, *cu_k;
+    int total_q;
+};
+
 struct Paging {
     const int32_t *block_table;
     int64_t bt_stride;
@@ -435,14 +443,15 @@ fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
 fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
               const int32_t *seqlens, float *lse, int causal, float scale, int num_splits, void *workspace,
               size_t workspace_bytes, cudaStream_t stream, const Paging *pg = nullptr,
-              const fa::AppendParams *ap = nullptr) {
+              const fa::AppendParams *ap = nullptr, const Varlen *vl = nullptr) {
     if (s.B == 0 || s.Lq == 0) {
         t_disp = {};
         return FA_OK;
     }
     Plan pl;
-    fa_status st = make_plan(s, causal, num_splits, seqlens != nullptr, s.Lk, &pl);
+    fa_status st = make_plan(s, causal, num_splits, seqlens != nullptr || vl != nullptr, s.Lk, &pl);
     if (st) return st;
+    if (vl) pl.comb_grid = (int)(((int64_t)s.Hq * vl->total_q + 3) / 4);
     if (workspace_bytes < pl.ws_bytes)
         return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
                     pl.ws_bytes);
@@ -485,6 +494,17 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.min_share = pl.min_share;
     p.tile_keys = pl.main.tile_keys;
     p.tile_shift = log2_exact(pl.main.tile_keys);
+    p.lse_sb = (int64_t)s.Hq * s.Lq;
+    p.lse_sh = s.Lq;
+    if (vl) {
+        p.cu_q = vl->cu_q;
+        p.cu_k = vl->cu_k;
+        p.total_q = vl->total_q;
+        p.q_sb = 0;
+        p.o_sb = 0;
+        p.lse_sb = 0;
+        p.lse_sh = vl->total_q;
+    }
     if (pg) {
         p.block_table = pg->block_table;
         p.bt_stride = pg->bt_stride;
@@ -754,6 +774,89 @@ fa_status fa_decode_kvcache_append(const fa_tensor *q, const fa_tensor *k_new, c
     a.capacity = s.Lk;
     return run(s, q, k_cache, v_cache, o, cache_seqlens, lse, causal, scale, num_splits, workspace, workspace_bytes,
                static_cast<cudaStream_t>(stream), block_table ? &pg : nullptr, &a);
+}
+
+// q [1, total_q, Hq, Dqk], k [1, total_k, Hkv, Dqk], v [1, total_k, Hkv, Dv],
+// o [1, total_q, Hq, Dv] (o may be null for the workspace query).
+fa_status check_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const fa_tensor *o, int batch,
+                       int max_q, int max_k, Shapes *s) {
+    fa_status st;
+    if ((st = check_tensor(q, "q")) || (st = check_tensor(k, "k")) || (st = check_tensor(v, "v"))) return st;
+    if (o && (st = check_tensor(o, "o"))) return st;
+    if (k->dtype != q->dtype || v->dtype != q->dtype || (o && o->dtype != q->dtype))
+        return fail(FA_ERR_INVALID_ARG, "q, k, v and o must share one element type");
+    if (q->shape[0] != 1 || k->shape[0] != 1 || v->shape[0] != 1 || (o && o->shape[0] != 1))
+        return fail(FA_ERR_INVALID_ARG, "packed tensors are [1, total, H, D]");
+    if (batch < 0 || max_q < 0 || max_k < 0) return fail(FA_ERR_INVALID_ARG, "negative batch or length");
+    if (q->shape[1] > INT32_MAX / 2 || k->shape[1] > INT32_MAX / 2)
+        return fail(FA_ERR_UNSUPPORTED, "too many packed tokens");
+    s->dtype = q->dtype;
+    s->B = batch;
+    s->Lq = max_q;
+    s->Hq = (int)q->shape[2];
+    s->Dqk = (int)q->shape[3];
+    s->Lk = max_k;
+    s->Hkv = (int)k->shape[2];
+    s->Dv = (int)v->shape[3];
+    if (k->shape[3] != s->Dqk || v->shape[1] != k->shape[1] || v->shape[2] != s->Hkv)
+        return fail(FA_ERR_INVALID_ARG, "k / v must be [1, total_k, Hkv, D] with q's Dqk");
+    if (o && (o->shape[1] != q->shape[1] || o->shape[2] != s->Hq || o->shape[3] != s->Dv))
+        return fail(FA_ERR_INVALID_ARG, "o must be [1, total_q, Hq, Dv]");
+    if (s->Hkv <= 0 || s->Hq <= 0 || s->Hq % s->Hkv)
+        return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", s->Hq, s->Hkv);
+    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128) ||
+          (s->Dqk == 256 && s->Dv == 256)))
+        return fail(FA_ERR_UNSUPPORTED,
+                    "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128), (256,256)}", s->Dqk, s->Dv);
+    s->g = s->Hq / s->Hkv;
+    const int64_t R = (int64_t)s->g * s->Lq;
+    if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * max_seqlen_q too large");
+    s->R = (int)R;
+    s->RB = (s->R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
+    const int64_t BR = (int64_t)s->B * s->RB;
+    if (BR > fa::kMaxPrefixEntries)
+        return fail(FA_ERR_UNSUPPORTED, "batch * ceil(g * max_seqlen_q / 8) = %lld exceeds %d", (long long)BR,
+                    fa::kMaxPrefixEntries);
+    s->BR = (int)BR;
+    return FA_OK;
+}
+
+fa_status fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const int32_t *cu_seqlens_q,
+                        const int32_t *cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k, fa_tensor *o,
+                        float *lse, int causal, float scale, int num_splits, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    Shapes s;
+    fa_status st = check_varlen(q, k, v, o, batch, max_seqlen_q, max_seqlen_k, &s);
+    if (st) return st;
+    if (!o) return fail(FA_ERR_INVALID_ARG, "o: null descriptor");
+    if (batch > 0 && (!cu_seqlens_q || !cu_seqlens_k))
+        return fail(FA_ERR_INVALID_ARG, "cu_seqlens_q / cu_seqlens_k: null pointer");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) | reinterpret_cast<uintptr_t>(cu_seqlens_k)) & 3u)
+        return fail(FA_ERR_INVALID_ARG, "cu_seqlens must be 4-byte aligned");
+    if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "scale must be finite");
+    const Varlen vl = {cu_seqlens_q, cu_seqlens_k, (int)q->shape[1]};
+    if (vl.total_q == 0) {
+        t_disp = {};
+        return FA_OK;
+    }
+    return run(s, q, k, v, o, nullptr, lse, causal, scale, num_splits, workspace, workspace_bytes,
+               static_cast<cudaStream_t>(stream), nullptr, nullptr, &vl);
+}
+
+fa_status fa_fwd_varlen_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int batch,
+                                       int max_seqlen_q, int max_seqlen_k, int num_splits, size_t *bytes) {
+    if (!bytes) return fail(FA_ERR_INVALID_ARG, "bytes: null pointer");
+    Shapes s;
+    fa_status st = check_varlen(q, k, v, nullptr, batch, max_seqlen_q, max_seqlen_k, &s);
+    if (st) return st;
+    if (s.B == 0 || s.Lq == 0) {
+        *bytes = 0;
+        return FA_OK;
+    }
+    Plan pl;
+    if ((st = make_plan(s, 0, num_splits, true, s.Lk, &pl))) return st;
+    *bytes = pl.ws_bytes;
+    return FA_OK;
 }
 
 fa_status fa_check_status(void *stream) {

@@ -33,14 +33,47 @@ __global__ void __launch_bounds__(kCombineThreads)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long row = (long long)blockIdx.x * (kCombineThreads / 32) + warp;
-    const long long rows = (long long)p.B * p.Hq * p.Lq;
-    const bool live = row < rows;
-    const int i = live ? (int)(row % p.Lq) : 0;
-    const int hq = live ? (int)((row / p.Lq) % p.Hq) : 0;
-    const int b = live ? (int)(row / ((long long)p.Lq * p.Hq)) : 0;
-    const int r = (hq % p.g) * p.Lq + i;
-    const int rb = r / kRowsPerCta, rr = r % kRowsPerCta, hkv = hq / p.g;
-    const int x = b * p.RB + rb;
+    // This warp's output row (b, hq, i), the token offset q0 of its batch's
+    // first query row, and its unit.  Dense rows are numbered (b, hq, i);
+    // packed variable-length rows (hq, token), the batch found in cu_q -- so
+    // only after the wait for them.
+    bool live = false;
+    int b = 0, hq = 0, i = 0, q0 = 0, rr = 0, hkv = 0, x = 0;
+    auto locate = [&]() {
+        int r = 0;
+        if (p.cu_q) {
+            live = row < (long long)p.Hq * p.total_q;
+            if (!live) return;
+            hq = (int)(row / p.total_q);
+            const int tok = (int)(row % p.total_q);
+            int lo = 0, hi = p.B;  // the batch b with cu_q[b] <= tok < cu_q[b + 1]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (p.cu_q[mid] <= tok) lo = mid;
+                else hi = mid;
+            }
+            b = lo;
+            q0 = p.cu_q[b];
+            i = tok - q0;
+            const BatchGeom G = batch_geom(p, b);
+            if (i >= G.Lq) {  // past the longest query length: not computed
+                live = false;
+                return;
+            }
+            r = (hq % p.g) * G.Lq + i;
+        } else {
+            live = row < (long long)p.B * p.Hq * p.Lq;
+            if (!live) return;
+            i = (int)(row % p.Lq);
+            hq = (int)((row / p.Lq) % p.Hq);
+            b = (int)(row / ((long long)p.Lq * p.Hq));
+            r = (hq % p.g) * p.Lq + i;
+        }
+        rr = r % kRowsPerCta;
+        hkv = hq / p.g;
+        x = b * p.RB + r / kRowsPerCta;
+    };
+    if (!p.cu_q) locate();
 
     // The partition and the partials' addresses are worked out before the
     // wait (dense inputs need no memory for it); cache lengths only after it.
@@ -63,7 +96,7 @@ __global__ void __launch_bounds__(kCombineThreads)
                 base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr;
         }
     };
-    if (!p.seqlens) plan();
+    if (uniform_batches(p) && live) plan();
 
     // Two passes over the same code: a warm-up pass before the wait for the
     // split-KV kernel, which merges eight copies of a shared-memory row into a
@@ -77,8 +110,9 @@ __global__ void __launch_bounds__(kCombineThreads)
             // Every CTA waits for the split-KV kernel before it exits, so this
             // grid completing implies that one completed too.
             pdl_wait_primary();
-            if (p.seqlens) plan();
+            if (p.cu_q) locate();
             if (!live) return;
+            if (!uniform_batches(p)) plan();
             if (t > 0 && nparts == 1) return;  // finished inside one piece by the split-KV kernel
         }
         const int tu = warm ? 1 : t, np = warm ? PPP : nparts;
@@ -86,9 +120,9 @@ __global__ void __launch_bounds__(kCombineThreads)
         const float *ws_o = warm ? sink : p.ws_o;
         const float *ws_lse = warm ? sink : p.ws_lse;
         T *op = warm ? reinterpret_cast<T *>(sink)
-                     : reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh +
-                           lane * EPL;
-        float *lse_out = warm ? sink : (p.lse ? p.lse + ((long long)b * p.Hq + hq) * p.Lq + i : nullptr);
+                     : reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)(q0 + i) * p.o_sl +
+                           (long long)hq * p.o_sh + lane * EPL;
+        float *lse_out = warm ? sink : (p.lse ? p.lse + b * p.lse_sb + hq * p.lse_sh + q0 + i : nullptr);
         const int lane_off = warm ? 0 : lane * EPL;
         float acc[EPL];
 #pragma unroll

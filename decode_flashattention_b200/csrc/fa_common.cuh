@@ -47,7 +47,17 @@ struct Params {
     int page_shift;        // log2(page)
     int num_blocks;
     int seqlen_add;        // tokens appended to every cache by this call (added to seqlens[b])
+    // Packed variable-length inputs (cu_q non-null): q / o are [1, total_q, H, D]
+    // and k / v [1, total_k, Hkv, D]; sequence b owns query tokens
+    // [cu_q[b], cu_q[b+1]) and key tokens [cu_k[b], cu_k[b+1]); Lq and Lk hold
+    // the largest lengths.  lse element (b, hq, i) is at
+    // b * lse_sb + hq * lse_sh + (query token offset) + i.
+    const int *cu_q;
+    const int *cu_k;
+    int64_t lse_sb, lse_sh;
+    int total_q;           // packed query tokens (the combine's row count is Hq * total_q)
 };
+
 
 // ------------------------------------------------------------------ schedule
 // Work is counted in key tiles.  A unit is (batch b, row block rb, kv head
@@ -61,7 +71,7 @@ struct Params {
 // CTA's first segment and slot 1 otherwise, and the combine kernel merges them.
 
 __host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int Lq, int causal) {
-    if (n <= 0) return 0;
+    if (n <= 0 || rb * kRowsPerCta >= R) return 0;  // no keys, or a row block past the batch's rows
     if (!causal) return n;
     // rows r0 .. r0 + cnt - 1 hold query positions i = r % Lq; the largest one
     // is r0 % Lq + cnt - 1 unless the run wraps past Lq - 1.
@@ -74,7 +84,6 @@ __host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int L
     return k > 0 ? k : 0;
 }
 
-// Keys present for batch b: cache_seqlens[b] clamped to [0, Lk], or Lk.
 // Keys present for batch b: Lk for dense inputs, else cache_seqlens[b] plus
 // the tokens appended by this call, clamped to [0, Lk].
 __host__ __device__ inline int batch_keys(const int *seqlens, int b, int Lk, int add = 0) {
@@ -82,6 +91,36 @@ __host__ __device__ inline int batch_keys(const int *seqlens, int b, int Lk, int
     const long long n = (long long)seqlens[b] + add;
     return n < 0 ? 0 : (n > Lk ? Lk : (int)n);
 }
+
+#if defined(__CUDACC__)
+// Row geometry of batch b: its query rows Lq, packed rows R = g * Lq, keys n
+// and the token offsets of its first query / key row (0 unless packed).
+struct BatchGeom {
+    int Lq, R, n, q0, k0;
+};
+
+__device__ __forceinline__ BatchGeom batch_geom(const Params &p, int b) {
+    BatchGeom G;
+    if (p.cu_q) {
+        const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+        int lq = q1 - q0, n = k1 - k0;
+        lq = lq < 0 ? 0 : (lq > p.Lq ? p.Lq : lq);
+        n = n < 0 ? 0 : (n > p.Lk ? p.Lk : n);
+        G.Lq = lq;
+        G.R = p.g * lq;
+        G.n = n;
+        G.q0 = q0;
+        G.k0 = k0;
+    } else {
+        G.Lq = p.Lq;
+        G.R = p.R;
+        G.n = batch_keys(p.seqlens, b, p.Lk, p.seqlen_add);
+        G.q0 = 0;
+        G.k0 = 0;
+    }
+    return G;
+}
+#endif
 
 // Tiles of tile_keys = 1 << tile_shift keys covering the visible keys.
 __host__ __device__ inline int unit_tiles(int n, int rb, int R, int Lq, int causal, int tile_shift) {
@@ -380,7 +419,8 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16 *dst, co
 
 __device__ __forceinline__ int entry_tiles(const Params &p, int x) {
     const int b = x / p.RB, rb = x - b * p.RB;
-    return unit_tiles(batch_keys(p.seqlens, b, p.Lk, p.seqlen_add), rb, p.R, p.Lq, p.causal, p.tile_shift);
+    const BatchGeom G = batch_geom(p, b);
+    return unit_tiles(G.n, rb, G.R, G.Lq, p.causal, p.tile_shift);
 }
 
 __device__ __forceinline__ int warp_sum(int v) {
@@ -397,16 +437,20 @@ __device__ __forceinline__ int warp_entry_tiles(const Params &p, int x0, int x1)
     return warp_sum(acc) * p.Hkv;
 }
 
-// Total tiles W.  Dense inputs (no seqlens): every batch has the same units.
+// Dense inputs (no cache lengths, not packed): every batch has the same units,
+// and the schedule needs no memory reads.
+__device__ __forceinline__ bool uniform_batches(const Params &p) { return !p.seqlens && !p.cu_q; }
+
+// Total tiles W.
 __device__ __forceinline__ int warp_total_tiles(const Params &p) {
     if (p.W_host >= 0) return p.W_host;
-    if (!p.seqlens) return warp_entry_tiles(p, 0, p.RB) * p.B;
+    if (uniform_batches(p)) return warp_entry_tiles(p, 0, p.RB) * p.B;
     return warp_entry_tiles(p, 0, p.B * p.RB);
 }
 
 // First tile position of entry x's units.
 __device__ __forceinline__ int warp_entry_begin(const Params &p, int x) {
-    if (!p.seqlens) {
+    if (uniform_batches(p)) {
         const int b = x / p.RB;
         return warp_entry_tiles(p, 0, p.RB) * b + warp_entry_tiles(p, b * p.RB, x);
     }
@@ -418,7 +462,7 @@ __device__ __forceinline__ int warp_entry_begin(const Params &p, int x) {
 __device__ __forceinline__ int warp_locate(const Params &p, int t, int *x_begin) {
     const int lane = threadIdx.x & 31;
     int x_lo = 0, x_hi = p.B * p.RB, run = 0;
-    if (!p.seqlens) {  // jump straight to the batch: all batches weigh the same
+    if (uniform_batches(p)) {  // jump straight to the batch: all batches weigh the same
         const int per_batch = warp_entry_tiles(p, 0, p.RB);
         const int b = t / per_batch;
         x_lo = b * p.RB;

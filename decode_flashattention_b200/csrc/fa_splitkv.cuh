@@ -133,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ============================================================ producer warp
         // Dense inputs: the schedule needs only the kernel's parameters, so it
         // is worked out before the wait and overlaps the previous kernel; cache
-        // lengths and the pool header are read only after the wait.
+        // or sequence lengths are read only after the wait.
         Partition pt = {0, 1};
         SegmentWalker wk;
         bool active = false;
@@ -143,12 +143,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             active = pt.W > 0 && cta < pt.P;
             if (active) wk.init(p, piece_start(pt, cta), piece_end(pt, cta));
         };
-        if (!p.seqlens) plan();
+        if (uniform_batches(p)) plan();
         pdl_wait_primary();
         // The combine kernel's CTAs may be scheduled now (they wait for this
         // grid to complete before reading anything it writes).
         pdl_launch_dependents();
-        if (p.seqlens) plan();
+        if (!uniform_batches(p)) plan();
 
         const T *__restrict__ qg = reinterpret_cast<const T *>(p.q);
         const uint64_t policy = l2_policy_evict_first();
@@ -157,6 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
         for (; active && !wk.done() && !stop; wk.advance(p)) {
             const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
+            const BatchGeom G = batch_geom(p, b);
+            const int kb = p.cu_q ? 0 : b;  // K / V batch coordinate (packed inputs: one batch of tokens)
             const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
             const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
             const int slot = (wk.pos == lo) ? 0 : 1;
@@ -178,10 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
 #pragma unroll
                         for (int c = 0; c < C::KBOX; ++c)
-                            tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, j, hkv, b, policy);
+                            tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
 #pragma unroll
                         for (int c = 0; c < C::VBOX; ++c)
-                            tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, j, hkv, b, policy);
+                            tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
                     }
                 } else {
                     // Paged K/V: the tile is gathered page by page.  A page of at
@@ -226,9 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int rq = rb * kRowsPerCta + r;
                         const T *src = qg;
                         uint32_t nbytes = 0;
-                        if (rq < p.R) {
-                            const int hq = hkv * p.g + rq / p.Lq, i = rq % p.Lq;
-                            src = qg + b * p.q_sb + (long long)i * p.q_sl + (long long)hq * p.q_sh + c * 8;
+                        if (rq < G.R) {
+                            const int hq = hkv * p.g + rq / G.Lq, i = rq % G.Lq;
+                            src = qg + b * p.q_sb + (long long)(G.q0 + i) * p.q_sl + (long long)hq * p.q_sh + c * 8;
                             nbytes = 16;
                         }
                         cp_async_16(qs + (r * C::Q_STRIDE + c * 8) * 2, src, nbytes);
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Merge of the four warps' (m, l, O) published in shared memory, then the
     // store of the final O / lse (unit finished here) or of the partial and its
     // log2-sum-exp.  Shared by both variants.
-    auto merge_store = [&](const StageMeta &md, bool warm) {
+    auto merge_store = [&](const StageMeta &md, bool warm, const BatchGeom &cg) {
         // thread -> (row, 8 consecutive dims); weights 2^(m_w - M) of the warps' partials
         constexpr int EPT = DV * kRowsPerCta / (32 * kConsumerWarps);
         constexpr int TPR = DV / EPT;
@@ -344,10 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float lse2 = L > 0.f ? M + log2f(L) : -INFINITY;
         const int rr = md.rb * kRowsPerCta + r;
         if (md.flags & kMetaWhole) {
-            if (rr < p.R) {
-                const int hq = md.hkv * p.g + rr / p.Lq, i = rr % p.Lq;
+            if (rr < cg.R) {
+                const int hq = md.hkv * p.g + rr / cg.Lq, i = rr % cg.Lq;
                 T *op = warm ? static_cast<T *>(sink)
-                             : og + md.b * p.o_sb + (long long)i * p.o_sl + (long long)hq * p.o_sh + d0;
+                             : og + md.b * p.o_sb + (long long)(cg.q0 + i) * p.o_sl + (long long)hq * p.o_sh + d0;
                 if constexpr (EPT % 8 == 0) {
 #pragma unroll
                     for (int e = 0; e < EPT; e += 8) store_row8<T>(op + e, v + e);
@@ -357,8 +359,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(v[e], v[e + 1]);
                 }
                 if (p.lse && (tid % TPR) == 0)
-                    *(warm ? static_cast<float *>(sink) : p.lse + ((long long)md.b * p.Hq + hq) * p.Lq + i) =
-                        lse2 * 0.69314718055994531f;
+                    *(warm ? static_cast<float *>(sink)
+                           : p.lse + md.b * p.lse_sb + hq * p.lse_sh + cg.q0 + i) = lse2 * 0.69314718055994531f;
             }
         } else {
             const long long base = ((long long)md.piece * 2 + md.slot) * kRowsPerCta + r;
@@ -386,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 8; ++j) vsw[j] = (dl >> 6) * C::BOX_BYTES + ((((dl & 63) >> 3) ^ j) << 4) + (dl & 7) * 2;
         int n = 0;
+        BatchGeom cg = {p.Lq, p.R, 0, 0, 0};
         float m = -INFINITY;  // running max of the warp's scores (base 2)
         float l = 0.f;        // this lane's share of the running sum
         float acc[EPL];
@@ -409,7 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const T *qs = reinterpret_cast<const T *>(smem + C::OFF_Q + s * C::Q_BYTES);
                 for (int d = lane; d < DQK; d += 32) qf32[d] = Cvt<T>::f1(qs[d]);
                 __syncwarp();
-                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk, p.seqlen_add);
+                cg = warm ? BatchGeom{p.Lq, p.R, 1 << 30, 0, 0} : batch_geom(p, md.b);
+                n = cg.n;
                 m = -INFINITY;
                 l = 0.f;
 #pragma unroll
@@ -466,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- cache slots at or beyond this batch's length may hold anything
             // (NaN included): zero those V rows so 0 * V stays 0.
             const uint32_t vbase = vst + kw * 128;
-            if (p.seqlens && jbase + C::KEYS_PER_WARP > n) {
+            if ((p.seqlens || p.cu_q) && jbase + C::KEYS_PER_WARP > n) {
                 for (int idx = lane; idx < C::KEYS_PER_WARP * C::VBOX * 8; idx += 32) {
                     const int key = idx / (C::VBOX * 8);
                     const int rem = idx % (C::VBOX * 8);
@@ -518,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
             }
             if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
-            merge_store(md, warm);
+            merge_store(md, warm, cg);
             // red / sm_m / sm_l are reused by the next segment, if there is one
             if (md.flags & kMetaFinal) break;
             if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
@@ -528,6 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t qf[DQK / 16][2];
         int lim[2] = {0, 0};
         int n = 0;
+        BatchGeom cg = {p.Lq, p.R, 0, 0, 0};
         float m[2] = {-INFINITY, -INFINITY};
         float l[2] = {0.f, 0.f};
         float acc[DV / 16][4];
@@ -553,14 +558,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][0]) : "r"(qrow + kk * 32));
                     asm volatile("ld.shared.b32 %0, [%1];" : "=r"(qf[kk][1]) : "r"(qrow + kk * 32 + 16));
                 }
-                n = warm ? (1 << 30) : batch_keys(p.seqlens, md.b, p.Lk, p.seqlen_add);
+                cg = warm ? BatchGeom{p.Lq, p.R, 1 << 30, 0, 0} : batch_geom(p, md.b);
+                n = cg.n;
                 // last visible key of this lane's two accumulator rows (bottom-right causal)
     #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int r = md.rb * kRowsPerCta + r_lo + e;
                     int lm = n - 1;
-                    if (p.causal && r < p.R) {
-                        const int c = r % p.Lq + n - p.Lq;
+                    if (p.causal && r < cg.R) {
+                        const int c = r % cg.Lq + n - cg.Lq;
                         lm = c < lm ? c : lm;
                     }
                     lim[e] = lm;
@@ -638,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // ---- cache slots at or beyond this batch's length may hold anything
             // (NaN included): zero those V rows so 0 * V stays 0.
-            if (p.seqlens && jbase + C::KEYS_PER_WARP > n) {
+            if ((p.seqlens || p.cu_q) && jbase + C::KEYS_PER_WARP > n) {
                 for (int idx = lane; idx < C::KEYS_PER_WARP * C::VBOX * 8; idx += 32) {
                     const int key = idx / (C::VBOX * 8);
                     const int rem = idx % (C::VBOX * 8);
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
-            merge_store(md, warm);
+            merge_store(md, warm, cg);
             // red / sm_m / sm_l are reused by the next segment, if there is one
             if (md.flags & kMetaFinal) break;
             if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;

@@ -196,6 +196,36 @@ FA_API fa_status fa_decode_kvcache_append(const fa_tensor *q, const fa_tensor *k
                                           void *stream);
 
 /*
+ * fa_fwd_varlen -- fa_fwd over packed variable-length sequences.
+ *
+ * The MXFlashAttn README's public entry points include
+ * flash_attn_varlen_func, and the CSDN "FlashAttention on Ascend CANN" post
+ * lists packed (not padded) variable-length input among the operator's
+ * features; the layout is FlashAttention's cu_seqlens convention:
+ *   q [1, total_q, Hq, Dqk], k [1, total_k, Hkv, Dqk], v [1, total_k, Hkv, Dv],
+ *   o [1, total_q, Hq, Dv] (fa_tensor, shape[0] = 1);
+ *   cu_seqlens_q / cu_seqlens_k: DEVICE int32 [batch + 1], non-decreasing,
+ *   cu[0] = 0; sequence b owns query tokens [cu_q[b], cu_q[b+1]) and key
+ *   tokens [cu_k[b], cu_k[b+1]);
+ *   max_seqlen_q / max_seqlen_k: bounds on the lengths (rows and keys beyond
+ *   them are not computed / not read);
+ *   lse, when not NULL: DEVICE fp32 [Hq, total_q] (contiguous).
+ * Attention runs within each sequence: query i of sequence b attends its own
+ * keys, with the causal mask aligned to the bottom-right corner of that
+ * sequence (key j visible iff j <= i + n_b - Lq_b); a sequence with no keys
+ * gives O = 0, lse = -inf.  scale, num_splits, workspace (size from
+ * fa_fwd_varlen_workspace_size), stream and errors as for fa_fwd.
+ */
+FA_API fa_status fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
+                               const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int batch,
+                               int max_seqlen_q, int max_seqlen_k, fa_tensor *o, float *lse, int causal, float scale,
+                               int num_splits, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace fa_fwd_varlen needs for these shapes on the current device. */
+FA_API fa_status fa_fwd_varlen_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, int batch,
+                                              int max_seqlen_q, int max_seqlen_k, int num_splits, size_t *bytes);
+
+/*
  * fa_decode_kvcache_noalloc -- fa_decode_kvcache for callers that cannot
  * allocate device memory (for example a plugin inside a serving runtime that
  * owns all device memory and forbids allocation after start-up, or a decode

@@ -242,3 +242,26 @@ def append_kv(k_cache, v_cache, k_new, v_new, seqlens, block_table=None):
                 kc[blk, pos % page] = k_new[b, t]
                 vc[blk, pos % page] = v_new[b, t]
     return kc, vc
+
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, causal: bool = False, scale: float | None = None,
+                     nthreads: int | None = None):
+    """The definition within each packed sequence: q [total_q, Hq, Dqk],
+    k [total_k, Hkv, Dqk], v [total_k, Hkv, Dv] (CPU); sequence b owns query
+    tokens [cu_q[b], cu_q[b+1]) and key tokens [cu_k[b], cu_k[b+1]).  Returns
+    (o [total_q, Hq, Dv], lse [Hq, total_q]), fp64."""
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64).reshape(-1)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64).reshape(-1)
+    total_q, Hq = int(q.shape[0]), int(q.shape[1])
+    Dv = int(v.shape[2])
+    o = np.zeros((total_q, Hq, Dv), dtype=np.float64)
+    lse = np.full((Hq, total_q), -np.inf, dtype=np.float64)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 <= q0:
+            continue
+        ob, lb = attention(q[q0:q1][None], k[k0:k1][None], v[k0:k1][None], causal=causal, scale=scale,
+                           nthreads=nthreads)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
