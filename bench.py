@@ -161,6 +161,28 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ helpers
+def tensor_roofline(w, seqlens, ms_per_call, prof):
+    """Roofline of a call on the tcgen05 kernel: bound by the tensor cores.
+    achieved = the call's multiply-add flops / its time; peak = the measured
+    sustained cuBLAS bf16 rate (the kernel runs back to back for seconds), the
+    same for fp16 (the nominal fp16 and bf16 rates are equal)."""
+    from decode_flashattention_b200 import workloads as wl
+
+    flops = wl.attn_flops(w, seqlens)
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        peak, kind = float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured (sustained)"
+    else:
+        peak, kind = 1400.0, "fallback (sustained)"
+    achieved = flops / (ms_per_call / 1e3) / 1e12
+    return {"bound": "tensor", "kernel": "tcgen05 dense kernel (whole call)", "achieved": round(achieved, 2),
+            "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "traffic": None, "algorithmic_flops_per_launch": flops, "kernel_us": round(ms_per_call * 1e3, 3),
+            "isolated_us": {"tcgen05": round(prof["main_ms"] / max(prof["main_launches"], 1) * 1e3, 3)}}
+
+
 def workload_of(args):
     """The named workload, with its batch size replaced when --batch is given."""
     import dataclasses
@@ -424,6 +446,7 @@ def run_ours(args):
     value = total_bytes / (ms / 1e3) / 1e12
     e2e_value = sum_over_ranks(bytes_per_step * E, world, device) / (e2e_ms / 1e3) / 1e12
     peak, peak_kind = peaks()
+    tc = dispatch.get("variant") == fa.VARIANT_TCGEN05
     # Roofline of the call.  Both kernels run back to back with programmatic
     # overlap, so no event pair can time one of them inside the timed region
     # without breaking that overlap; the achieved figure therefore charges the
@@ -467,7 +490,7 @@ def run_ours(args):
             "parallelism": f"replicas{world}" if world > 1 else "single_gpu",
             "dispatch": dispatch,
         },
-        "roofline": {
+        "roofline": tensor_roofline(w, sl0, ms / K, prof) if tc else {
             "bound": "hbm",
             "kernel": "split-KV kernel, charged with the whole call (combine and boundaries included)",
             "achieved": round(achieved, 1) if achieved else None,

@@ -31,14 +31,14 @@ __all__ = [
     "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
     "last_dispatch", "force_variant", "profile_enable", "profile_read", "launch_count",
-    "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR",
+    "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR", "VARIANT_TCGEN05",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 _lib = None
 
-VARIANT_AUTO, VARIANT_MMA, VARIANT_SCALAR = 0, 1, 2
+VARIANT_AUTO, VARIANT_MMA, VARIANT_SCALAR, VARIANT_TCGEN05 = 0, 1, 2, 3
 _STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_WORKSPACE",
            4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
 _DTYPE = {torch.float16: 0, torch.bfloat16: 1}

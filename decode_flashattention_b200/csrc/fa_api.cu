@@ -251,6 +251,8 @@ struct Plan {
     size_t ws_bytes;
     int comb_smem;
     int comb_grid;
+    bool prefill = false;  // the tcgen05 kernel: one CTA per (block of 128 rows, kv head, batch), no combine
+    int rb128 = 0;
 };
 
 // The tensor-core variant puts the keys on the MMA's 16-row side, so even one
@@ -305,6 +307,30 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     fa_status st = device_state(&dev);
     if (st) return st;
     int variant = choose_variant(s);
+    // Calls with at least 128 packed rows (prefill-shaped) on dense K / V run on
+    // the tcgen05 kernel: 128 rows fill its M side, and the whole key range is
+    // one CTA's work (no split, no combine).
+    const bool tc_shape = !kvcache && s.R >= 128 && s.Dqk == 128 && s.Dv == 128;
+    if (variant == FA_VARIANT_TCGEN05 || (g_force_variant.load() == FA_VARIANT_AUTO && tc_shape)) {
+        if (!tc_shape && (kvcache || s.Dqk != 128 || s.Dv != 128))
+            return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 128/128");
+        if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, &pl->main))
+            return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d", s.dtype);
+        if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
+        pl->prefill = true;
+        pl->rb128 = (s.R + 127) / 128;
+        pl->P = (int)std::min<int64_t>((int64_t)pl->rb128 * s.Hkv * s.B, INT32_MAX);
+        pl->P_param = pl->P;
+        pl->min_share = 0;
+        pl->W = -1;
+        pl->need_combine = pl->need_workspace = false;
+        pl->pieces = 0;
+        pl->ws_o_off = pl->ws_lse_off = pl->ws_bytes = 0;
+        pl->comb_smem = pl->comb_grid = 0;
+        if (pl->rb128 > 65535 * 16 || s.Hkv > 65535 || s.B > 65535)
+            return fail(FA_ERR_UNSUPPORTED, "grid too large for the tcgen05 variant");
+        return FA_OK;
+    }
     bool ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.Dqk, s.Dv, &pl->main)
                                            : fa::get_mma_kernel(s.dtype, s.Dqk, s.Dv, &pl->main);
     if (variant == FA_VARIANT_SCALAR && ok && s.R != 1)
@@ -557,7 +583,26 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         }
     }
 
-    const bool launch_main = pl.P > 0;
+    if (pl.prefill) {
+        CUtensorMap tmK, tmV;
+        if ((st = encode_kv_map(k, pl.main.tile_keys, &tmK, "k"))) return st;
+        if ((st = encode_kv_map(v, pl.main.tile_keys, &tmV, "v"))) return st;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)pl.rb128, (unsigned)s.Hkv, (unsigned)s.B);
+        cfg.blockDim = dim3((unsigned)pl.main.threads);
+        cfg.dynamicSmemBytes = (size_t)pl.main.smem;
+        cfg.stream = stream;
+        void *args[] = {&tmK, &tmV, &p};
+        if (prof && (st = prof_record(&rec->e0, stream))) return st;
+        cudaError_t e = cudaLaunchKernelExC(&cfg, pl.main.fn, args);
+        if (e != cudaSuccess) return cuda_fail(e, "launch of the tcgen05 kernel");
+        g_launches.fetch_add(1);
+        if (prof) {
+            rec->has_comb = false;
+            if ((st = prof_record(&rec->e1, stream)) || (st = prof_record(&rec->e2, stream))) return st;
+        }
+    }
+    const bool launch_main = pl.P > 0 && !pl.prefill;
     if (launch_main) {
         CUtensorMap tmK, tmV;
         const int box_rows = pg ? (int)std::min<int64_t>(k->shape[1], pl.main.tile_keys) : pl.main.tile_keys;
@@ -583,7 +628,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         if (e != cudaSuccess) return cuda_fail(e, "launch of the split-KV kernel");
         g_launches.fetch_add(1);
         if (prof && (st = prof_record(&rec->e1, stream))) return st;
-    } else if (prof) {
+    } else if (prof && !pl.prefill) {
         if ((st = prof_record(&rec->e0, stream)) || (st = prof_record(&rec->e1, stream))) return st;
     }
     if (pl.need_combine) {
@@ -604,7 +649,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         if (e != cudaSuccess) return cuda_fail(e, "launch of the combine kernel");
         g_launches.fetch_add(1);
     }
-    if (prof) {
+    if (prof && !pl.prefill) {
         rec->has_comb = pl.need_combine;
         if ((st = prof_record(&rec->e2, stream))) return st;
     }
@@ -616,7 +661,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     d.smem_bytes = pl.main.smem;
     d.tile_keys = pl.main.tile_keys;
     d.stages = pl.main.stages;
-    d.rows_per_cta = fa::kRowsPerCta;
+    d.rows_per_cta = pl.prefill ? 128 : fa::kRowsPerCta;
     d.units = (int)((int64_t)s.B * s.RB * s.Hkv);
     d.min_share_tiles = pl.min_share;
     d.combine_launched = pl.need_combine ? 1 : 0;
@@ -884,7 +929,7 @@ void fa_last_dispatch(fa_dispatch_info *info) {
 }
 
 fa_status fa_force_variant(int variant) {
-    if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_SCALAR)
+    if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_TCGEN05)
         return fail(FA_ERR_INVALID_ARG, "unknown variant %d", variant);
     g_force_variant.store(variant);
     return FA_OK;

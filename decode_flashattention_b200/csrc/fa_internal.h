@@ -20,6 +20,9 @@ bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 // LSE-weighted combine of split partials.
 bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
 
+// Dense attention on tcgen05 for calls with many packed rows (fa_prefill.cu).
+bool get_prefill_kernel(int dtype, int dqk, int dv, KernelInfo *out);
+
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 

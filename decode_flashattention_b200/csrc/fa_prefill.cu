@@ -1,0 +1,416 @@
+// fa_prefill.cu -- dense attention for many packed query rows on the 5th-gen
+// tensor cores (tcgen05 + TMEM): the prefill-shaped calls of fa_fwd.
+//
+// One CTA per (batch, kv head, block of 128 packed query rows).  Packed row r
+// of kv head hkv is query head hkv * g + r / Lq at position r % Lq (the same
+// packing as the split-KV kernel), so the g heads of a GQA group share every
+// K / V tile.  The CTA walks all key tiles its rows can see (128 keys each):
+//
+//   S  = Q K^T        tcgen05.mma (M 128 rows, N 128 keys, K = head dim),
+//                     fp32 accumulator in TMEM columns [0, 128)
+//   softmax           one thread per row reads its S row from TMEM
+//                     (tcgen05.ld), masks, and runs the base-2 online
+//                     softmax (running max m, sum l in fp32); P goes to
+//                     shared memory in the operand layout, O in TMEM is
+//                     rescaled by 2^(m_old - m_new) (tcgen05.ld / st)
+//   O += P V          tcgen05.mma (M 128 rows, N = head dim, K 128 keys),
+//                     fp32 accumulator in TMEM columns [128, 256)
+//
+// (the tiled online softmax of "昇腾CANN上的FlashAttention工程实战", with the
+// Cube / Vector split of the ops-transformer walkthrough mapped onto the
+// tensor core and the CUDA cores).  A producer warp streams K and V tiles with
+// TMA (128-byte swizzle, the canonical K-major layout for K and the
+// MN-major one for V) into a 2-stage ring; tcgen05.commit releases a stage
+// once its PV product is done.  Every wait is bounded; on a timeout the CTA
+// records the error, waits (bounded) for its last tensor-core work and frees
+// its TMEM before returning.
+#include <type_traits>
+
+#include "fa_common.cuh"
+#include "fa_internal.h"
+
+namespace fa {
+
+namespace pf {
+
+constexpr int kRows = 128;       // packed query rows per CTA (MMA M)
+constexpr int kKeys = 128;       // keys per tile (MMA N of S, K of PV)
+constexpr int kD = 128;          // head dim (both products)
+constexpr int kStages = 2;
+constexpr int kBox = kRows * 128;                   // one 64-column box of 128 rows (bytes)
+constexpr int kTile = 2 * kBox;                     // 128 rows x 128 elements
+constexpr int OFF_Q = 0;
+constexpr int OFF_P = OFF_Q + kTile;
+constexpr int OFF_KV = OFF_P + kTile;               // stage s: K at OFF_KV + s * 2 * kTile, V after it
+constexpr int OFF_BAR = OFF_KV + kStages * 2 * kTile;
+constexpr int NBAR = 2 * kStages + 3;               // full[2], empty[2], s_done, o_done, compute sync
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort flag, 4 warp maxima
+constexpr int SMEM = OFF_MISC + 64 + 1024;          // + slack to align the base to 1024 B
+constexpr int kThreads = 160;                       // 4 compute warps (TMEM lanes 0-127) + 1 producer
+constexpr uint32_t kTmemCols = 256;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+
+__device__ __forceinline__ void tma_load_4d_plain(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1,
+                                                  int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of the tcgen05 operands: 128-byte swizzle,
+// start address, leading / stride byte offsets (16-byte units), descriptor
+// version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;  // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, A and B of one
+// 16-bit type, A K-major, B K-major or MN-major, M x N.
+__device__ __forceinline__ uint32_t instr_desc(bool bf16, int M, int N, bool b_mn_major) {
+    uint32_t d = 1u << 4;  // D: fp32
+    d |= (bf16 ? 1u : 0u) << 7;
+    d |= (bf16 ? 1u : 0u) << 10;
+    d |= (b_mn_major ? 1u : 0u) << 16;
+    d |= (uint32_t)(N >> 3) << 17;
+    d |= (uint32_t)(M >> 4) << 24;
+    return d;
+}
+
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+}  // namespace pf
+
+template <typename T>
+__global__ void __launch_bounds__(pf::kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+    using namespace pf;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rb = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
+    const uint32_t s_bar = smem_u32(&bars[2 * kStages]);
+    const uint32_t o_bar = smem_u32(&bars[2 * kStages + 1]);
+    const uint32_t cs_bar = smem_u32(&bars[2 * kStages + 2]);  // bounded sync of the 4 compute warps
+    uint32_t cs_phase = 0;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *warp_keys = reinterpret_cast<int *>(smem + OFF_MISC + 16);
+
+    // ---- this thread's row (compute warps): head, query position, last visible key
+    const int r = rb * kRows + tid;  // packed row
+    const bool row_live = tid < kRows && r < p.R;
+    const int hq = row_live ? hkv * p.g + r / p.Lq : 0;
+    const int qi = row_live ? r % p.Lq : 0;
+    const int n = p.Lk;
+    int lim = -1;  // last visible key of the row
+    if (row_live) {
+        lim = n - 1;
+        if (p.causal) {
+            const int c = qi + n - p.Lq;
+            lim = c < lim ? c : lim;
+        }
+    }
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(s_bar, 1);
+        mbar_init(o_bar, 1);
+        mbar_init(cs_bar, 4);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {  // TMEM: S in columns [0, 128), O in [128, 256)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // keys the block's rows can see (tiles to walk)
+    {
+        int kv = lim + 1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kv = max(kv, __shfl_xor_sync(0xffffffffu, kv, off));
+        if (lane == 0 && warp < 4) warp_keys[warp] = kv;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int kmax = max(max(warp_keys[0], warp_keys[1]), max(warp_keys[2], warp_keys[3]));
+    const int ntiles = (kmax + kKeys - 1) / kKeys;
+
+    pdl_wait_primary();
+
+    if (warp == 4) {
+        // ================================================= producer: K / V tiles by TMA
+        if (lane == 0) {
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j % kStages, use = j / kStages;
+                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
+                const uint32_t kd = sb + OFF_KV + s * 2 * kTile, vd = kd + kTile;
+                mbar_expect_tx(full_bar(s), 2 * kTile);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_4d_plain(kd + c * kBox, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
+                    tma_load_4d_plain(vd + c * kBox, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
+                }
+                mbar_arrive(full_bar(s));
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================================================= compute warps: one row per thread
+        // Q rows into the operand layout (K-major, 128-byte swizzle): row tid,
+        // 16-byte chunk c of the head dim at box c / 8, swizzled chunk (c % 8) ^ (tid % 8)
+        {
+            const T *qg = reinterpret_cast<const T *>(p.q);
+            const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
+            for (int c = 0; c < kD / 8; ++c) {
+                const uint32_t dst =
+                    sb + OFF_Q + (c >> 3) * kBox + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
+                cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            fence_proxy_async_smem();
+        }
+        constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+        const uint32_t idesc_s = instr_desc(bf16, kRows, kKeys, false);
+        const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);
+        const uint32_t t_s = tmem, t_o = tmem + kKeys;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
+        float m = -INFINITY, l = 0.f;
+        // every Q row is in shared memory
+        bool ok = consumer_sync_bounded(cs_bar, cs_phase, abort_flag, p.status, kWaitLimitNs);
+
+        for (int j = 0; j < ntiles && ok; ++j) {
+            const int s = j % kStages, use = j / kStages;
+            ok = mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            const uint32_t kb = sb + OFF_KV + s * 2 * kTile, vb = kb + kTile;
+            if (tid == 0) {  // S = Q K^T
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                    umma(t_s, smem_desc(sb + OFF_Q + off, 16, 1024), smem_desc(kb + off, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(s_bar);
+            }
+            __syncwarp();
+            ok = mbar_wait(s_bar, j & 1, abort_flag, p.status, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+
+            // ---- this row's scores, masked, base 2
+            float x[kKeys];
+#pragma unroll
+            for (int c = 0; c < kKeys / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(t_s + lane_off + c * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+            }
+            const int key0 = j * kKeys;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < kKeys; ++e) {
+                x[e] = key0 + e <= lim ? x[e] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[e]);
+            }
+            const float mn = fmaxf(m, mx);
+            const float base = mn == -INFINITY ? 0.f : mn;
+            const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
+            float sum = 0.f;
+            uint32_t pk[kKeys / 2];
+#pragma unroll
+            for (int e = 0; e < kKeys; e += 2) {
+                const float p0 = fast_exp2(x[e] - base), p1 = fast_exp2(x[e + 1] - base);
+                sum += p0 + p1;
+                pk[e / 2] = Mma<T>::pack(p0, p1);
+            }
+            l = l * alpha + sum;
+            m = mn;
+
+            if (j > 0) {
+                // the previous PV product is done: O may be rescaled and P rewritten
+                ok = mbar_wait(o_bar, (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int c = 0; c < kD / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(t_o + lane_off + c * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                        tmem_st32(t_o + lane_off + c * 32, v);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // ---- P row into the operand layout (keys as K, K-major, swizzled)
+#pragma unroll
+            for (int c = 0; c < kKeys / 8; ++c) {
+                const uint32_t dst = sb + OFF_P + (c >> 3) * kBox + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[c * 4]),
+                             "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (!consumer_sync_bounded(cs_bar, cs_phase, abort_flag, p.status, kWaitLimitNs)) {
+                ok = false;
+                break;
+            }
+            if (tid == 0) {  // O += P V
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    const uint32_t aoff = (kk >> 2) * kBox + (kk & 3) * 32;
+                    umma(t_o, smem_desc(sb + OFF_P + aoff, 16, 1024), smem_desc(vb + kk * 2048, kBox, 1024), idesc_o,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(o_bar);
+                umma_commit(empty_bar(s));
+            }
+            __syncwarp();
+        }
+
+        // ---- epilogue: O / l, lse
+        if (ok && ntiles > 0) {
+            ok = mbar_wait(o_bar, (ntiles - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        if (ok) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            T *og = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)qi * p.o_sl + (long long)hq * p.o_sh;
+#pragma unroll
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t v[32];
+                if (ntiles > 0) {
+                    tmem_ld32(t_o + lane_off + c * 32, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                if (row_live) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(v[e + z]) * inv;
+                        store_row8<T>(og + c * 32 + e, f);
+                    }
+                }
+            }
+            if (row_live && p.lse)
+                p.lse[b * p.lse_sb + hq * p.lse_sh + qi] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        } else if (tid == 0) {
+            // timed out: wait (bounded) for the tensor core's last work before TMEM is freed
+            volatile int no_abort = 0;
+            mbar_wait(o_bar, 0, &no_abort, nullptr, kWaitLimitNs / 8);
+            mbar_wait(o_bar, 1, &no_abort, nullptr, kWaitLimitNs / 8);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
+template <typename T>
+static void fill(KernelInfo *out) {
+    out->fn = reinterpret_cast<const void *>(&prefill_kernel<T>);
+    out->threads = pf::kThreads;
+    out->smem = pf::SMEM;
+    out->tile_keys = pf::kKeys;
+    out->stages = pf::kStages;
+    out->variant = 3;  // FA_VARIANT_TCGEN05
+}
+
+bool get_prefill_kernel(int dtype, int dqk, int dv, KernelInfo *out) {
+    if (dqk != 128 || dv != 128) return false;
+    if (dtype == 0) {
+        fill<__half>(out);
+        return true;
+    }
+    if (dtype == 1) {
+        fill<__nv_bfloat16>(out);
+        return true;
+    }
+    return false;
+}
+
+}  // namespace fa

@@ -82,6 +82,11 @@ WORKLOADS["gqa_decode_hd256_bf16"] = Workload(
     "gqa_decode_hd256_bf16", "fwd", "blhd", torch.bfloat16, B=8, Lq=1, Hq=16, Hkv=4, Lk=8192, Dqk=256, Dv=256,
     causal=False, seed=1006, description="GQA decode bf16 B8 Hq16 Hkv4 D256 kvLen8192, non-causal")
 
+# Long prefill (the tcgen05 kernel): GQA 4, 4K queries over 4K keys, causal.
+WORKLOADS["gqa_prefill4k_bf16"] = Workload(
+    "gqa_prefill4k_bf16", "fwd", "blhd", torch.bfloat16, B=1, Lq=4096, Hq=32, Hkv=8, Lk=4096, Dqk=128, Dv=128,
+    causal=True, seed=1007, description="prefill bf16 B1 Lq4096 Hq32 Hkv8 D128 Lk4096, causal (tcgen05 kernel)")
+
 # the workload the bench reports by default (single-row decode over a 4K context)
 DEFAULT_BENCH = "decode_hld_fp16"
 
@@ -185,6 +190,23 @@ def kv_bytes(w: Workload, seqlens=None) -> int:
     else:
         total = w.B * w.Lk
     return total * w.Hkv * (w.Dqk + w.Dv) * elt
+
+
+def attn_flops(w: Workload, seqlens=None) -> int:
+    """Multiply-add flops of one call, 2 * (Dqk + Dv) per visible (row, key)
+    pair: every query row of every head against the keys it sees (all n
+    keys, or j <= i + n - Lq under the bottom-right causal mask)."""
+    if w.call in ("kvcache", "paged"):
+        ns = [int(x) for x in torch.as_tensor(seqlens).tolist()]
+    else:
+        ns = [w.Lk] * w.B
+    vis = 0
+    for n in ns:
+        if w.causal:
+            vis += sum(max(0, min(n, i + n - w.Lq + 1)) for i in range(w.Lq))
+        else:
+            vis += n * w.Lq
+    return 2 * (w.Dqk + w.Dv) * vis * w.Hq
 
 
 def tokens_per_call(w: Workload) -> int:

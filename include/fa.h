@@ -88,7 +88,12 @@ typedef struct fa_tensor {
 } fa_tensor;
 
 /* Which kernels the calling thread's last compute call launched. */
-typedef enum fa_variant { FA_VARIANT_AUTO = 0, FA_VARIANT_MMA = 1, FA_VARIANT_SCALAR = 2 } fa_variant;
+typedef enum fa_variant {
+    FA_VARIANT_AUTO = 0,
+    FA_VARIANT_MMA = 1,     /* split-KV kernel, mma.sync tensor-core products */
+    FA_VARIANT_SCALAR = 2,  /* split-KV kernel, fp32 FMA products (one packed row) */
+    FA_VARIANT_TCGEN05 = 3  /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 128/128) */
+} fa_variant;
 
 typedef struct fa_dispatch_info {
     int32_t variant;          /* fa_variant of the main kernel */
@@ -274,10 +279,15 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      (g * Lq == 1), the "scalar fp32 dot product" form of
  *                      "SmallQ FlashAttention for Ascend 910B", section
  *                      "算法要点".
- * The library's own choice is FA_VARIANT_MMA for every shape: measured on
- * B200 it is faster than the FMA variant even for one packed row.  A forced
- * variant that does not support the call's shapes makes the call fail with
- * FA_ERR_UNSUPPORTED.
+ *   FA_VARIANT_TCGEN05 one CTA per 128 packed query rows on the 5th-gen tensor
+ *                      cores (tcgen05.mma, accumulators in TMEM), whole key
+ *                      range per CTA, no split and no combine; dense fa_fwd
+ *                      calls with head dims 128/128.
+ * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
+ * least 128 packed rows (g * Lq >= 128) and head dims 128/128 (prefill-shaped
+ * calls); FA_VARIANT_MMA otherwise -- measured on B200 it is faster than the
+ * FMA variant even for one packed row.  A forced variant that does not
+ * support the call's shapes makes the call fail with FA_ERR_UNSUPPORTED.
  */
 FA_API fa_status fa_force_variant(int variant);
 

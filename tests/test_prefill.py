@@ -1,0 +1,74 @@
+"""GPU parity of the tcgen05 kernel (dense fa_fwd with >= 128 packed rows,
+head dims 128/128) against the oracle: ragged query and key lengths, causal
+bottom-right alignment including rows with no visible key, GQA packing,
+fp16 / bf16, several batches; full-size prefill on sampled rows."""
+import numpy as np
+import pytest
+import torch
+
+import decode_flashattention_b200 as fa
+import oracle
+from decode_flashattention_b200 import workloads as wl
+
+from helpers import compare, o_to_numpy, lse_to_numpy, oracle_full
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _reset():
+    yield
+    fa.force_variant(fa.VARIANT_AUTO)
+    torch.cuda.synchronize()
+    fa.check_status()
+
+
+CASES = [  # B, Lq, Hq, Hkv, Lk, causal
+    (1, 128, 1, 1, 128, False), (1, 129, 1, 1, 1, False), (2, 300, 2, 1, 700, True), (1, 1000, 4, 4, 1000, True),
+    (3, 64, 8, 4, 257, False), (1, 32, 8, 2, 128, True), (1, 1, 128, 1, 3000, False), (1, 500, 2, 2, 200, True),
+    (1, 257, 16, 2, 129, True), (2, 160, 4, 1, 4000, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(c) for c in CASES])
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_tcgen05_parity(case, dt):
+    B, Lq, Hq, Hkv, Lk, causal = case
+    w = wl.Workload("pf", "fwd", "blhd", dt, B=B, Lq=Lq, Hq=Hq, Hkv=Hkv, Lk=Lk, Dqk=128, Dv=128, causal=causal,
+                    seed=Lq + Lk)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    o, lse = fa.fa_fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.last_dispatch()["variant"] == fa.VARIANT_TCGEN05
+    ro, rl = oracle_full(q, k, v, causal)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, "tcgen05")
+
+
+def test_forced_on_fewer_rows_and_refused_for_caches():
+    w = wl.Workload("pf2", "fwd", "blhd", torch.bfloat16, B=2, Lq=3, Hq=2, Hkv=2, Lk=300, Dqk=128, Dv=128,
+                    causal=True, seed=4)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)
+    o, lse = fa.fa_fwd(q, k, v, causal=True)  # 6 rows in a 128-row tile: the rest is padding
+    torch.cuda.synchronize()
+    ro, rl = oracle_full(q, k, v, True)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, torch.bfloat16, "tcgen05 forced")
+    sl = torch.tensor([10, 300], dtype=torch.int32, device=DEV)
+    with pytest.raises(fa.FaError, match="tcgen05"):
+        fa.fa_decode_kvcache(q, k, v, sl)
+
+
+def test_full_size_prefill_sampled_rows():
+    w = wl.WORKLOADS["gqa_prefill4k_bf16"]
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    o, lse = fa.fa_fwd(q, k, v, causal=w.causal)
+    torch.cuda.synchronize()
+    assert fa.last_dispatch()["variant"] == fa.VARIANT_TCGEN05
+    rng = np.random.default_rng(0)
+    rows = np.stack([rng.integers(0, w.B, 48), rng.integers(0, w.Hq, 48), rng.integers(0, w.Lq, 48)], 1)
+    ro, rl = oracle.attention(q.cpu(), k.cpu(), v.cpu(), causal=w.causal, rows=rows)
+    got_o = o.float().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
+    got_l = lse.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    compare(got_o, got_l, ro, rl, w.dtype, "prefill 4k")
