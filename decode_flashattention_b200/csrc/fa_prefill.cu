@@ -7,14 +7,16 @@
 // K / V tile.  The CTA walks all key tiles its rows can see (128 keys each):
 //
 //   S  = Q K^T        tcgen05.mma (M 128 rows, N 128 keys, K = head dim),
-//                     fp32 accumulator in TMEM columns [0, 128)
+//                     fp32 accumulator in TMEM, two buffers: the next
+//                     tile's S is computed while this tile's softmax runs
 //   softmax           one thread per row reads its S row from TMEM
 //                     (tcgen05.ld), masks, and runs the base-2 online
 //                     softmax (running max m, sum l in fp32); P goes to
 //                     shared memory in the operand layout, O in TMEM is
 //                     rescaled by 2^(m_old - m_new) (tcgen05.ld / st)
 //   O += P V          tcgen05.mma (M 128 rows, N = head dim, K 128 keys),
-//                     fp32 accumulator in TMEM columns [128, 256)
+//                     fp32 accumulator in TMEM (it runs while the next
+//                     tile's softmax starts)
 //
 // (the tiled online softmax of "昇腾CANN上的FlashAttention工程实战", with the
 // Cube / Vector split of the ops-transformer walkthrough mapped onto the
@@ -43,11 +45,11 @@ constexpr int OFF_Q = 0;
 constexpr int OFF_P = OFF_Q + kTile;
 constexpr int OFF_KV = OFF_P + kTile;               // stage s: K at OFF_KV + s * 2 * kTile, V after it
 constexpr int OFF_BAR = OFF_KV + kStages * 2 * kTile;
-constexpr int NBAR = 2 * kStages + 3;               // full[2], empty[2], s_done, o_done, compute sync
+constexpr int NBAR = 2 * kStages + 4;               // full[2], empty[2], s_done[2], o_done, compute sync
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort flag, 4 warp maxima
 constexpr int SMEM = OFF_MISC + 64 + 1024;          // + slack to align the base to 1024 B
 constexpr int kThreads = 160;                       // 4 compute warps (TMEM lanes 0-127) + 1 producer
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;  // S double buffer [0, 256), O [256, 384)
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
 
@@ -143,9 +145,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
-    const uint32_t s_bar = smem_u32(&bars[2 * kStages]);
-    const uint32_t o_bar = smem_u32(&bars[2 * kStages + 1]);
-    const uint32_t cs_bar = smem_u32(&bars[2 * kStages + 2]);  // bounded sync of the 4 compute warps
+    auto s_bar = [&](int buf) { return smem_u32(&bars[2 * kStages + buf]); };
+    const uint32_t o_bar = smem_u32(&bars[2 * kStages + 2]);
+    const uint32_t cs_bar = smem_u32(&bars[2 * kStages + 3]);  // bounded sync of the 4 compute warps
     uint32_t cs_phase = 0;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
@@ -171,13 +173,14 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
-        mbar_init(s_bar, 1);
+        mbar_init(s_bar(0), 1);
+        mbar_init(s_bar(1), 1);
         mbar_init(o_bar, 1);
         mbar_init(cs_bar, 4);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {  // TMEM: S in columns [0, 128), O in [128, 256)
+    if (warp == 0) {  // TMEM: S double buffer in columns [0, 256), O in [256, 384)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(kTmemCols)
                      : "memory");
@@ -233,31 +236,45 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
         const uint32_t idesc_s = instr_desc(bf16, kRows, kKeys, false);
         const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);
-        const uint32_t t_s = tmem, t_o = tmem + kKeys;
+        const uint32_t t_o = tmem + 2 * kKeys;  // S buffers at tmem, tmem + kKeys
+        // S_jj = Q K_jj^T into S buffer jj % 2, issued by one thread once tile jj
+        // has landed (issue_s_ready: the caller knows it has).
+        auto issue_s_ready = [&](int jj) -> bool {
+            const int st = jj % kStages;
+            const uint32_t kbase = sb + OFF_KV + st * 2 * kTile;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
+                umma(tmem + (jj & 1) * kKeys, smem_desc(sb + OFF_Q + off, 16, 1024), smem_desc(kbase + off, 16, 1024),
+                     idesc_s, kk > 0);
+            }
+            umma_commit(s_bar(jj & 1));
+            return true;
+        };
+        auto issue_s = [&](int jj) -> bool {
+            const int st = jj % kStages;
+            if (!mbar_wait(full_bar(st), (jj / kStages) & 1, abort_flag, p.status, kWaitLimitNs)) return false;
+            return issue_s_ready(jj);
+        };
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
         float m = -INFINITY, l = 0.f;
         // every Q row is in shared memory
         bool ok = consumer_sync_bounded(cs_bar, cs_phase, abort_flag, p.status, kWaitLimitNs);
+        if (ok && tid == 0 && ntiles > 0) ok = issue_s(0);
 
         for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kStages, use = j / kStages;
-            ok = mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) {
-                ok = false;
-                break;
-            }
-            const uint32_t kb = sb + OFF_KV + s * 2 * kTile, vb = kb + kTile;
-            if (tid == 0) {  // S = Q K^T
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                    umma(t_s, smem_desc(sb + OFF_Q + off, 16, 1024), smem_desc(kb + off, 16, 1024), idesc_s, kk > 0);
-                }
-                umma_commit(s_bar);
+            const int s = j % kStages;
+            const uint32_t vb = sb + OFF_KV + s * 2 * kTile + kTile;
+            // the next tile's S now if its K has landed, else just before this tile's PV
+            bool next_issued = false;
+            if (tid == 0 && j + 1 < ntiles &&
+                mbar_try_wait(full_bar((j + 1) % kStages), ((j + 1) / kStages) & 1)) {
+                ok = issue_s_ready(j + 1);
+                next_issued = true;
             }
             __syncwarp();
-            ok = mbar_wait(s_bar, j & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = mbar_wait(s_bar(j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs) && ok;
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -269,7 +286,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
             for (int c = 0; c < kKeys / 32; ++c) {
                 uint32_t v[32];
-                tmem_ld32(t_s + lane_off + c * 32, v);
+                tmem_ld32(tmem + (j & 1) * kKeys + lane_off + c * 32, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
@@ -330,6 +347,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                 ok = false;
                 break;
             }
+            if (tid == 0 && j + 1 < ntiles && !next_issued) ok = issue_s(j + 1) && ok;
             if (tid == 0) {  // O += P V
                 tc_fence_after();
 #pragma unroll
