@@ -281,34 +281,53 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             }
             tc_fence_after();
 
-            // ---- this row's scores, masked, base 2
+            // ---- this row's scores (raw fp32): the four TMEM loads in flight at once
+            uint32_t v0[32], v1[32], v2[32], v3[32];
+            {
+                const uint32_t ts = tmem + (j & 1) * kKeys + lane_off;
+                tmem_ld32(ts, v0);
+                tmem_ld32(ts + 32, v1);
+                tmem_ld32(ts + 64, v2);
+                tmem_ld32(ts + 96, v3);
+                tmem_wait_ld();
+            }
             float x[kKeys];
 #pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tmem + (j & 1) * kKeys + lane_off + c * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+            for (int e = 0; e < 32; ++e) {
+                x[e] = __uint_as_float(v0[e]);
+                x[32 + e] = __uint_as_float(v1[e]);
+                x[64 + e] = __uint_as_float(v2[e]);
+                x[96 + e] = __uint_as_float(v3[e]);
             }
+            // mask only where some row of the warp has keys of this tile hidden
             const int key0 = j * kKeys;
-            float mx = -INFINITY;
+            if (!__all_sync(0xffffffffu, key0 + kKeys - 1 <= lim)) {
 #pragma unroll
-            for (int e = 0; e < kKeys; ++e) {
-                x[e] = key0 + e <= lim ? x[e] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[e]);
+                for (int e = 0; e < kKeys; ++e) x[e] = key0 + e <= lim ? x[e] : -INFINITY;
             }
+            // row max with independent chains, in base-2 units (scale > 0)
+            float mxa[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxa[e] = x[e];
+#pragma unroll
+            for (int e = 8; e < kKeys; ++e) mxa[e & 7] = fmaxf(mxa[e & 7], x[e]);
+            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
+                             p.scale_log2;
             const float mn = fmaxf(m, mx);
             const float base = mn == -INFINITY ? 0.f : mn;
             const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
-            float sum = 0.f;
+            // p = 2^(x * scale_log2 - base): one FFMA and one ex2 per score
+            float suma[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             uint32_t pk[kKeys / 2];
 #pragma unroll
             for (int e = 0; e < kKeys; e += 2) {
-                const float p0 = fast_exp2(x[e] - base), p1 = fast_exp2(x[e + 1] - base);
-                sum += p0 + p1;
+                const float p0 = fast_exp2(fmaf(x[e], p.scale_log2, -base));
+                const float p1 = fast_exp2(fmaf(x[e + 1], p.scale_log2, -base));
+                suma[(e >> 1) & 7] += p0 + p1;
                 pk[e / 2] = Mma<T>::pack(p0, p1);
             }
+            const float sum = ((suma[0] + suma[1]) + (suma[2] + suma[3])) + ((suma[4] + suma[5]) + (suma[6] + suma[7]));
             l = l * alpha + sum;
             m = mn;
 
@@ -321,15 +340,23 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                 }
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                    const uint32_t to = t_o + lane_off;
+                    tmem_ld32(to, v0);
+                    tmem_ld32(to + 32, v1);
+                    tmem_ld32(to + 64, v2);
+                    tmem_ld32(to + 96, v3);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < kD / 32; ++c) {
-                        uint32_t v[32];
-                        tmem_ld32(t_o + lane_off + c * 32, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tmem_st32(t_o + lane_off + c * 32, v);
+                    for (int e = 0; e < 32; ++e) {
+                        v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                        v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                        v2[e] = __float_as_uint(__uint_as_float(v2[e]) * alpha);
+                        v3[e] = __float_as_uint(__uint_as_float(v3[e]) * alpha);
                     }
+                    tmem_st32(to, v0);
+                    tmem_st32(to + 32, v1);
+                    tmem_st32(to + 64, v2);
+                    tmem_st32(to + 96, v3);
                     tmem_wait_st();
                 }
             }
