@@ -916,6 +916,9 @@ fa_status fa_check_status(void *stream) {
     if (v) {
         unsigned zero = 0;
         cudaMemcpy(dev->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (v & fa::kStatusLayout)
+            return fail(FA_ERR_CUDA, "a kernel found its shared-memory base misaligned and wrote nothing (status 0x%x)",
+                        v);
         return fail(FA_ERR_TIMEOUT, "a kernel gave up waiting on its copy pipeline (status 0x%x)", v);
     }
     t_err.clear();

@@ -19,6 +19,7 @@ constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
 constexpr int kMaxPrefixEntries = 8192;              // B * row-blocks bound
 constexpr unsigned kStatusTimeout = 1u;
+constexpr unsigned kStatusLayout = 2u;  // a kernel found its shared-memory base misaligned and did nothing
 
 struct Params {
     const void *q;  // [B, Lq, Hq, Dqk]

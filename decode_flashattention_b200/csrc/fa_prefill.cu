@@ -36,22 +36,39 @@ namespace fa {
 namespace pf {
 
 constexpr int kRows = 128;       // packed query rows per CTA (MMA M)
-constexpr int kKeys = 128;       // keys per tile (MMA N of S, K of PV)
 constexpr int kD = 128;          // head dim (both products)
 constexpr int kStages = 2;
-constexpr int kBox = kRows * 128;                   // one 64-column box of 128 rows (bytes)
-constexpr int kTile = 2 * kBox;                     // 128 rows x 128 elements
-constexpr int OFF_Q = 0;
-constexpr int OFF_P = OFF_Q + kTile;
-constexpr int OFF_KV = OFF_P + kTile;               // stage s: K at OFF_KV + s * 2 * kTile, V after it
-constexpr int OFF_BAR = OFF_KV + kStages * 2 * kTile;
+constexpr int kBoxQ = kRows * 128;                  // one 64-column box of 128 rows (bytes): Q and P
+constexpr int kTileQ = 2 * kBoxQ;                   // Q: 128 rows x 128 elements
 constexpr int NBAR = 2 * kStages + 4;               // full[2], empty[2], s_done[2], o_done, compute sync
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;        // tmem base, abort flag, 4 warp maxima
-constexpr int SMEM = OFF_MISC + 64 + 1024;          // + slack to align the base to 1024 B
 constexpr int kThreads = 160;                       // 4 compute warps (TMEM lanes 0-127) + 1 producer
-constexpr uint32_t kTmemCols = 512;  // S double buffer [0, 256), O [256, 384)
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
-static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+
+// Shared-memory layout for KEYS keys per tile.  KEYS = 128: one CTA per SM,
+// a 2-stage ring of 64 KB K + V stages, S double-buffered in TMEM (512 columns).
+// KEYS = 64: half the stage and P sizes, so two CTAs share an SM (their
+// softmax warps interleave on each sub-partition), 256 TMEM columns each; the
+// base must then already be 1024-byte aligned (checked at run time) since
+// there is no room for alignment slack.
+template <int KEYS>
+struct Cfg {
+    static constexpr int kKeys = KEYS;
+    static constexpr int kBoxKV = KEYS * 128;         // one 64-column box of K or V (bytes)
+    static constexpr int kTileKV = 2 * kBoxKV;        // K or V tile: KEYS rows x 128 elements
+    static constexpr int kStageBytes = 2 * kTileKV;   // K + V
+    static constexpr int kPBytes = kRows * KEYS * 2;  // P: 128 rows x KEYS keys
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_P = OFF_Q + kTileQ;
+    static constexpr int OFF_KV = OFF_P + kPBytes;
+    static constexpr int OFF_BAR = OFF_KV + kStages * kStageBytes;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, 4 warp maxima
+    static constexpr int SLACK = KEYS == 128 ? 1024 : 0;
+    static constexpr int SMEM = OFF_MISC + 64 + SLACK;
+    static constexpr uint32_t kTmemCols = KEYS == 128 ? 512 : 256;  // S x 2 [0, 2 KEYS), O [2 KEYS, 2 KEYS + 128)
+    static constexpr int kMinBlocks = KEYS == 128 ? 1 : 2;
+    static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+    static_assert(KEYS == 128 || 2 * (SMEM + 1024) <= 233472, "two CTAs fit an SM");
+};
 
 __device__ __forceinline__ void tma_load_4d_plain(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1,
                                                   int c2, int c3) {
@@ -132,26 +149,32 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 
 }  // namespace pf
 
-template <typename T>
-__global__ void __launch_bounds__(pf::kThreads, 1)
+template <typename T, int KEYS>
+__global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
     using namespace pf;
+    using C = Cfg<KEYS>;
+    constexpr int kKeys = KEYS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     const uint32_t sb = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (C::SLACK == 0 && smem != smem_raw) {  // no room to align: the base must already be aligned
+        if (tid == 0) atomicOr(p.status, kStatusLayout);
+        return;
+    }
     const int rb = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
     auto s_bar = [&](int buf) { return smem_u32(&bars[2 * kStages + buf]); };
     const uint32_t o_bar = smem_u32(&bars[2 * kStages + 2]);
     const uint32_t cs_bar = smem_u32(&bars[2 * kStages + 3]);  // bounded sync of the 4 compute warps
     uint32_t cs_phase = 0;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-    int *warp_keys = reinterpret_cast<int *>(smem + OFF_MISC + 16);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
+    int *warp_keys = reinterpret_cast<int *>(smem + C::OFF_MISC + 16);
 
     // ---- this thread's row (compute warps): head, query position, last visible key
     const int r = rb * kRows + tid;  // packed row
@@ -182,7 +205,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     }
     if (warp == 0) {  // TMEM: S double buffer in columns [0, 256), O in [256, 384)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(kTmemCols)
+                     "r"(C::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -208,11 +231,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             for (int j = 0; j < ntiles; ++j) {
                 const int s = j % kStages, use = j / kStages;
                 if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
-                const uint32_t kd = sb + OFF_KV + s * 2 * kTile, vd = kd + kTile;
-                mbar_expect_tx(full_bar(s), 2 * kTile);
+                const uint32_t kd = sb + C::OFF_KV + s * C::kStageBytes, vd = kd + C::kTileKV;
+                mbar_expect_tx(full_bar(s), C::kStageBytes);
                 for (int c = 0; c < 2; ++c) {
-                    tma_load_4d_plain(kd + c * kBox, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
-                    tma_load_4d_plain(vd + c * kBox, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
+                    tma_load_4d_plain(kd + c * C::kBoxKV, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
+                    tma_load_4d_plain(vd + c * C::kBoxKV, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
                 }
                 mbar_arrive(full_bar(s));
             }
@@ -227,7 +250,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
             for (int c = 0; c < kD / 8; ++c) {
                 const uint32_t dst =
-                    sb + OFF_Q + (c >> 3) * kBox + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
+                    sb + C::OFF_Q + (c >> 3) * kBoxQ + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
                 cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
@@ -241,13 +264,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         // has landed (issue_s_ready: the caller knows it has).
         auto issue_s_ready = [&](int jj) -> bool {
             const int st = jj % kStages;
-            const uint32_t kbase = sb + OFF_KV + st * 2 * kTile;
+            const uint32_t kbase = sb + C::OFF_KV + st * C::kStageBytes;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * kBox + (kk & 3) * 32;
-                umma(tmem + (jj & 1) * kKeys, smem_desc(sb + OFF_Q + off, 16, 1024), smem_desc(kbase + off, 16, 1024),
-                     idesc_s, kk > 0);
+                const uint32_t aoff = (kk >> 2) * kBoxQ + (kk & 3) * 32, boff = (kk >> 2) * C::kBoxKV + (kk & 3) * 32;
+                umma(tmem + (jj & 1) * kKeys, smem_desc(sb + C::OFF_Q + aoff, 16, 1024),
+                     smem_desc(kbase + boff, 16, 1024), idesc_s, kk > 0);
             }
             umma_commit(s_bar(jj & 1));
             return true;
@@ -265,7 +288,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 
         for (int j = 0; j < ntiles && ok; ++j) {
             const int s = j % kStages;
-            const uint32_t vb = sb + OFF_KV + s * 2 * kTile + kTile;
+            const uint32_t vb = sb + C::OFF_KV + s * C::kStageBytes + C::kTileKV;
             // the next tile's S now if its K has landed, else just before this tile's PV
             bool next_issued = false;
             if (tid == 0 && j + 1 < ntiles &&
@@ -287,8 +310,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                 const uint32_t ts = tmem + (j & 1) * kKeys + lane_off;
                 tmem_ld32(ts, v0);
                 tmem_ld32(ts + 32, v1);
-                tmem_ld32(ts + 64, v2);
-                tmem_ld32(ts + 96, v3);
+                if constexpr (kKeys == 128) {
+                    tmem_ld32(ts + 64, v2);
+                    tmem_ld32(ts + 96, v3);
+                }
                 tmem_wait_ld();
             }
             float x[kKeys];
@@ -296,8 +321,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             for (int e = 0; e < 32; ++e) {
                 x[e] = __uint_as_float(v0[e]);
                 x[32 + e] = __uint_as_float(v1[e]);
-                x[64 + e] = __uint_as_float(v2[e]);
-                x[96 + e] = __uint_as_float(v3[e]);
+                if constexpr (kKeys == 128) {
+                    x[64 + e] = __uint_as_float(v2[e]);
+                    x[96 + e] = __uint_as_float(v3[e]);
+                }
             }
             // mask only where some row of the warp has keys of this tile hidden
             const int key0 = j * kKeys;
@@ -340,30 +367,28 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                 }
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                    const uint32_t to = t_o + lane_off;
-                    tmem_ld32(to, v0);
-                    tmem_ld32(to + 32, v1);
-                    tmem_ld32(to + 64, v2);
-                    tmem_ld32(to + 96, v3);
-                    tmem_wait_ld();
+                    // O row in 64-column halves (fewer live registers with two CTAs per SM)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
-                        v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
-                        v2[e] = __float_as_uint(__uint_as_float(v2[e]) * alpha);
-                        v3[e] = __float_as_uint(__uint_as_float(v3[e]) * alpha);
+                    for (int h = 0; h < kD / 64; ++h) {
+                        const uint32_t to = t_o + lane_off + h * 64;
+                        tmem_ld32(to, v0);
+                        tmem_ld32(to + 32, v1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                            v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                        }
+                        tmem_st32(to, v0);
+                        tmem_st32(to + 32, v1);
                     }
-                    tmem_st32(to, v0);
-                    tmem_st32(to + 32, v1);
-                    tmem_st32(to + 64, v2);
-                    tmem_st32(to + 96, v3);
                     tmem_wait_st();
                 }
             }
             // ---- P row into the operand layout (keys as K, K-major, swizzled)
 #pragma unroll
             for (int c = 0; c < kKeys / 8; ++c) {
-                const uint32_t dst = sb + OFF_P + (c >> 3) * kBox + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
+                const uint32_t dst = sb + C::OFF_P + (c >> 3) * kBoxQ + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
                 asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[c * 4]),
                              "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
                              : "memory");
@@ -379,9 +404,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kBox + (kk & 3) * 32;
-                    umma(t_o, smem_desc(sb + OFF_P + aoff, 16, 1024), smem_desc(vb + kk * 2048, kBox, 1024), idesc_o,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+                    const uint32_t aoff = (kk >> 2) * kBoxQ + (kk & 3) * 32;
+                    umma(t_o, smem_desc(sb + C::OFF_P + aoff, 16, 1024), smem_desc(vb + kk * 2048, C::kBoxKV, 1024),
+                         idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(o_bar);
                 umma_commit(empty_bar(s));
@@ -431,28 +456,33 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols) : "memory");
     }
 }
 
-template <typename T>
+template <typename T, int KEYS>
 static void fill(KernelInfo *out) {
-    out->fn = reinterpret_cast<const void *>(&prefill_kernel<T>);
+    out->fn = reinterpret_cast<const void *>(&prefill_kernel<T, KEYS>);
     out->threads = pf::kThreads;
-    out->smem = pf::SMEM;
-    out->tile_keys = pf::kKeys;
+    out->smem = pf::Cfg<KEYS>::SMEM;
+    out->tile_keys = KEYS;
     out->stages = pf::kStages;
     out->variant = 3;  // FA_VARIANT_TCGEN05
 }
 
+// 128-key tiles, one CTA per SM.  (64-key tiles with two CTAs per SM measured
+// the same on a 4K causal prefill -- 332 vs 334 us -- the doubled per-tile
+// overhead cancelling the second CTA's interleaving.)
+constexpr int kPrefillKeys = 128;
+
 bool get_prefill_kernel(int dtype, int dqk, int dv, KernelInfo *out) {
     if (dqk != 128 || dv != 128) return false;
     if (dtype == 0) {
-        fill<__half>(out);
+        fill<__half, kPrefillKeys>(out);
         return true;
     }
     if (dtype == 1) {
-        fill<__nv_bfloat16>(out);
+        fill<__nv_bfloat16, kPrefillKeys>(out);
         return true;
     }
     return false;
