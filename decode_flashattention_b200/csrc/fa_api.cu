@@ -252,7 +252,7 @@ struct Plan {
     int comb_smem;
     int comb_grid;
     bool prefill = false;  // the tcgen05 kernel: one CTA per (block of 128 rows, kv head, batch), no combine
-    int rb128 = 0;
+    int row_blocks = 0;
 };
 
 // The tensor-core variant puts the keys on the MMA's 16-row side, so even one
@@ -314,12 +314,14 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     if (variant == FA_VARIANT_TCGEN05 || (g_force_variant.load() == FA_VARIANT_AUTO && tc_shape)) {
         if (!tc_shape && (kvcache || s.Dqk != 128 || s.Dv != 128))
             return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 128/128");
-        if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, &pl->main))
+        // two 128-row tiles per CTA once there is more than one tile of rows
+        const int form = s.R > 128 ? 1 : 0;
+        if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, form, &pl->main))
             return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d", s.dtype);
         if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
         pl->prefill = true;
-        pl->rb128 = (s.R + 127) / 128;
-        pl->P = (int)std::min<int64_t>((int64_t)pl->rb128 * s.Hkv * s.B, INT32_MAX);
+        pl->row_blocks = (s.R + pl->main.rows - 1) / pl->main.rows;
+        pl->P = (int)std::min<int64_t>((int64_t)pl->row_blocks * s.Hkv * s.B, INT32_MAX);
         pl->P_param = pl->P;
         pl->min_share = 0;
         pl->W = -1;
@@ -327,7 +329,7 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
         pl->pieces = 0;
         pl->ws_o_off = pl->ws_lse_off = pl->ws_bytes = 0;
         pl->comb_smem = pl->comb_grid = 0;
-        if (pl->rb128 > 65535 * 16 || s.Hkv > 65535 || s.B > 65535)
+        if (pl->row_blocks > 65535 * 16 || s.Hkv > 65535 || s.B > 65535)
             return fail(FA_ERR_UNSUPPORTED, "grid too large for the tcgen05 variant");
         return FA_OK;
     }
@@ -588,7 +590,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
         if ((st = encode_kv_map(k, pl.main.tile_keys, &tmK, "k"))) return st;
         if ((st = encode_kv_map(v, pl.main.tile_keys, &tmV, "v"))) return st;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)pl.rb128, (unsigned)s.Hkv, (unsigned)s.B);
+        cfg.gridDim = dim3((unsigned)pl.row_blocks, (unsigned)s.Hkv, (unsigned)s.B);
         cfg.blockDim = dim3((unsigned)pl.main.threads);
         cfg.dynamicSmemBytes = (size_t)pl.main.smem;
         cfg.stream = stream;
@@ -661,7 +663,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     d.smem_bytes = pl.main.smem;
     d.tile_keys = pl.main.tile_keys;
     d.stages = pl.main.stages;
-    d.rows_per_cta = pl.prefill ? 128 : fa::kRowsPerCta;
+    d.rows_per_cta = pl.prefill ? pl.main.rows : fa::kRowsPerCta;
     d.units = (int)((int64_t)s.B * s.RB * s.Hkv);
     d.min_share_tiles = pl.min_share;
     d.combine_launched = pl.need_combine ? 1 : 0;

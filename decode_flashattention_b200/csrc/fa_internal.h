@@ -13,6 +13,7 @@ struct KernelInfo {
     int tile_keys;   // keys per pipeline stage (main kernels)
     int stages;      // pipeline depth (main kernels)
     int variant;     // fa_variant
+    int rows;        // packed query rows per CTA (tcgen05 kernels)
 };
 
 // Main split-KV kernel using mma.sync (keys as M, packed rows as N).
@@ -21,7 +22,8 @@ bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
 
 // Dense attention on tcgen05 for calls with many packed rows (fa_prefill.cu).
-bool get_prefill_kernel(int dtype, int dqk, int dv, KernelInfo *out);
+// form 0: one 128-row tile per CTA; form 1: two 128-row tiles per CTA.
+bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out);
 
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);

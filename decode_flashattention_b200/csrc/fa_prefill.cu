@@ -26,6 +26,10 @@
 // once its PV product is done.  Every wait is bounded; on a timeout the CTA
 // records the error, waits (bounded) for its last tensor-core work and frees
 // its TMEM before returning.
+//
+// A second form (prefill2_kernel) puts two 128-row query tiles in one CTA with
+// a dedicated MMA warp, so the softmax of one tile overlaps the other tile's
+// products and two softmax warps share each sub-partition.
 #include <type_traits>
 
 #include "fa_common.cuh"
@@ -460,6 +464,359 @@ __global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (256 packed rows), used once a call has more than
+// one tile of rows.  Softmax group g (warps 2 + 4g .. 5 + 4g, one row per
+// thread; a warp reaches TMEM lanes 32 (w % 4) .. +31, so each sub-partition
+// runs one warp of each group) owns tile g.  One MMA thread issues, per
+// 64-key K / V tile j,
+//   S_A(j), S_B(j)          once tile j has landed (early, while the groups
+//                           still run the softmax of tile j - 1, when it can),
+//   PV_A(j), PV_B(j)        each once its group has written P(j),
+// so the tensor core works on one group's products while the two groups'
+// softmax warps interleave on every sub-partition.  S is double-buffered per
+// group, P has one 16 KB buffer per group in shared memory, O accumulates in
+// TMEM.  TMEM columns: S_A [0, 128), S_B [128, 256), O_A [256, 384),
+// O_B [384, 512).  K / V stream in a ring of 32 KB stages, each released by a
+// tcgen05.commit after both PV products of its tile.
+namespace pf2 {
+constexpr int kKeys = 64;
+constexpr int kRing = 4;
+constexpr int kBoxKV = kKeys * 128;              // one 64-column box of K or V (bytes)
+constexpr int kTileKV = 2 * kBoxKV;              // 64 keys x 128 elements
+constexpr int kStageBytes = 2 * kTileKV;         // K + V: 32 KB
+constexpr int kPBytes = pf::kRows * kKeys * 2;   // 128 rows x 64 keys: one box
+constexpr int OFF_Q = 0;                         // Q_A, Q_B
+constexpr int OFF_P = OFF_Q + 2 * pf::kTileQ;    // P_A, P_B
+constexpr int OFF_KV = OFF_P + 2 * kPBytes;
+constexpr int OFF_BAR = OFF_KV + kRing * kStageBytes;
+// full[kRing], empty[kRing], s_done[2 groups][2 buffers], p_ready[2], o_done[2], q_ready, drain
+constexpr int NBAR = 2 * kRing + 4 + 2 + 2 + 2;
+constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base, abort flag, 8 warp maxima
+constexpr int SMEM = OFF_MISC + 64 + 1024;       // + alignment slack
+constexpr int kThreads = 320;                    // an MMA warp, a producer warp, 8 softmax warps
+// The MMA warp is warp 0: a warp scheduler that keeps issuing from one ready
+// warp falls back to the oldest one when it stalls, so the MMA thread gets an
+// issue slot at each softmax stall instead of waiting behind the softmax
+// warps' arithmetic bursts on its sub-partition.
+constexpr int kMmaWarp = 0, kProducerWarp = 1, kFirstSoftmaxWarp = 2;
+constexpr int kCtaRows = 2 * pf::kRows;
+constexpr uint32_t kTmemCols = 512;
+static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+}  // namespace pf2
+
+template <typename T>
+__global__ void __launch_bounds__(pf2::kThreads, 1)
+    prefill2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+    using namespace pf;
+    using namespace pf2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~static_cast<uintptr_t>(1023));
+    const uint32_t sb = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // row blocks in reverse order: under a causal mask the late rows see the
+    // most keys, so the longest CTAs start first
+    const int rb = gridDim.x - 1 - blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty_bar = [&](int s) { return smem_u32(&bars[kRing + s]); };
+    auto s_bar = [&](int g, int buf) { return smem_u32(&bars[2 * kRing + 2 * g + buf]); };
+    auto p_bar = [&](int g) { return smem_u32(&bars[2 * kRing + 4 + g]); };
+    auto o_bar = [&](int g) { return smem_u32(&bars[2 * kRing + 6 + g]); };
+    const uint32_t q_bar = smem_u32(&bars[2 * kRing + 8]);
+    const uint32_t drain_bar = smem_u32(&bars[2 * kRing + 9]);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    int *warp_keys = reinterpret_cast<int *>(smem + OFF_MISC + 16);
+
+    // ---- softmax threads: group, row, head, query position, last visible key
+    const bool softmax = warp >= kFirstSoftmaxWarp;
+    const int grp = ((warp - kFirstSoftmaxWarp) >> 2) & 1, quarter = warp & 3;  // TMEM lanes 32 (warp % 4) ..
+    const int trow = quarter * 32 + lane;  // row within the group's tile = TMEM lane
+    const int r = rb * kCtaRows + grp * kRows + trow;
+    const bool row_live = softmax && r < p.R;
+    const int hq = row_live ? hkv * p.g + r / p.Lq : 0;
+    const int qi = row_live ? r % p.Lq : 0;
+    const int n = p.Lk;
+    int lim = -1;
+    if (row_live) {
+        lim = n - 1;
+        if (p.causal) {
+            const int c = qi + n - p.Lq;
+            lim = c < lim ? c : lim;
+        }
+    }
+    if (tid == 0) {
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(s_bar(g, 0), 1);
+            mbar_init(s_bar(g, 1), 1);
+            mbar_init(p_bar(g), 4);  // one arrival per softmax warp of the group
+            mbar_init(o_bar(g), 1);
+        }
+        mbar_init(q_bar, 8);  // one arrival per softmax warp
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    {
+        int kv = lim + 1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kv = max(kv, __shfl_xor_sync(0xffffffffu, kv, off));
+        if (lane == 0 && softmax) warp_keys[warp - kFirstSoftmaxWarp] = kv;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    int kmax = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) kmax = max(kmax, warp_keys[w]);
+    const int ntiles = (kmax + kKeys - 1) / kKeys;
+    constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+
+    pdl_wait_primary();
+
+    if (warp == kProducerWarp) {
+        // ================================================= producer: K / V tiles by TMA
+        if (lane == 0) {
+            int issued = 0;
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j % kRing, use = j / kRing;
+                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
+                const uint32_t kd = sb + OFF_KV + s * kStageBytes, vd = kd + kTileKV;
+                mbar_expect_tx(full_bar(s), kStageBytes);
+                for (int c = 0; c < 2; ++c) {
+                    tma_load_4d_plain(kd + c * kBoxKV, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
+                    tma_load_4d_plain(vd + c * kBoxKV, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
+                }
+                mbar_arrive(full_bar(s));
+                issued = j + 1;
+            }
+            if (*abort_flag) {
+                // let the copies still in flight land before the CTA's shared memory is released
+                volatile int no_abort = 0;
+                for (int j = issued - kRing < 0 ? 0 : issued - kRing; j < issued; ++j)
+                    mbar_wait(full_bar(j % kRing), (j / kRing) & 1, &no_abort, nullptr, kWaitLimitNs / 16);
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ================================================= MMA issue (one thread)
+        if (lane == 0) {
+            const uint32_t idesc_s = instr_desc(bf16, kRows, kKeys, false);
+            const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);
+            // Every operand descriptor is a base descriptor plus a constant
+            // offset (16-byte units in the low bits; all shared addresses stay
+            // below 256 KB, so the sum never carries out of the address field).
+            // Computing them ahead keeps the issue loop to the MMAs themselves:
+            // a tcgen05.mma holds the thread until the tensor core accepts it.
+            const uint64_t dq0 = smem_desc(sb + OFF_Q, 16, 1024), dq1 = smem_desc(sb + OFF_Q + kTileQ, 16, 1024);
+            const uint64_t dk0 = smem_desc(sb + OFF_KV, 16, 1024);
+            const uint64_t dv0 = smem_desc(sb + OFF_KV + kTileKV, kBoxKV, 1024);
+            const uint64_t dp0 = smem_desc(sb + OFF_P, 16, 1024);
+            auto issue_s = [&](int j) {  // S_A(j), S_B(j) into S buffer j % 2 of each group; tile j has landed
+                const uint64_t dk = dk0 + (uint64_t)(((j % kRing) * kStageBytes) >> 4);
+                tc_fence_after();
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    const uint32_t ts = tmem + g * 2 * kKeys + (j & 1) * kKeys;
+                    const uint64_t dqg = g ? dq1 : dq0;
+#pragma unroll
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        umma(ts, dqg + (uint64_t)((((kk >> 2) * kBoxQ) + (kk & 3) * 32) >> 4),
+                             dk + (uint64_t)((((kk >> 2) * kBoxKV) + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
+                    umma_commit(s_bar(g, j & 1));
+                }
+            };
+            bool ok = ntiles > 0 && mbar_wait(q_bar, 0, abort_flag, p.status, kWaitLimitNs) &&
+                      mbar_wait(full_bar(0), 0, abort_flag, p.status, kWaitLimitNs);
+            if (ok) issue_s(0);
+            for (int j = 0; j < ntiles && ok; ++j) {
+                // S of tile j + 1 now if it has landed: its buffers were last read
+                // by the softmax of tile j - 1, whose P both groups have signalled
+                bool next = j + 1 >= ntiles;
+                if (!next && mbar_try_wait(full_bar((j + 1) % kRing), ((j + 1) / kRing) & 1)) {
+                    issue_s(j + 1);
+                    next = true;
+                }
+                const uint64_t dv = dv0 + (uint64_t)(((j % kRing) * kStageBytes) >> 4);
+                for (int g = 0; g < 2 && ok; ++g) {
+                    ok = mbar_wait(p_bar(g), j & 1, abort_flag, p.status, kWaitLimitNs);
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk)
+                        umma(tmem + 4 * kKeys + g * kD, dp0 + (uint64_t)((g * kPBytes + kk * 32) >> 4),
+                             dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(o_bar(g));
+                }
+                umma_commit(empty_bar(j % kRing));
+                if (ok && !next) {
+                    ok = mbar_wait(full_bar((j + 1) % kRing), ((j + 1) / kRing) & 1, abort_flag, p.status,
+                                   kWaitLimitNs);
+                    if (ok) issue_s(j + 1);
+                }
+            }
+            // every product this thread issued is done before TMEM can be freed
+            umma_commit(drain_bar);
+            volatile int no_abort = 0;
+            mbar_wait(drain_bar, 0, &no_abort, p.status, kWaitLimitNs);
+        }
+        __syncwarp();
+    } else {
+        // ================================================= softmax group grp: one row per thread
+        // Q row into the operand layout (K-major, 128-byte swizzle)
+        {
+            const T *qg = reinterpret_cast<const T *>(p.q);
+            const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
+            for (int c = 0; c < kD / 8; ++c) {
+                const uint32_t dst =
+                    sb + OFF_Q + grp * kTileQ + (c >> 3) * kBoxQ + trow * 128 + ((((c & 7) ^ (trow & 7))) << 4);
+                cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_bar);
+        }
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const uint32_t t_s = tmem + grp * 2 * kKeys, t_o = tmem + 4 * kKeys + grp * kD;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntiles && ok; ++j) {
+            ok = mbar_wait(s_bar(grp, j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t v0[32], v1[32];
+            tmem_ld32(t_s + (j & 1) * kKeys + lane_off, v0);
+            tmem_ld32(t_s + (j & 1) * kKeys + lane_off + 32, v1);
+            tmem_wait_ld();
+            float x[kKeys];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                x[e] = __uint_as_float(v0[e]);
+                x[32 + e] = __uint_as_float(v1[e]);
+            }
+            const int key0 = j * kKeys;
+            if (!__all_sync(0xffffffffu, key0 + kKeys - 1 <= lim)) {
+#pragma unroll
+                for (int e = 0; e < kKeys; ++e) x[e] = key0 + e <= lim ? x[e] : -INFINITY;
+            }
+            float mxa[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mxa[e] = x[e];
+#pragma unroll
+            for (int e = 8; e < kKeys; ++e) mxa[e & 7] = fmaxf(mxa[e & 7], x[e]);
+            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
+                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
+                             p.scale_log2;
+            const float mn = fmaxf(m, mx);
+            const float base = mn == -INFINITY ? 0.f : mn;
+            const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
+            float suma[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[kKeys / 2];
+#pragma unroll
+            for (int e = 0; e < kKeys; e += 2) {
+                const float p0 = fast_exp2(fmaf(x[e], p.scale_log2, -base));
+                const float p1 = fast_exp2(fmaf(x[e + 1], p.scale_log2, -base));
+                suma[(e >> 1) & 3] += p0 + p1;
+                pk[e / 2] = Mma<T>::pack(p0, p1);
+            }
+            l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
+            m = mn;
+            if (j > 0) {
+                // PV(j - 1) is done: O may be rescaled and P rewritten
+                ok = mbar_wait(o_bar(grp), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int h = 0; h < kD / 64; ++h) {
+                        const uint32_t to = t_o + lane_off + h * 64;
+                        tmem_ld32(to, v0);
+                        tmem_ld32(to + 32, v1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                            v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                        }
+                        tmem_st32(to, v0);
+                        tmem_st32(to + 32, v1);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row into the operand layout (keys as K, K-major, swizzled)
+#pragma unroll
+            for (int c = 0; c < kKeys / 8; ++c) {
+                const uint32_t dst = sb + OFF_P + grp * kPBytes + trow * 128 + ((c ^ (trow & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[c * 4]),
+                             "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_bar(grp));  // this warp's rows of P(j) are written
+        }
+        if (ok && ntiles > 0) {
+            ok = mbar_wait(o_bar(grp), (ntiles - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+        }
+        if (ok) {
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            T *og = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)qi * p.o_sl + (long long)hq * p.o_sh;
+#pragma unroll
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t v[32];
+                if (ntiles > 0) {
+                    tmem_ld32(t_o + lane_off + c * 32, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                if (row_live) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(v[e + z]) * inv;
+                        store_row8<T>(og + c * 32 + e, f);
+                    }
+                }
+            }
+            if (row_live && p.lse)
+                p.lse[b * p.lse_sb + hq * p.lse_sh + qi] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    }
+}
+
 template <typename T, int KEYS>
 static void fill(KernelInfo *out) {
     out->fn = reinterpret_cast<const void *>(&prefill_kernel<T, KEYS>);
@@ -468,6 +825,18 @@ static void fill(KernelInfo *out) {
     out->tile_keys = KEYS;
     out->stages = pf::kStages;
     out->variant = 3;  // FA_VARIANT_TCGEN05
+    out->rows = pf::kRows;
+}
+
+template <typename T>
+static void fill2(KernelInfo *out) {
+    out->fn = reinterpret_cast<const void *>(&prefill2_kernel<T>);
+    out->threads = pf2::kThreads;
+    out->smem = pf2::SMEM;
+    out->tile_keys = pf2::kKeys;
+    out->stages = pf2::kRing;
+    out->variant = 3;  // FA_VARIANT_TCGEN05
+    out->rows = pf2::kCtaRows;
 }
 
 // 128-key tiles, one CTA per SM.  (64-key tiles with two CTAs per SM measured
@@ -475,17 +844,16 @@ static void fill(KernelInfo *out) {
 // overhead cancelling the second CTA's interleaving.)
 constexpr int kPrefillKeys = 128;
 
-bool get_prefill_kernel(int dtype, int dqk, int dv, KernelInfo *out) {
-    if (dqk != 128 || dv != 128) return false;
-    if (dtype == 0) {
-        fill<__half, kPrefillKeys>(out);
-        return true;
+bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out) {
+    if (dqk != 128 || dv != 128 || dtype < 0 || dtype > 1) return false;
+    if (form == 1) {
+        if (dtype == 0) fill2<__half>(out);
+        else fill2<__nv_bfloat16>(out);
+    } else {
+        if (dtype == 0) fill<__half, kPrefillKeys>(out);
+        else fill<__nv_bfloat16, kPrefillKeys>(out);
     }
-    if (dtype == 1) {
-        fill<__nv_bfloat16, kPrefillKeys>(out);
-        return true;
-    }
-    return false;
+    return true;
 }
 
 }  // namespace fa
