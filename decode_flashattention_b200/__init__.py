@@ -30,8 +30,9 @@ __all__ = [
     "fa_decode_kvcache_append", "fa_fwd_varlen", "flash_attn_varlen_func",
     "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
-    "last_dispatch", "force_variant", "profile_enable", "profile_read", "launch_count",
+    "last_dispatch", "force_variant", "force_tcgen05_form", "profile_enable", "profile_read", "launch_count",
     "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR", "VARIANT_TCGEN05",
+    "TCGEN05_AUTO", "TCGEN05_ONE_TILE", "TCGEN05_TWO_TILES", "TCGEN05_ONE_TILE_MMA",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +40,7 @@ _LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 _lib = None
 
 VARIANT_AUTO, VARIANT_MMA, VARIANT_SCALAR, VARIANT_TCGEN05 = 0, 1, 2, 3
+TCGEN05_AUTO, TCGEN05_ONE_TILE, TCGEN05_TWO_TILES, TCGEN05_ONE_TILE_MMA = 0, 1, 2, 3
 _STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_WORKSPACE",
            4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
 _DTYPE = {torch.float16: 0, torch.bfloat16: 1}
@@ -52,7 +54,8 @@ class FaTensor(ctypes.Structure):
 class FaDispatchInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "variant", "grid", "block", "smem_bytes", "tile_keys", "stages", "rows_per_cta", "units",
-        "min_share_tiles", "combine_launched")] + [("work_tiles", ctypes.c_int64)]
+        "min_share_tiles", "combine_launched")] + [("work_tiles", ctypes.c_int64), ("tcgen05_form", ctypes.c_int32),
+                                                   ("reserved", ctypes.c_int32)]
 
 
 class FaError(RuntimeError):
@@ -92,6 +95,7 @@ def load_library():
         "fa_last_error": (ctypes.c_char_p, []),
         "fa_last_dispatch": (None, [P(FaDispatchInfo)]),
         "fa_force_variant": (i32, [i32]),
+        "fa_force_tcgen05_form": (i32, [i32]),
         "fa_profile_enable": (i32, [i32]),
         "fa_profile_read": (i32, [P(ctypes.c_double), P(ctypes.c_int64), P(ctypes.c_double),
                                   P(ctypes.c_int64)]),
@@ -393,11 +397,16 @@ def check_status(device=None):
 def last_dispatch() -> dict:
     info = FaDispatchInfo()
     load_library().fa_last_dispatch(ctypes.byref(info))
-    return {n: getattr(info, n) for n, _ in FaDispatchInfo._fields_}
+    return {n: getattr(info, n) for n, _ in FaDispatchInfo._fields_ if n != "reserved"}
 
 
 def force_variant(variant: int):
     _check(load_library().fa_force_variant(int(variant)))
+
+
+def force_tcgen05_form(form: int):
+    """Force the tcgen05 kernel's form (TCGEN05_AUTO restores the library's choice)."""
+    _check(load_library().fa_force_tcgen05_form(int(form)))
 
 
 def profile_enable(on: bool):

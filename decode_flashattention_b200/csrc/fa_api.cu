@@ -39,6 +39,7 @@ thread_local std::string t_err;
 thread_local fa_dispatch_info t_disp = {};
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_force_variant{FA_VARIANT_AUTO};
+std::atomic<int> g_force_tc_form{FA_TCGEN05_AUTO};
 
 fa_status fail(fa_status s, const char *fmt, ...) {
     char buf[512];
@@ -314,8 +315,15 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     if (variant == FA_VARIANT_TCGEN05 || (g_force_variant.load() == FA_VARIANT_AUTO && tc_shape)) {
         if (!tc_shape && (kvcache || s.Dqk != 128 || s.Dv != 128))
             return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 128/128");
-        // two 128-row tiles per CTA once there is more than one tile of rows
-        const int form = s.R > 128 ? 1 : 0;
+        // Two 128-row tiles per CTA while that still gives every SM a CTA (the
+        // tiles' softmax and products overlap); with fewer CTAs than SMs one
+        // tile per CTA, in the MMA-warp pipeline for a single tile of rows.
+        int form = g_force_tc_form.load();
+        if (form == FA_TCGEN05_AUTO) {
+            const int64_t pairs = (int64_t)((s.R + 255) / 256) * s.Hkv * s.B;
+            form = pairs >= dev->sms ? FA_TCGEN05_TWO_TILES
+                                     : (s.R <= 128 ? FA_TCGEN05_ONE_TILE_MMA : FA_TCGEN05_ONE_TILE);
+        }
         if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, form, &pl->main))
             return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d", s.dtype);
         if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
@@ -668,6 +676,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     d.min_share_tiles = pl.min_share;
     d.combine_launched = pl.need_combine ? 1 : 0;
     d.work_tiles = pl.W;
+    d.tcgen05_form = pl.prefill ? pl.main.form : 0;
     t_disp = d;
     t_err.clear();
     return FA_OK;
@@ -937,6 +946,13 @@ fa_status fa_force_variant(int variant) {
     if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_TCGEN05)
         return fail(FA_ERR_INVALID_ARG, "unknown variant %d", variant);
     g_force_variant.store(variant);
+    return FA_OK;
+}
+
+fa_status fa_force_tcgen05_form(int form) {
+    if (form < FA_TCGEN05_AUTO || form > FA_TCGEN05_ONE_TILE_MMA)
+        return fail(FA_ERR_INVALID_ARG, "unknown tcgen05 form %d", form);
+    g_force_tc_form.store(form);
     return FA_OK;
 }
 

@@ -14,6 +14,7 @@ struct KernelInfo {
     int stages;      // pipeline depth (main kernels)
     int variant;     // fa_variant
     int rows;        // packed query rows per CTA (tcgen05 kernels)
+    int form;        // fa_tcgen05_form (tcgen05 kernels)
 };
 
 // Main split-KV kernel using mma.sync (keys as M, packed rows as N).
@@ -22,7 +23,7 @@ bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
 
 // Dense attention on tcgen05 for calls with many packed rows (fa_prefill.cu).
-// form 0: one 128-row tile per CTA; form 1: two 128-row tiles per CTA.
+// form: an fa_tcgen05_form other than FA_TCGEN05_AUTO.
 bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out);
 
 // Main split-KV kernel using fp32 FMA dot products (one packed row).

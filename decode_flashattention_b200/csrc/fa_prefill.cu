@@ -27,11 +27,12 @@
 // records the error, waits (bounded) for its last tensor-core work and frees
 // its TMEM before returning.
 //
-// A second form (prefill2_kernel) puts two 128-row query tiles in one CTA with
-// a dedicated MMA warp, so the softmax of one tile overlaps the other tile's
-// products and two softmax warps share each sub-partition.
+// A second kernel (prefill3_kernel) puts two 128-row query tiles in one CTA
+// with a dedicated MMA warp, so the softmax of one tile overlaps the other
+// tile's products and two softmax warps share each sub-partition.
 #include <type_traits>
 
+#include "fa.h"
 #include "fa_common.cuh"
 #include "fa_internal.h"
 
@@ -465,51 +466,46 @@ __global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// Two query tiles per CTA (256 packed rows), used once a call has more than
-// one tile of rows.  Softmax group g (warps 2 + 4g .. 5 + 4g, one row per
-// thread; a warp reaches TMEM lanes 32 (w % 4) .. +31, so each sub-partition
-// runs one warp of each group) owns tile g.  One MMA thread issues, per
-// 64-key K / V tile j,
-//   S_A(j), S_B(j)          once tile j has landed (early, while the groups
-//                           still run the softmax of tile j - 1, when it can),
-//   PV_A(j), PV_B(j)        each once its group has written P(j),
-// so the tensor core works on one group's products while the two groups'
-// softmax warps interleave on every sub-partition.  S is double-buffered per
-// group, P has one 16 KB buffer per group in shared memory, O accumulates in
-// TMEM.  TMEM columns: S_A [0, 128), S_B [128, 256), O_A [256, 384),
-// O_B [384, 512).  K / V stream in a ring of 32 KB stages, each released by a
-// tcgen05.commit after both PV products of its tile.
-namespace pf2 {
-constexpr int kKeys = 64;
-constexpr int kRing = 4;
-constexpr int kBoxKV = kKeys * 128;              // one 64-column box of K or V (bytes)
-constexpr int kTileKV = 2 * kBoxKV;              // 64 keys x 128 elements
-constexpr int kStageBytes = 2 * kTileKV;         // K + V: 32 KB
-constexpr int kPBytes = pf::kRows * kKeys * 2;   // 128 rows x 64 keys: one box
+// Two query tiles per CTA with 128-key K / V tiles: every tensor-core product
+// is M 128 x N 128, and per 128 keys the MMA warp issues 32 products, five
+// commits and two waits.  K and V tiles stream separately through a ring of
+// three 32 KB slots (K(j), V(j), K(j + 1), ...).  S is single-buffered per
+// group; per tile j the MMA warp issues, for group A then group B,
+//   PV_g(j) once the group has written P_g(j) (so it has read S_g(j)),
+//   S_g(j + 1) right behind it (the tensor core runs them in order),
+// so one group's products run while the other group's softmax does.  P goes
+// through shared memory (one 32 KB buffer per group).  The softmax keeps a
+// running max m that only moves when a tile's max exceeds it by more than
+// 2^8 (p = 2^(s - m) then stays below 256, exact in fp32 and representable
+// in the 16-bit P), so O is rescaled only on those tiles.
+namespace pf3 {
+constexpr int kKeys = 128;
+constexpr int kSlots = 3;
+constexpr int kBox = kKeys * 128;                // one 64-column box of 128 rows (bytes)
+constexpr int kSlotBytes = 2 * kBox;             // a K or V tile: 128 keys x 128 elements
+constexpr int kPBytes = 2 * kBox;                // P: 128 rows x 128 keys
 constexpr int OFF_Q = 0;                         // Q_A, Q_B
 constexpr int OFF_P = OFF_Q + 2 * pf::kTileQ;    // P_A, P_B
 constexpr int OFF_KV = OFF_P + 2 * kPBytes;
-constexpr int OFF_BAR = OFF_KV + kRing * kStageBytes;
-// full[kRing], empty[kRing], s_done[2 groups][2 buffers], p_ready[2], o_done[2], q_ready, drain
-constexpr int NBAR = 2 * kRing + 4 + 2 + 2 + 2;
+constexpr int OFF_BAR = OFF_KV + kSlots * kSlotBytes;
+// full[kSlots], empty[kSlots], s_done[2], p_ready[2], o_done[2], q_ready, drain
+constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base, abort flag, 8 warp maxima
 constexpr int SMEM = OFF_MISC + 64 + 1024;       // + alignment slack
 constexpr int kThreads = 320;                    // an MMA warp, a producer warp, 8 softmax warps
-// The MMA warp is warp 0: a warp scheduler that keeps issuing from one ready
-// warp falls back to the oldest one when it stalls, so the MMA thread gets an
-// issue slot at each softmax stall instead of waiting behind the softmax
-// warps' arithmetic bursts on its sub-partition.
 constexpr int kMmaWarp = 0, kProducerWarp = 1, kFirstSoftmaxWarp = 2;
-constexpr int kCtaRows = 2 * pf::kRows;
-constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemCols = 512;              // S_A, S_B, O_A, O_B: 128 columns each
+constexpr float kLazyMax = 8.f;                  // log2 of the largest p before the max moves
 static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
-}  // namespace pf2
+}  // namespace pf3
 
-template <typename T>
-__global__ void __launch_bounds__(pf2::kThreads, 1)
-    prefill2_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
+// TILES: query tiles per CTA (2; or 1 when two-tile CTAs would leave SMs idle).
+template <typename T, int TILES>
+__global__ void __launch_bounds__(pf3::kThreads, 1)
+    prefill3_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
     using namespace pf;
-    using namespace pf2;
+    using namespace pf3;
+    constexpr int kCtaRows = TILES * kRows;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -520,12 +516,12 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
     const int rb = gridDim.x - 1 - blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-    auto empty_bar = [&](int s) { return smem_u32(&bars[kRing + s]); };
-    auto s_bar = [&](int g, int buf) { return smem_u32(&bars[2 * kRing + 2 * g + buf]); };
-    auto p_bar = [&](int g) { return smem_u32(&bars[2 * kRing + 4 + g]); };
-    auto o_bar = [&](int g) { return smem_u32(&bars[2 * kRing + 6 + g]); };
-    const uint32_t q_bar = smem_u32(&bars[2 * kRing + 8]);
-    const uint32_t drain_bar = smem_u32(&bars[2 * kRing + 9]);
+    auto empty_bar = [&](int s) { return smem_u32(&bars[kSlots + s]); };
+    auto s_bar = [&](int g) { return smem_u32(&bars[2 * kSlots + g]); };
+    auto p_bar = [&](int g) { return smem_u32(&bars[2 * kSlots + 2 + g]); };
+    auto o_bar = [&](int g) { return smem_u32(&bars[2 * kSlots + 4 + g]); };
+    const uint32_t q_bar = smem_u32(&bars[2 * kSlots + 6]);
+    const uint32_t drain_bar = smem_u32(&bars[2 * kSlots + 7]);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
     int *warp_keys = reinterpret_cast<int *>(smem + OFF_MISC + 16);
@@ -535,7 +531,7 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
     const int grp = ((warp - kFirstSoftmaxWarp) >> 2) & 1, quarter = warp & 3;  // TMEM lanes 32 (warp % 4) ..
     const int trow = quarter * 32 + lane;  // row within the group's tile = TMEM lane
     const int r = rb * kCtaRows + grp * kRows + trow;
-    const bool row_live = softmax && r < p.R;
+    const bool row_live = softmax && grp < TILES && r < p.R;
     const int hq = row_live ? hkv * p.g + r / p.Lq : 0;
     const int qi = row_live ? r % p.Lq : 0;
     const int n = p.Lk;
@@ -548,13 +544,12 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
         }
     }
     if (tid == 0) {
-        for (int s = 0; s < kRing; ++s) {
+        for (int s = 0; s < kSlots; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
         }
         for (int g = 0; g < 2; ++g) {
-            mbar_init(s_bar(g, 0), 1);
-            mbar_init(s_bar(g, 1), 1);
+            mbar_init(s_bar(g), 1);
             mbar_init(p_bar(g), 4);  // one arrival per softmax warp of the group
             mbar_init(o_bar(g), 1);
         }
@@ -583,89 +578,92 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
 #pragma unroll
     for (int w = 0; w < 8; ++w) kmax = max(kmax, warp_keys[w]);
     const int ntiles = (kmax + kKeys - 1) / kKeys;
+    // a last row block of at most 128 rows leaves group B without rows: its
+    // products and softmax are skipped
+    const int ngroups = TILES == 2 && rb * kCtaRows + kRows < p.R ? 2 : 1;
     constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
 
     pdl_wait_primary();
 
     if (warp == kProducerWarp) {
-        // ================================================= producer: K / V tiles by TMA
+        // ================================================= producer: K(0), V(0), K(1), ... by TMA
         if (lane == 0) {
             int issued = 0;
-            for (int j = 0; j < ntiles; ++j) {
-                const int s = j % kRing, use = j / kRing;
+            for (int q = 0; q < 2 * ntiles; ++q) {
+                const int s = q % kSlots, use = q / kSlots;
                 if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
-                const uint32_t kd = sb + OFF_KV + s * kStageBytes, vd = kd + kTileKV;
-                mbar_expect_tx(full_bar(s), kStageBytes);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_4d_plain(kd + c * kBoxKV, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
-                    tma_load_4d_plain(vd + c * kBoxKV, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
-                }
+                const uint32_t dst = sb + OFF_KV + s * kSlotBytes;
+                const CUtensorMap *map = (q & 1) ? &tmV : &tmK;
+                mbar_expect_tx(full_bar(s), kSlotBytes);
+                for (int c = 0; c < 2; ++c) tma_load_4d_plain(dst + c * kBox, map, full_bar(s), c * 64, (q >> 1) * kKeys, hkv, b);
                 mbar_arrive(full_bar(s));
-                issued = j + 1;
+                issued = q + 1;
             }
             if (*abort_flag) {
                 // let the copies still in flight land before the CTA's shared memory is released
                 volatile int no_abort = 0;
-                for (int j = issued - kRing < 0 ? 0 : issued - kRing; j < issued; ++j)
-                    mbar_wait(full_bar(j % kRing), (j / kRing) & 1, &no_abort, nullptr, kWaitLimitNs / 16);
+                for (int q = issued - kSlots < 0 ? 0 : issued - kSlots; q < issued; ++q)
+                    mbar_wait(full_bar(q % kSlots), (q / kSlots) & 1, &no_abort, nullptr, kWaitLimitNs / 16);
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ================================================= MMA issue (one thread)
         if (lane == 0) {
-            const uint32_t idesc_s = instr_desc(bf16, kRows, kKeys, false);
-            const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);
-            // Every operand descriptor is a base descriptor plus a constant
-            // offset (16-byte units in the low bits; all shared addresses stay
-            // below 256 KB, so the sum never carries out of the address field).
-            // Computing them ahead keeps the issue loop to the MMAs themselves:
-            // a tcgen05.mma holds the thread until the tensor core accepts it.
-            const uint64_t dq0 = smem_desc(sb + OFF_Q, 16, 1024), dq1 = smem_desc(sb + OFF_Q + kTileQ, 16, 1024);
-            const uint64_t dk0 = smem_desc(sb + OFF_KV, 16, 1024);
-            const uint64_t dv0 = smem_desc(sb + OFF_KV + kTileKV, kBoxKV, 1024);
+            const uint32_t idesc = instr_desc(bf16, kRows, kKeys, false);   // S: N = 128 keys, K-major K
+            const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);     // PV: N = 128 dims, MN-major V
+            // Operand descriptors: a base descriptor plus a constant offset in
+            // 16-byte units (every shared address stays below 256 KB, so the sum
+            // never carries out of the address field).
+            const uint64_t dq0 = smem_desc(sb + OFF_Q, 16, 1024);
             const uint64_t dp0 = smem_desc(sb + OFF_P, 16, 1024);
-            auto issue_s = [&](int j) {  // S_A(j), S_B(j) into S buffer j % 2 of each group; tile j has landed
-                const uint64_t dk = dk0 + (uint64_t)(((j % kRing) * kStageBytes) >> 4);
-                tc_fence_after();
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    const uint32_t ts = tmem + g * 2 * kKeys + (j & 1) * kKeys;
-                    const uint64_t dqg = g ? dq1 : dq0;
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk)
-                        umma(ts, dqg + (uint64_t)((((kk >> 2) * kBoxQ) + (kk & 3) * 32) >> 4),
-                             dk + (uint64_t)((((kk >> 2) * kBoxKV) + (kk & 3) * 32) >> 4), idesc_s, kk > 0);
-                    umma_commit(s_bar(g, j & 1));
-                }
+            const uint64_t dk0 = smem_desc(sb + OFF_KV, 16, 1024);        // a slot holding K
+            const uint64_t dv0 = smem_desc(sb + OFF_KV, kBox, 1024);      // a slot holding V
+            auto wait = [&](uint32_t bar, uint32_t parity) {
+                return mbar_wait(bar, parity, abort_flag, p.status, kWaitLimitNs);
             };
-            bool ok = ntiles > 0 && mbar_wait(q_bar, 0, abort_flag, p.status, kWaitLimitNs) &&
-                      mbar_wait(full_bar(0), 0, abort_flag, p.status, kWaitLimitNs);
-            if (ok) issue_s(0);
-            for (int j = 0; j < ntiles && ok; ++j) {
-                // S of tile j + 1 now if it has landed: its buffers were last read
-                // by the softmax of tile j - 1, whose P both groups have signalled
-                bool next = j + 1 >= ntiles;
-                if (!next && mbar_try_wait(full_bar((j + 1) % kRing), ((j + 1) / kRing) & 1)) {
-                    issue_s(j + 1);
-                    next = true;
+            // S_g(j) = Q_g K(j)^T; K(j) is ring entry 2j
+            auto issue_s = [&](int g, int j) {
+                const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * kSlotBytes) >> 4);
+                const uint64_t dq = dq0 + (uint64_t)((g * kTileQ) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (uint32_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+                    umma(tmem + g * kKeys, dq + off, dk + off, idesc, kk > 0);
                 }
-                const uint64_t dv = dv0 + (uint64_t)(((j % kRing) * kStageBytes) >> 4);
-                for (int g = 0; g < 2 && ok; ++g) {
-                    ok = mbar_wait(p_bar(g), j & 1, abort_flag, p.status, kWaitLimitNs);
+                umma_commit(s_bar(g));
+            };
+            bool ok = ntiles > 0 && wait(q_bar, 0) && wait(full_bar(0), 0);
+            if (ok) {
+                tc_fence_after();
+                for (int g = 0; g < ngroups; ++g) issue_s(g, 0);
+                umma_commit(empty_bar(0));  // K(0) read once its products are done
+            }
+            for (int j = 0; j < ntiles && ok; ++j) {
+                const int qv = 2 * j + 1, qk = 2 * j + 2;  // ring entries of V(j), K(j + 1)
+                const bool more = j + 1 < ntiles;
+                const uint64_t dv = dv0 + (uint64_t)(((qv % kSlots) * kSlotBytes) >> 4);
+                for (int g = 0; g < ngroups && ok; ++g) {
+                    // P_g(j) written (S_g(j) read, O_g rescaled); V(j) landed
+                    ok = wait(p_bar(g), j & 1) && (g > 0 || wait(full_bar(qv % kSlots), (qv / kSlots) & 1));
                     if (!ok) break;
                     tc_fence_after();
+                    const uint64_t dp = dp0 + (uint64_t)((g * kPBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk)
-                        umma(tmem + 4 * kKeys + g * kD, dp0 + (uint64_t)((g * kPBytes + kk * 32) >> 4),
+                        umma(tmem + 2 * kKeys + g * kD, dp + (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4),
                              dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(o_bar(g));
-                }
-                umma_commit(empty_bar(j % kRing));
-                if (ok && !next) {
-                    ok = mbar_wait(full_bar((j + 1) % kRing), ((j + 1) / kRing) & 1, abort_flag, p.status,
-                                   kWaitLimitNs);
-                    if (ok) issue_s(j + 1);
+                    if (g == ngroups - 1) umma_commit(empty_bar(qv % kSlots));  // V(j) read by its products
+                    if (more) {
+                        if (g == 0) {
+                            ok = wait(full_bar(qk % kSlots), (qk / kSlots) & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        issue_s(g, j + 1);
+                        if (g == ngroups - 1) umma_commit(empty_bar(qk % kSlots));  // K(j + 1) read by its products
+                    }
                 }
             }
             // every product this thread issued is done before TMEM can be freed
@@ -676,7 +674,6 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
         __syncwarp();
     } else {
         // ================================================= softmax group grp: one row per thread
-        // Q row into the operand layout (K-major, 128-byte swizzle)
         {
             const T *qg = reinterpret_cast<const T *>(p.q);
             const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
@@ -691,25 +688,27 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
             if (lane == 0) mbar_arrive(q_bar);
         }
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t t_s = tmem + grp * 2 * kKeys, t_o = tmem + 4 * kKeys + grp * kD;
-        float m = -INFINITY, l = 0.f;
-        bool ok = true;
+        const uint32_t t_s = tmem + grp * kKeys + lane_off, t_o = tmem + 2 * kKeys + grp * kD + lane_off;
+        const uint32_t p_row = sb + OFF_P + grp * kPBytes + trow * 128;
+        float m = -INFINITY, l = 0.f;  // m in base-2 units of the scaled scores
+        bool ok = grp < ngroups;  // a group without rows has nothing to do
         for (int j = 0; j < ntiles && ok; ++j) {
-            ok = mbar_wait(s_bar(grp, j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = mbar_wait(s_bar(grp), j & 1, abort_flag, p.status, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            uint32_t v0[32], v1[32];
-            tmem_ld32(t_s + (j & 1) * kKeys + lane_off, v0);
-            tmem_ld32(t_s + (j & 1) * kKeys + lane_off + 32, v1);
-            tmem_wait_ld();
             float x[kKeys];
+            {
+                uint32_t v[4][32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                x[e] = __uint_as_float(v0[e]);
-                x[32 + e] = __uint_as_float(v1[e]);
+                for (int c = 0; c < 4; ++c) tmem_ld32(t_s + c * 32, v[c]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[c][e]);
             }
             const int key0 = j * kKeys;
             if (!__all_sync(0xffffffffu, key0 + kKeys - 1 <= lim)) {
@@ -724,54 +723,58 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
             const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
                                    fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
                              p.scale_log2;
-            const float mn = fmaxf(m, mx);
+            // the running max moves only when this tile's max is more than 2^8 above it
+            const float mn = mx > m + kLazyMax ? mx : m;
             const float base = mn == -INFINITY ? 0.f : mn;
-            const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
-            float suma[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[kKeys / 2];
-#pragma unroll
-            for (int e = 0; e < kKeys; e += 2) {
-                const float p0 = fast_exp2(fmaf(x[e], p.scale_log2, -base));
-                const float p1 = fast_exp2(fmaf(x[e + 1], p.scale_log2, -base));
-                suma[(e >> 1) & 3] += p0 + p1;
-                pk[e / 2] = Mma<T>::pack(p0, p1);
-            }
-            l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
+            const float alpha = fast_exp2(m - base);  // 1 when m stays, 0 while nothing was seen
             m = mn;
+            // PV_g(j - 1) is done: it ran before S_g(j) on the tensor core; the
+            // wait makes it visible and frees P_g for this tile
             if (j > 0) {
-                // PV(j - 1) is done: O may be rescaled and P rewritten
                 ok = mbar_wait(o_bar(grp), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                    for (int h = 0; h < kD / 64; ++h) {
-                        const uint32_t to = t_o + lane_off + h * 64;
-                        tmem_ld32(to, v0);
-                        tmem_ld32(to + 32, v1);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
-                            v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
-                        }
-                        tmem_st32(to, v0);
-                        tmem_st32(to + 32, v1);
-                    }
-                    tmem_wait_st();
-                }
             }
-            // P row into the operand layout (keys as K, K-major, swizzled)
+            // p = 2^(x * scale_log2 - m), packed and stored to P in the operand
+            // layout (keys as K, K-major, 128-byte swizzle) eight keys at a time
+            float suma[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < kKeys / 8; ++c) {
-                const uint32_t dst = sb + OFF_P + grp * kPBytes + trow * 128 + ((c ^ (trow & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[c * 4]),
-                             "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float p0 = fast_exp2(fmaf(x[c * 8 + e], p.scale_log2, -base));
+                    const float p1 = fast_exp2(fmaf(x[c * 8 + e + 1], p.scale_log2, -base));
+                    suma[(e >> 1) & 3] += p0 + p1;
+                    pk[e >> 1] = Mma<T>::pack(p0, p1);
+                }
+                const uint32_t dst = p_row + (c >> 3) * kBox + (((c & 7) ^ (trow & 7)) << 4);
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
+                             "r"(pk[2]), "r"(pk[3])
                              : "memory");
             }
+            // O_g *= alpha where the max moved (after the scores are spent: fewer live registers)
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                for (int h = 0; h < kD / 64; ++h) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(t_o + h * 64, v0);
+                    tmem_ld32(t_o + h * 64 + 32, v1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                        v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                    }
+                    tmem_st32(t_o + h * 64, v0);
+                    tmem_st32(t_o + h * 64 + 32, v1);
+                }
+                tmem_wait_st();
+            }
+            l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
@@ -789,7 +792,7 @@ __global__ void __launch_bounds__(pf2::kThreads, 1)
             for (int c = 0; c < kD / 32; ++c) {
                 uint32_t v[32];
                 if (ntiles > 0) {
-                    tmem_ld32(t_o + lane_off + c * 32, v);
+                    tmem_ld32(t_o + c * 32, v);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
@@ -826,17 +829,7 @@ static void fill(KernelInfo *out) {
     out->stages = pf::kStages;
     out->variant = 3;  // FA_VARIANT_TCGEN05
     out->rows = pf::kRows;
-}
-
-template <typename T>
-static void fill2(KernelInfo *out) {
-    out->fn = reinterpret_cast<const void *>(&prefill2_kernel<T>);
-    out->threads = pf2::kThreads;
-    out->smem = pf2::SMEM;
-    out->tile_keys = pf2::kKeys;
-    out->stages = pf2::kRing;
-    out->variant = 3;  // FA_VARIANT_TCGEN05
-    out->rows = pf2::kCtaRows;
+    out->form = FA_TCGEN05_ONE_TILE;
 }
 
 // 128-key tiles, one CTA per SM.  (64-key tiles with two CTAs per SM measured
@@ -844,16 +837,36 @@ static void fill2(KernelInfo *out) {
 // overhead cancelling the second CTA's interleaving.)
 constexpr int kPrefillKeys = 128;
 
+template <typename T, int TILES>
+static void fill3(KernelInfo *out) {
+    out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES>);
+    out->threads = pf3::kThreads;
+    out->smem = pf3::SMEM;
+    out->tile_keys = pf3::kKeys;
+    out->stages = pf3::kSlots;
+    out->variant = 3;  // FA_VARIANT_TCGEN05
+    out->rows = TILES * pf::kRows;
+    out->form = TILES == 2 ? FA_TCGEN05_TWO_TILES : FA_TCGEN05_ONE_TILE_MMA;
+}
+
 bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out) {
     if (dqk != 128 || dv != 128 || dtype < 0 || dtype > 1) return false;
-    if (form == 1) {
-        if (dtype == 0) fill2<__half>(out);
-        else fill2<__nv_bfloat16>(out);
-    } else {
+    switch (form) {
+    case FA_TCGEN05_ONE_TILE:
         if (dtype == 0) fill<__half, kPrefillKeys>(out);
         else fill<__nv_bfloat16, kPrefillKeys>(out);
+        return true;
+    case FA_TCGEN05_TWO_TILES:
+        if (dtype == 0) fill3<__half, 2>(out);
+        else fill3<__nv_bfloat16, 2>(out);
+        return true;
+    case FA_TCGEN05_ONE_TILE_MMA:
+        if (dtype == 0) fill3<__half, 1>(out);
+        else fill3<__nv_bfloat16, 1>(out);
+        return true;
+    default:
+        return false;
     }
-    return true;
 }
 
 }  // namespace fa

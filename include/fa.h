@@ -107,6 +107,8 @@ typedef struct fa_dispatch_info {
     int32_t min_share_tiles;  /* least tiles a CTA is given */
     int32_t combine_launched; /* 1 if the LSE combine kernel was launched */
     int64_t work_tiles;       /* total key tiles (known on the host for fa_fwd; -1 for kvcache) */
+    int32_t tcgen05_form;     /* fa_tcgen05_form of the tcgen05 kernel (0 for the other variants) */
+    int32_t reserved;
 } fa_dispatch_info;
 
 /*
@@ -290,6 +292,31 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  * support the call's shapes makes the call fail with FA_ERR_UNSUPPORTED.
  */
 FA_API fa_status fa_force_variant(int variant);
+
+/*
+ * Forms of the tcgen05 kernel (all: 128 packed rows per query tile, 128-key
+ * K / V tiles, accumulators in TMEM, the whole key range per CTA):
+ *   FA_TCGEN05_ONE_TILE       one tile per CTA; the softmax warps issue the
+ *                             products themselves and S is double-buffered, so
+ *                             the next tile's QK^T runs during this tile's softmax;
+ *   FA_TCGEN05_TWO_TILES      two tiles per CTA and a dedicated MMA warp: one
+ *                             tile's products run while the other tile's
+ *                             softmax does (S single-buffered per tile);
+ *   FA_TCGEN05_ONE_TILE_MMA   the two-tile kernel's pipeline with one tile.
+ * The library's choice: two tiles when that still gives every SM a CTA
+ * (ceil(R / 256) * Hkv * B >= SMs), else the MMA-warp pipeline for calls of at
+ * most 128 packed rows, else one tile per CTA.
+ */
+typedef enum {
+    FA_TCGEN05_AUTO = 0,
+    FA_TCGEN05_ONE_TILE = 1,
+    FA_TCGEN05_TWO_TILES = 2,
+    FA_TCGEN05_ONE_TILE_MMA = 3
+} fa_tcgen05_form;
+
+/* Tuning / test hook: force the tcgen05 kernel's form for later calls of this
+ * process (FA_TCGEN05_AUTO restores the library's choice). */
+FA_API fa_status fa_force_tcgen05_form(int form);
 
 /*
  * Profiling: while enabled, each compute call brackets its main kernel and

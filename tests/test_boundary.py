@@ -122,6 +122,14 @@ def test_force_variant_rejects_unknown():
     assert fa.load_library().fa_force_variant(0) == OK
 
 
+def test_force_tcgen05_form_rejects_unknown():
+    lib = fa.load_library()
+    assert lib.fa_force_tcgen05_form(4) == INVALID
+    assert lib.fa_force_tcgen05_form(-1) == INVALID
+    for form in (fa.TCGEN05_ONE_TILE, fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA, fa.TCGEN05_AUTO):
+        assert lib.fa_force_tcgen05_form(form) == OK
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_cuda_error():
     q, k, v, o = good("q"), good("k"), good("v"), good("o")

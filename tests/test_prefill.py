@@ -21,8 +21,12 @@ DEV = "cuda"
 def _reset():
     yield
     fa.force_variant(fa.VARIANT_AUTO)
+    fa.force_tcgen05_form(fa.TCGEN05_AUTO)
     torch.cuda.synchronize()
     fa.check_status()
+
+
+FORMS = [fa.TCGEN05_ONE_TILE, fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA]
 
 
 CASES = [  # B, Lq, Hq, Hkv, Lk, causal
@@ -72,3 +76,42 @@ def test_full_size_prefill_sampled_rows():
     got_o = o.float().cpu().numpy()[rows[:, 0], rows[:, 2], rows[:, 1]]
     got_l = lse.cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
     compare(got_o, got_l, ro, rl, w.dtype, "prefill 4k")
+
+
+FORM_CASES = [  # B, Lq, Hq, Hkv, Lk, causal: ragged row blocks (R % 256 below and above 128), short and long keys
+    (1, 200, 2, 1, 300, True), (2, 130, 4, 2, 129, False), (1, 700, 1, 1, 700, True), (3, 96, 8, 2, 1000, True),
+    (1, 64, 32, 8, 2500, False), (1, 1, 256, 1, 77, False),
+    (1, 300, 2, 1, 100, True),  # causal with Lq > Lk: the first 200 positions see no key
+]
+
+
+@pytest.mark.parametrize("form", FORMS)
+@pytest.mark.parametrize("case", FORM_CASES, ids=[str(c) for c in FORM_CASES])
+def test_every_form_parity(form, case):
+    B, Lq, Hq, Hkv, Lk, causal = case
+    dt = torch.bfloat16 if (Lq + form) % 2 else torch.float16
+    w = wl.Workload("pf_form", "fwd", "blhd", dt, B=B, Lq=Lq, Hq=Hq, Hkv=Hkv, Lk=Lk, Dqk=128, Dv=128, causal=causal,
+                    seed=Lq * 7 + Lk + form)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)
+    fa.force_tcgen05_form(form)
+    o, lse = fa.fa_fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    d = fa.last_dispatch()
+    assert d["variant"] == fa.VARIANT_TCGEN05 and d["tcgen05_form"] == form
+    assert d["rows_per_cta"] == (256 if form == fa.TCGEN05_TWO_TILES else 128)
+    ro, rl = oracle_full(q, k, v, causal)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 form {form}")
+
+
+def test_automatic_form_choice():
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for (B, Lq, Hq, Hkv), want in (((1, 4096, 32, 8), fa.TCGEN05_TWO_TILES),   # 64 x 8 two-tile CTAs
+                                   ((1, 300, 16, 16), fa.TCGEN05_ONE_TILE),    # 2 x 16 two-tile CTAs
+                                   ((2, 32, 32, 8), fa.TCGEN05_ONE_TILE_MMA)):  # 128 rows, 16 CTAs
+        assert ((B > 0) and ((Lq * Hq // Hkv + 255) // 256) * Hkv * B >= sms) == (want == fa.TCGEN05_TWO_TILES)
+        q = torch.zeros(B, Lq, Hq, 128, dtype=torch.bfloat16, device=DEV)
+        k = torch.zeros(B, 256, Hkv, 128, dtype=torch.bfloat16, device=DEV)
+        fa.fa_fwd(q, k, k, causal=True)
+        torch.cuda.synchronize()
+        assert fa.last_dispatch()["tcgen05_form"] == want
