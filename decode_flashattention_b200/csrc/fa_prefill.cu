@@ -116,6 +116,17 @@ __device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, ui
         : "memory");
 }
 
+// The same with A read from tensor memory (M rows in lanes, two 16-bit K
+// elements per 32-bit column, K-major).
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
@@ -473,8 +484,12 @@ __global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
 // group; per tile j the MMA warp issues, for group A then group B,
 //   PV_g(j) once the group has written P_g(j) (so it has read S_g(j)),
 //   S_g(j + 1) right behind it (the tensor core runs them in order),
-// so one group's products run while the other group's softmax does.  P goes
-// through shared memory (one 32 KB buffer per group).  The softmax keeps a
+// so one group's products run while the other group's softmax does.  P stays
+// in TMEM: the softmax writes it (two 16-bit values per 32-bit column) over the
+// S columns it has just read, and PV_g(j) takes its A operand from there, so
+// P costs no shared-memory bandwidth (the S products already use all of it:
+// Q and K reads of 8 KB per 64-cycle M 128 x N 128 x K 16 product).  The
+// softmax keeps a
 // running max m that only moves when a tile's max exceeds it by more than
 // 2^8 (p = 2^(s - m) then stays below 256, exact in fp32 and representable
 // in the 16-bit P), so O is rescaled only on those tiles.
@@ -483,10 +498,8 @@ constexpr int kKeys = 128;
 constexpr int kSlots = 3;
 constexpr int kBox = kKeys * 128;                // one 64-column box of 128 rows (bytes)
 constexpr int kSlotBytes = 2 * kBox;             // a K or V tile: 128 keys x 128 elements
-constexpr int kPBytes = 2 * kBox;                // P: 128 rows x 128 keys
 constexpr int OFF_Q = 0;                         // Q_A, Q_B
-constexpr int OFF_P = OFF_Q + 2 * pf::kTileQ;    // P_A, P_B
-constexpr int OFF_KV = OFF_P + 2 * kPBytes;
+constexpr int OFF_KV = OFF_Q + 2 * pf::kTileQ;
 constexpr int OFF_BAR = OFF_KV + kSlots * kSlotBytes;
 // full[kSlots], empty[kSlots], s_done[2], p_ready[2], o_done[2], q_ready, drain
 constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
@@ -616,7 +629,6 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // 16-byte units (every shared address stays below 256 KB, so the sum
             // never carries out of the address field).
             const uint64_t dq0 = smem_desc(sb + OFF_Q, 16, 1024);
-            const uint64_t dp0 = smem_desc(sb + OFF_P, 16, 1024);
             const uint64_t dk0 = smem_desc(sb + OFF_KV, 16, 1024);        // a slot holding K
             const uint64_t dv0 = smem_desc(sb + OFF_KV, kBox, 1024);      // a slot holding V
             auto wait = [&](uint32_t bar, uint32_t parity) {
@@ -648,11 +660,10 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     ok = wait(p_bar(g), j & 1) && (g > 0 || wait(full_bar(qv % kSlots), (qv / kSlots) & 1));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint64_t dp = dp0 + (uint64_t)((g * kPBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < kKeys / 16; ++kk)
-                        umma(tmem + 2 * kKeys + g * kD, dp + (uint64_t)((((kk >> 2) * kBox) + (kk & 3) * 32) >> 4),
-                             dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kKeys / 16; ++kk)  // P_g(j): 16 keys = 8 TMEM columns per step
+                        umma_ts(tmem + 2 * kKeys + g * kD, tmem + g * kKeys + kk * 8,
+                                dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(o_bar(g));
                     if (g == ngroups - 1) umma_commit(empty_bar(qv % kSlots));  // V(j) read by its products
                     if (more) {
@@ -689,7 +700,6 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         }
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t t_s = tmem + grp * kKeys + lane_off, t_o = tmem + 2 * kKeys + grp * kD + lane_off;
-        const uint32_t p_row = sb + OFF_P + grp * kPBytes + trow * 128;
         float m = -INFINITY, l = 0.f;  // m in base-2 units of the scaled scores
         bool ok = grp < ngroups;  // a group without rows has nothing to do
         for (int j = 0; j < ntiles && ok; ++j) {
@@ -728,36 +738,32 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             const float base = mn == -INFINITY ? 0.f : mn;
             const float alpha = fast_exp2(m - base);  // 1 when m stays, 0 while nothing was seen
             m = mn;
-            // PV_g(j - 1) is done: it ran before S_g(j) on the tensor core; the
-            // wait makes it visible and frees P_g for this tile
-            if (j > 0) {
+            // p = 2^(x * scale_log2 - m), packed two keys per 32-bit column and
+            // written over this row's S columns [0, 64) in TMEM: the A operand of
+            // PV_g(j).  (The scores are all in registers by now; PV_g(j - 1),
+            // which read the previous P there, finished before S_g(j) did.)
+            float suma[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = fast_exp2(fmaf(x[h * 64 + 2 * c], p.scale_log2, -base));
+                    const float p1 = fast_exp2(fmaf(x[h * 64 + 2 * c + 1], p.scale_log2, -base));
+                    suma[c & 3] += p0 + p1;
+                    pk[c] = Mma<T>::pack(p0, p1);
+                }
+                tmem_st32(t_s + h * 32, pk);
+            }
+            // O_g *= alpha where the max moved.  PV_g(j - 1) is complete (it ran
+            // before S_g(j)); the wait on its barrier makes that visible here.
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 ok = mbar_wait(o_bar(grp), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-            }
-            // p = 2^(x * scale_log2 - m), packed and stored to P in the operand
-            // layout (keys as K, K-major, 128-byte swizzle) eight keys at a time
-            float suma[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < kKeys / 8; ++c) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const float p0 = fast_exp2(fmaf(x[c * 8 + e], p.scale_log2, -base));
-                    const float p1 = fast_exp2(fmaf(x[c * 8 + e + 1], p.scale_log2, -base));
-                    suma[(e >> 1) & 3] += p0 + p1;
-                    pk[e >> 1] = Mma<T>::pack(p0, p1);
-                }
-                const uint32_t dst = p_row + (c >> 3) * kBox + (((c & 7) ^ (trow & 7)) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
-                             "r"(pk[2]), "r"(pk[3])
-                             : "memory");
-            }
-            // O_g *= alpha where the max moved (after the scores are spent: fewer live registers)
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
                 for (int h = 0; h < kD / 64; ++h) {
                     uint32_t v0[32], v1[32];
@@ -772,10 +778,9 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     tmem_st32(t_o + h * 64, v0);
                     tmem_st32(t_o + h * 64 + 32, v1);
                 }
-                tmem_wait_st();
             }
+            tmem_wait_st();
             l = l * alpha + ((suma[0] + suma[1]) + (suma[2] + suma[3]));
-            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(p_bar(grp));  // this warp's rows of P(j) are written
