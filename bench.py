@@ -477,7 +477,7 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16" if w.dtype.__repr__().endswith("float16") else "bf16",
+        "dtype": "f16" if w.dtype == torch.float16 else "bf16",
         "data": "synthetic: Q/K/V i.i.d. N(0,1), seeded; no dataset or weights",
         "config": {
             "workload": name, "description": w.description, "call": w.call, "layout": w.layout,
