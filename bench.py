@@ -161,7 +161,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ helpers
-def tensor_roofline(w, seqlens, ms_per_call, prof):
+def tensor_roofline(w, seqlens, ms_per_call, prof, traffic=None):
     """Roofline of a call on the tcgen05 kernel: bound by the tensor cores.
     achieved = the call's multiply-add flops / its time; peak = the measured
     sustained cuBLAS bf16 rate (the kernel runs back to back for seconds), the
@@ -179,7 +179,7 @@ def tensor_roofline(w, seqlens, ms_per_call, prof):
     achieved = flops / (ms_per_call / 1e3) / 1e12
     return {"bound": "tensor", "kernel": "tcgen05 dense kernel (whole call)", "achieved": round(achieved, 2),
             "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-            "traffic": None, "algorithmic_flops_per_launch": flops, "kernel_us": round(ms_per_call * 1e3, 3),
+            "traffic": traffic, "algorithmic_flops_per_launch": flops, "kernel_us": round(ms_per_call * 1e3, 3),
             "isolated_us": {"tcgen05": round(prof["main_ms"] / max(prof["main_launches"], 1) * 1e3, 3)}}
 
 
@@ -217,8 +217,9 @@ def kernel_source_hash():
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the split-KV kernel from a committed ncu
-    capture, if it was taken on the current kernel sources."""
+    """DRAM bytes per launch of the workload's main kernel (split-KV or
+    tcgen05) from a committed ncu capture, if it was taken on the current
+    kernel sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -490,7 +491,7 @@ def run_ours(args):
             "parallelism": f"replicas{world}" if world > 1 else "single_gpu",
             "dispatch": dispatch,
         },
-        "roofline": tensor_roofline(w, sl0, ms / K, prof) if tc else {
+        "roofline": tensor_roofline(w, sl0, ms / K, prof, traffic) if tc else {
             "bound": "hbm",
             "kernel": "split-KV kernel, charged with the whole call (combine and boundaries included)",
             "achieved": round(achieved, 1) if achieved else None,
