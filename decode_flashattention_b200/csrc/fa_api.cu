@@ -156,7 +156,28 @@ fa_status check_tensor(const fa_tensor *t, const char *name) {
 struct Shapes {
     int dtype;
     int B, Lq, Hq, Lk, Hkv, Dqk, Dv, g, R, RB, BR;
+    int KDqk, KDv;  // head dims of the kernel instance that runs the call (>= Dqk, Dv)
 };
+
+// Head dims: any multiple of 8 from 8 to 256 (a TMA row stride must be a
+// multiple of 16 bytes).  A call runs on the compiled instance that covers
+// both dims -- (192, 128) for MLA-shaped dims, else the square instance 64,
+// 128 or 256 -- the dims past the call's read as zeros (TMA fills the columns
+// past a row's end, the query rows are zero-filled) and are never written.
+fa_status kernel_dims(Shapes *s) {
+    auto ok_dim = [](int d) { return d >= 8 && d <= 256 && d % 8 == 0; };
+    if (!ok_dim(s->Dqk) || !ok_dim(s->Dv))
+        return fail(FA_ERR_UNSUPPORTED, "head dims (Dqk %d, Dv %d): each must be a multiple of 8 from 8 to 256",
+                    s->Dqk, s->Dv);
+    auto pad = [](int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : 256); };
+    if (s->Dqk > 128 && s->Dqk <= 192 && s->Dv <= 128) {
+        s->KDqk = 192;
+        s->KDv = 128;
+    } else {
+        s->KDqk = s->KDv = std::max(pad(s->Dqk), pad(s->Dv));
+    }
+    return FA_OK;
+}
 
 // Paged K/V: K and V are [num_blocks, page, Hkv, D]; batch b's key j is row
 // j % page of block block_table[b * bt_stride + j / page].
@@ -221,10 +242,7 @@ fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
         return fail(FA_ERR_INVALID_ARG, "o must be [B, Lq, Hq, Dv]");
     if (s->Hkv <= 0 || s->Hq <= 0) return fail(FA_ERR_INVALID_ARG, "head counts must be positive");
     if (s->Hq % s->Hkv) return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", s->Hq, s->Hkv);
-    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128) ||
-          (s->Dqk == 256 && s->Dv == 256)))
-        return fail(FA_ERR_UNSUPPORTED,
-                    "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128), (256,256)}", s->Dqk, s->Dv);
+    if ((st = kernel_dims(s))) return st;
     s->g = s->Hq / s->Hkv;
     int64_t R = (int64_t)s->g * s->Lq;
     if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * Lq too large");
@@ -341,14 +359,14 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
             return fail(FA_ERR_UNSUPPORTED, "grid too large for the tcgen05 variant");
         return FA_OK;
     }
-    bool ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.Dqk, s.Dv, &pl->main)
-                                           : fa::get_mma_kernel(s.dtype, s.Dqk, s.Dv, &pl->main);
+    bool ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.KDqk, s.KDv, &pl->main)
+                                           : fa::get_mma_kernel(s.dtype, s.KDqk, s.KDv, &pl->main);
     if (variant == FA_VARIANT_SCALAR && ok && s.R != 1)
         return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
     if (!ok) return fail(FA_ERR_UNSUPPORTED, "no kernel for variant %d, dtype %d, head dims (%d, %d)", variant,
                          s.dtype, s.Dqk, s.Dv);
-    if (!fa::get_combine_kernel(s.dtype, s.Dv, &pl->comb))
-        return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.Dv);
+    if (!fa::get_combine_kernel(s.dtype, s.KDv, &pl->comb))
+        return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.KDv);
     if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
     pl->comb_smem = 0;
     int comb_occ = 0;
@@ -391,7 +409,7 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     }
     pl->need_workspace = pl->need_combine;
     pl->pieces = (size_t)pl->P_param;  // one piece per CTA
-    const size_t o_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta * s.Dv : 0;
+    const size_t o_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta * s.KDv : 0;
     const size_t lse_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta : 0;
     pl->ws_o_off = 0;
     pl->ws_lse_off = pl->ws_o_off + ((o_floats * 4 + 255) & ~size_t(255));
@@ -523,6 +541,8 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.R = s.R;
     p.RB = s.RB;
     p.Lk = s.Lk;
+    p.dqk = s.Dqk;
+    p.dv = s.Dv;
     p.causal = causal ? 1 : 0;
     float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)s.Dqk);
     p.scale_log2 = sc * 1.4426950408889634f;
@@ -860,10 +880,7 @@ fa_status check_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
         return fail(FA_ERR_INVALID_ARG, "o must be [1, total_q, Hq, Dv]");
     if (s->Hkv <= 0 || s->Hq <= 0 || s->Hq % s->Hkv)
         return fail(FA_ERR_INVALID_ARG, "Hq (%d) must be a positive multiple of Hkv (%d)", s->Hq, s->Hkv);
-    if (!((s->Dqk == 64 && s->Dv == 64) || (s->Dqk == 128 && s->Dv == 128) || (s->Dqk == 192 && s->Dv == 128) ||
-          (s->Dqk == 256 && s->Dv == 256)))
-        return fail(FA_ERR_UNSUPPORTED,
-                    "head dims (Dqk %d, Dv %d) not in {(64,64), (128,128), (192,128), (256,256)}", s->Dqk, s->Dv);
+    if ((st = kernel_dims(s))) return st;
     s->g = s->Hq / s->Hkv;
     const int64_t R = (int64_t)s->g * s->Lq;
     if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * max_seqlen_q too large");

@@ -189,9 +189,10 @@ __global__ void __launch_bounds__(kCombineThreads)
                 lse2 = M + log2f(L);
             }
         }
+        const int dmax = warm ? DV : p.dv;  // only the call's Dv dims (a multiple of 8) are written
 #pragma unroll
         for (int e = 0; e < EPL; e += 2)
-            *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(acc[e], acc[e + 1]);
+            if (lane_off + e < dmax) *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(acc[e], acc[e + 1]);
         if (lse_out && lane == 0) *lse_out = lse2 == -INFINITY ? -INFINITY : lse2 * 0.69314718055994531f;
         __syncwarp();
     }

@@ -32,6 +32,7 @@ struct Params {
     const int *seqlens;    // [B] or null (then every batch has Lk keys)
     unsigned *status;      // device status word (timeouts)
     int B, Lq, Hq, Hkv, g, R, RB, Lk;
+    int dqk, dv;           // the call's head dims (the kernel's DQK / DV may be larger: columns past them are zero)
     int causal;
     float scale_log2;      // scale * log2(e)
     int P;                 // CTAs launched

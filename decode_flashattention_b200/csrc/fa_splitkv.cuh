@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int rq = rb * kRowsPerCta + r;
                         const T *src = qg;
                         uint32_t nbytes = 0;
-                        if (rq < G.R) {
+                        if (rq < G.R && c * 8 < p.dqk) {  // dims past the call's head dim stay zero
                             const int hq = hkv * p.g + rq / G.Lq, i = rq % G.Lq;
                             src = qg + b * p.q_sb + (long long)(G.q0 + i) * p.q_sl + (long long)hq * p.q_sh + c * 8;
                             nbytes = 16;
@@ -350,13 +350,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int hq = md.hkv * p.g + rr / cg.Lq, i = rr % cg.Lq;
                 T *op = warm ? static_cast<T *>(sink)
                              : og + md.b * p.o_sb + (long long)(cg.q0 + i) * p.o_sl + (long long)hq * p.o_sh + d0;
+                // only the call's Dv dims (a multiple of 8) are written
+                const int dmax = warm ? DV : p.dv;
                 if constexpr (EPT % 8 == 0) {
 #pragma unroll
-                    for (int e = 0; e < EPT; e += 8) store_row8<T>(op + e, v + e);
+                    for (int e = 0; e < EPT; e += 8)
+                        if (d0 + e < dmax) store_row8<T>(op + e, v + e);
                 } else {
+                    if (d0 < dmax) {
 #pragma unroll
-                    for (int e = 0; e < EPT; e += 2)
-                        *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(v[e], v[e + 1]);
+                        for (int e = 0; e < EPT; e += 2)
+                            *reinterpret_cast<uint32_t *>(op + e) = Mma<T>::pack(v[e], v[e + 1]);
+                    }
                 }
                 if (p.lse && (tid % TPR) == 0)
                     *(warm ? static_cast<float *>(sink)

@@ -64,7 +64,8 @@ def good(name, **kw):
 
 
 @pytest.mark.parametrize("case,expect", [
-    ("dtype_mismatch", INVALID), ("bad_gqa", INVALID), ("head_dim_96", UNSUPPORTED),
+    ("dtype_mismatch", INVALID), ("bad_gqa", INVALID), ("head_dim_264", UNSUPPORTED), ("head_dim_12", UNSUPPORTED),
+    ("head_dim_v_264", UNSUPPORTED),
     ("last_dim_strided", UNSUPPORTED), ("stride_not_16B", UNSUPPORTED), ("misaligned", UNSUPPORTED),
     ("null_o", INVALID), ("batch_mismatch", INVALID), ("nan_scale", INVALID), ("fp32", UNSUPPORTED),
     ("too_many_row_blocks", UNSUPPORTED), ("null_data", INVALID), ("o_shape", INVALID),
@@ -76,8 +77,12 @@ def test_host_validation(case, expect):
         v = good("v", dtype=1)
     elif case == "bad_gqa":
         q = desc([1, 1, 3, 128]); o = desc([1, 1, 3, 128])
-    elif case == "head_dim_96":
-        q, k, v, o = desc([1, 1, 8, 96]), desc([1, 64, 2, 96]), desc([1, 64, 2, 96]), desc([1, 1, 8, 96])
+    elif case == "head_dim_264":  # above the largest kernel's 256
+        q, k, v, o = desc([1, 1, 8, 264]), desc([1, 64, 2, 264]), desc([1, 64, 2, 264]), desc([1, 1, 8, 264])
+    elif case == "head_dim_12":  # rows of 24 bytes: no 16-byte row stride
+        q, k, v, o = desc([1, 1, 8, 12]), desc([1, 64, 2, 12]), desc([1, 64, 2, 12]), desc([1, 1, 8, 12])
+    elif case == "head_dim_v_264":
+        v, o = desc([1, 64, 2, 264]), desc([1, 1, 8, 264])
     elif case == "last_dim_strided":
         k = desc([1, 64, 2, 128], stride=[64 * 2 * 256, 2 * 256, 256, 2])
     elif case == "stride_not_16B":
@@ -133,6 +138,15 @@ def test_force_tcgen05_form_rejects_unknown():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_cuda_error():
     q, k, v, o = good("q"), good("k"), good("v"), good("o")
+    assert call_fwd(q, k, v, o) == CUDA
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+@pytest.mark.parametrize("dqk,dv", [(8, 8), (32, 32), (40, 40), (80, 80), (96, 96), (112, 112), (160, 128), (160, 160),
+                                    (200, 200), (64, 128), (128, 64), (256, 96)])
+def test_any_multiple_of_8_head_dims_pass_validation(dqk, dv):
+    # validation accepts them; with no device the call then fails on CUDA
+    q, k, v, o = desc([1, 1, 8, dqk]), desc([1, 64, 2, dqk]), desc([1, 64, 2, dv]), desc([1, 1, 8, dv])
     assert call_fwd(q, k, v, o) == CUDA
 
 
