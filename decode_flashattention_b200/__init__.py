@@ -30,7 +30,7 @@ __all__ = [
     "fa_decode_kvcache_append", "fa_fwd_varlen", "flash_attn_varlen_func",
     "flash_attn_func", "flash_attn_with_kvcache",
     "fwd_workspace_size", "kvcache_workspace_size", "hld_as_blhd", "check_status",
-    "last_dispatch", "force_variant", "force_tcgen05_form", "profile_enable", "profile_read", "launch_count",
+    "last_dispatch", "force_variant", "force_tcgen05_form", "test_stall_next_call", "profile_enable", "profile_read", "launch_count",
     "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR", "VARIANT_TCGEN05",
     "TCGEN05_AUTO", "TCGEN05_ONE_TILE", "TCGEN05_TWO_TILES", "TCGEN05_ONE_TILE_MMA",
 ]
@@ -96,6 +96,7 @@ def load_library():
         "fa_last_dispatch": (None, [P(FaDispatchInfo)]),
         "fa_force_variant": (i32, [i32]),
         "fa_force_tcgen05_form": (i32, [i32]),
+        "fa_test_stall_next_call": (i32, [ctypes.c_ulonglong]),
         "fa_profile_enable": (i32, [i32]),
         "fa_profile_read": (i32, [P(ctypes.c_double), P(ctypes.c_int64), P(ctypes.c_double),
                                   P(ctypes.c_int64)]),
@@ -402,6 +403,13 @@ def last_dispatch() -> dict:
 
 def force_variant(variant: int):
     _check(load_library().fa_force_variant(int(variant)))
+
+
+def test_stall_next_call(wait_limit_ns: int):
+    """Test hook: the next split-KV call leaves one pipeline stage empty and
+    bounds its waits by wait_limit_ns, so it ends with FA_ERR_TIMEOUT in the
+    device status word (read by check_status)."""
+    _check(load_library().fa_test_stall_next_call(int(wait_limit_ns)))
 
 
 def force_tcgen05_form(form: int):

@@ -40,6 +40,9 @@ thread_local fa_dispatch_info t_disp = {};
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_force_variant{FA_VARIANT_AUTO};
 std::atomic<int> g_force_tc_form{FA_TCGEN05_AUTO};
+// Test hook (fa_test_stall_next_call): the next call's wait bound, 0 = none pending.
+std::atomic<unsigned long long> g_stall_next{0};
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 
 fa_status fail(fa_status s, const char *fmt, ...) {
     char buf[512];
@@ -543,6 +546,14 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.Lk = s.Lk;
     p.dqk = s.Dqk;
     p.dv = s.Dv;
+    p.wait_limit_ns = kWaitLimitNs;
+    p.stall = 0;
+    if (!pl.prefill) {  // the hook acts on the split-KV kernel
+        if (const unsigned long long lim = g_stall_next.exchange(0)) {
+            p.wait_limit_ns = lim;
+            p.stall = 1;
+        }
+    }
     p.causal = causal ? 1 : 0;
     float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)s.Dqk);
     p.scale_log2 = sc * 1.4426950408889634f;
@@ -963,6 +974,13 @@ fa_status fa_force_variant(int variant) {
     if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_TCGEN05)
         return fail(FA_ERR_INVALID_ARG, "unknown variant %d", variant);
     g_force_variant.store(variant);
+    return FA_OK;
+}
+
+fa_status fa_test_stall_next_call(unsigned long long wait_limit_ns) {
+    if (wait_limit_ns == 0 || wait_limit_ns > kWaitLimitNs)
+        return fail(FA_ERR_INVALID_ARG, "wait limit %llu ns: must be in (0, %llu]", wait_limit_ns, kWaitLimitNs);
+    g_stall_next.store(wait_limit_ns);
     return FA_OK;
 }
 

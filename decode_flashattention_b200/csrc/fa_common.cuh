@@ -33,6 +33,8 @@ struct Params {
     unsigned *status;      // device status word (timeouts)
     int B, Lq, Hq, Hkv, g, R, RB, Lk;
     int dqk, dv;           // the call's head dims (the kernel's DQK / DV may be larger: columns past them are zero)
+    unsigned long long wait_limit_ns;  // bound of every wait on a pipeline barrier
+    int stall;             // test hook: the first CTA leaves its first stage empty
     int causal;
     float scale_log2;      // scale * log2(e)
     int P;                 // CTAs launched

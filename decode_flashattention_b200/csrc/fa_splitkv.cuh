@@ -89,7 +89,6 @@ struct SplitCfg {
     static_assert((KBOX + VBOX) * (TK / 16) <= 64, "paged boxes per tile: at most two per lane");
 };
 
-constexpr uint64_t kWaitLimitNs = 4000000000ull;  // 4 s
 
 template <typename T, int DQK, int DV, int STAGES, bool FMA, int KB = 2>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -164,7 +163,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot = (wk.pos == lo) ? 0 : 1;
             for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
                 const int s = it % STAGES, use = it / STAGES;
-                const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                // test hook: the first CTA leaves its first stage empty (no copy,
+                // no arrival), so its consumers' wait on it runs out
+                if (p.stall && cta == 0 && it == 0) continue;
+                const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
                 if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's control flow uniform
                     stop = true;
                     break;
@@ -247,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool done_sent = false;
         {
             const int use = it / STAGES;
-            bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
             ok = __all_sync(0xffffffffu, ok);
             if (lane == 0) {
                 StageMeta m = {0, 0, 0, 0, kMetaDone, 0, 0, 0};
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (s == s_done && done_sent) continue;
                 const int last_use = (it - 1 - s) / STAGES;
                 volatile int no_abort = 0;
-                mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, kWaitLimitNs / 8);
+                mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
             }
         }
         return;
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool warm = it < 0;
             if (it == 0) pdl_wait_primary();  // outputs and workspace are written below
             const int s = warm ? 0 : it % STAGES, use = warm ? 0 : it / STAGES;
-            const bool ok = warm || mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
+            const bool ok = warm || mbar_wait(full_bar(s), use & 1, abort_flag, p.status, p.wait_limit_ns);
             if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;
             StageMeta md = {0, 0, 0, 0, kMetaFirst | kMetaLast | (it == -1 ? kMetaWhole : 0), 0, 0, 0};
             if (!warm) md = meta[s];
@@ -526,11 +528,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 *reinterpret_cast<float2 *>(dst) = make_float2(acc[0], acc[1]);
             }
-            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
+            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, p.wait_limit_ns)) break;
             merge_store(md, warm, cg);
             // red / sm_m / sm_l are reused by the next segment, if there is one
             if (md.flags & kMetaFinal) break;
-            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
+            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, p.wait_limit_ns)) break;
         }
     } else {
         // ========================================================= tensor-core consumer
@@ -546,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool warm = it < 0;
             if (it == 0) pdl_wait_primary();  // outputs and workspace are written below
             const int s = warm ? 0 : it % STAGES, use = warm ? 0 : it / STAGES;
-            const bool ok = warm || mbar_wait(full_bar(s), use & 1, abort_flag, p.status, kWaitLimitNs);
+            const bool ok = warm || mbar_wait(full_bar(s), use & 1, abort_flag, p.status, p.wait_limit_ns);
             if (__any_sync(0xffffffffu, !ok || *abort_flag)) break;
             StageMeta md = {0, 0, 0, 0, kMetaFirst | kMetaLast | (it == -1 ? kMetaWhole : 0), 0, 0, 0};
             if (!warm) md = meta[s];
@@ -699,11 +701,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     buf[(r_lo + 1) * C::RED_STRIDE + d + 8] = acc[t][3];
                 }
             }
-            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
+            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, p.wait_limit_ns)) break;
             merge_store(md, warm, cg);
             // red / sm_m / sm_l are reused by the next segment, if there is one
             if (md.flags & kMetaFinal) break;
-            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, kWaitLimitNs)) break;
+            if (!consumer_sync_bounded(ep_bar, ep_phase, abort_flag, p.status, p.wait_limit_ns)) break;
         }
     }
 }

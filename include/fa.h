@@ -324,6 +324,18 @@ typedef enum {
 FA_API fa_status fa_force_tcgen05_form(int form);
 
 /*
+ * Test hook for the failure path: the next split-KV compute call of this
+ * process bounds its pipeline waits by wait_limit_ns (instead of 4 s) and its
+ * first CTA leaves its first pipeline stage empty -- no copy, no arrival --
+ * so that CTA's consumers give up after wait_limit_ns, record
+ * FA_ERR_TIMEOUT in the device status word and return (as do the producer,
+ * after a bounded wait for its copies in flight).  The call's outputs are
+ * then unspecified; fa_check_status reports the timeout and later calls run
+ * normally.  FA_ERR_INVALID_ARG unless 0 < wait_limit_ns <= 4e9.
+ */
+FA_API fa_status fa_test_stall_next_call(unsigned long long wait_limit_ns);
+
+/*
  * Profiling: while enabled, each compute call brackets its main kernel and
  * its combine kernel with CUDA events on the call's stream (and launches them
  * without programmatic overlap, so each event pair times one kernel alone).

@@ -127,6 +127,12 @@ def test_force_variant_rejects_unknown():
     assert fa.load_library().fa_force_variant(0) == OK
 
 
+def test_stall_hook_rejects_out_of_range_limits():
+    lib = fa.load_library()
+    assert lib.fa_test_stall_next_call(ctypes.c_ulonglong(0)) == INVALID
+    assert lib.fa_test_stall_next_call(ctypes.c_ulonglong(5_000_000_000)) == INVALID
+
+
 def test_force_tcgen05_form_rejects_unknown():
     lib = fa.load_library()
     assert lib.fa_force_tcgen05_form(4) == INVALID
