@@ -1,35 +1,37 @@
 // fa_prefill.cu -- dense attention for many packed query rows on the 5th-gen
 // tensor cores (tcgen05 + TMEM): the prefill-shaped calls of fa_fwd.
 //
-// One CTA per (batch, kv head, block of 128 packed query rows).  Packed row r
-// of kv head hkv is query head hkv * g + r / Lq at position r % Lq (the same
-// packing as the split-KV kernel), so the g heads of a GQA group share every
-// K / V tile.  The CTA walks all key tiles its rows can see (128 keys each):
+// Packed row r of kv head hkv is query head hkv * g + r / Lq at position
+// r % Lq (the same packing as the split-KV kernel), so the g heads of a GQA
+// group share every K / V tile; a CTA walks all 128-key tiles its rows can
+// see (no split, no combine).  Per tile, for a 128-row query tile:
 //
 //   S  = Q K^T        tcgen05.mma (M 128 rows, N 128 keys, K = head dim),
-//                     fp32 accumulator in TMEM, two buffers: the next
-//                     tile's S is computed while this tile's softmax runs
+//                     fp32 accumulator in TMEM
 //   softmax           one thread per row reads its S row from TMEM
 //                     (tcgen05.ld), masks, and runs the base-2 online
-//                     softmax (running max m, sum l in fp32); P goes to
-//                     shared memory in the operand layout, O in TMEM is
+//                     softmax (running max m, sum l in fp32); O in TMEM is
 //                     rescaled by 2^(m_old - m_new) (tcgen05.ld / st)
 //   O += P V          tcgen05.mma (M 128 rows, N = head dim, K 128 keys),
-//                     fp32 accumulator in TMEM (it runs while the next
-//                     tile's softmax starts)
+//                     fp32 accumulator in TMEM
 //
 // (the tiled online softmax of "昇腾CANN上的FlashAttention工程实战", with the
 // Cube / Vector split of the ops-transformer walkthrough mapped onto the
-// tensor core and the CUDA cores).  A producer warp streams K and V tiles with
-// TMA (128-byte swizzle, the canonical K-major layout for K and the
-// MN-major one for V) into a 2-stage ring; tcgen05.commit releases a stage
-// once its PV product is done.  Every wait is bounded; on a timeout the CTA
-// records the error, waits (bounded) for its last tensor-core work and frees
-// its TMEM before returning.
+// tensor core and the CUDA cores).  K and V arrive by TMA (128-byte swizzle,
+// the canonical K-major layout for K and the MN-major one for V), and
+// tcgen05.commit releases a stage once its products are done.  Two kernels:
 //
-// A second kernel (prefill3_kernel) puts two 128-row query tiles in one CTA
-// with a dedicated MMA warp, so the softmax of one tile overlaps the other
-// tile's products and two softmax warps share each sub-partition.
+//   prefill_kernel    one query tile per CTA; its four softmax warps issue
+//                     the products themselves; S is double-buffered in TMEM
+//                     (the next tile's QK^T runs during this tile's softmax);
+//                     P goes through shared memory
+//   prefill3_kernel   one or two query tiles per CTA, a dedicated MMA warp
+//                     and a TMA warp; with two tiles one tile's products run
+//                     during the other's softmax; P stays in TMEM
+//
+// Every wait is bounded; on a timeout the CTA records the error, waits
+// (bounded) for its last tensor-core work and copies, and frees its TMEM
+// before returning.
 #include <type_traits>
 
 #include "fa.h"

@@ -286,10 +286,11 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      (g * Lq == 1), the "scalar fp32 dot product" form of
  *                      "SmallQ FlashAttention for Ascend 910B", section
  *                      "算法要点".
- *   FA_VARIANT_TCGEN05 one CTA per 128 packed query rows on the 5th-gen tensor
- *                      cores (tcgen05.mma, accumulators in TMEM), whole key
- *                      range per CTA, no split and no combine; dense fa_fwd
- *                      calls with head dims 128/128.
+ *   FA_VARIANT_TCGEN05 the 5th-gen tensor cores (tcgen05.mma, S, P and O in
+ *                      TMEM) on blocks of 128 or 256 packed query rows (see
+ *                      fa_tcgen05_form), whole key range per CTA, no split
+ *                      and no combine; dense fa_fwd calls with head dims
+ *                      128/128.
  * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
  * least 128 packed rows (g * Lq >= 128) and head dims 128/128 (prefill-shaped
  * calls); FA_VARIANT_MMA otherwise -- measured on B200 it is faster than the
