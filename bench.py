@@ -207,12 +207,19 @@ def peaks():
 
 
 def kernel_source_hash():
+    """Hash of the library's CUDA / C++ sources with comments and whitespace
+    removed: it changes when the code does, not when a comment does."""
+    import re
+
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "decode_flashattention_b200", "csrc")
+    strip = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+                text = strip.sub(lambda m: m.group(0) if m.group(0).startswith('"') else " ", fh.read())
+            h.update(f.encode())
+            h.update("".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
