@@ -292,3 +292,26 @@ def test_append_host_validation(case):
                                       0, 0, 0.0, None, 0, None)
     assert st == INVALID
     assert fa.load_library().fa_last_error()
+
+
+def test_missing_library_fails_loudly():
+    # no fallback: without the built library every call raises (fresh interpreter,
+    # the binding pointed at a path that does not exist)
+    import subprocess
+    import sys
+
+    code = (
+        "import torch, decode_flashattention_b200 as fa\n"
+        "fa._LIB_PATH = '/nonexistent/libfa_b200.so'\n"
+        "q = torch.zeros(1, 1, 8, 128, dtype=torch.float16)\n"
+        "k = torch.zeros(1, 64, 2, 128, dtype=torch.float16)\n"
+        "try:\n"
+        "    fa.fa_fwd(q, k, k)\n"
+        "except RuntimeError as e:\n"
+        "    print('raised:', e)\n"
+        "else:\n"
+        "    print('returned')\n"
+    )
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=300)
+    assert "raised:" in out.stdout and "missing" in out.stdout, out.stdout + out.stderr
