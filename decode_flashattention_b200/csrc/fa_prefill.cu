@@ -162,6 +162,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         : "memory");
 }
 
+// Packed fp32 pairs and a three-input max (sm_100): half the instructions of
+// the scalar forms for the softmax's elementwise work.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t pack2f(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack2f(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {  // a * b + c, per lane
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -727,13 +753,16 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
 #pragma unroll
                 for (int e = 0; e < kKeys; ++e) x[e] = key0 + e <= lim ? x[e] : -INFINITY;
             }
+            // row max: eight independent chains of three-input max
             float mxa[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mxa[e] = x[e];
+            for (int e = 0; e < 8; ++e) mxa[e] = fmaxf(x[2 * e], x[2 * e + 1]);
 #pragma unroll
-            for (int e = 8; e < kKeys; ++e) mxa[e & 7] = fmaxf(mxa[e & 7], x[e]);
-            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
+            for (int e = 16; e < kKeys; e += 16)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mxa[c] = max3f(mxa[c], x[e + 2 * c], x[e + 2 * c + 1]);
+            const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]),
+                                   fmaxf(mxa[6], mxa[7])) *
                              p.scale_log2;
             // the running max moves only when this tile's max is more than 2^8 above it
             const float mn = mx > m + kLazyMax ? mx : m;
@@ -744,19 +773,26 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // written over this row's S columns [0, 64) in TMEM: the A operand of
             // PV_g(j).  (The scores are all in registers by now; PV_g(j - 1),
             // which read the previous P there, finished before S_g(j) did.)
-            float suma[4] = {0.f, 0.f, 0.f, 0.f};
+            // y = x * scale_log2 - base on key pairs (one packed FMA), p = 2^y,
+            // sums in two packed accumulators
+            const uint64_t sc2 = pack2f(p.scale_log2, p.scale_log2), nb2 = pack2f(-base, -base);
+            uint64_t sum2[2] = {pack2f(0.f, 0.f), pack2f(0.f, 0.f)};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    const float p0 = fast_exp2(fmaf(x[h * 64 + 2 * c], p.scale_log2, -base));
-                    const float p1 = fast_exp2(fmaf(x[h * 64 + 2 * c + 1], p.scale_log2, -base));
-                    suma[c & 3] += p0 + p1;
+                    float y0, y1;
+                    unpack2f(ffma2(pack2f(x[h * 64 + 2 * c], x[h * 64 + 2 * c + 1]), sc2, nb2), y0, y1);
+                    const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+                    sum2[c & 1] = fadd2(sum2[c & 1], pack2f(p0, p1));
                     pk[c] = Mma<T>::pack(p0, p1);
                 }
                 tmem_st32(t_s + h * 32, pk);
             }
+            float suma[4];
+            unpack2f(sum2[0], suma[0], suma[1]);
+            unpack2f(sum2[1], suma[2], suma[3]);
             // O_g *= alpha where the max moved.  PV_g(j - 1) is complete (it ran
             // before S_g(j)); the wait on its barrier makes that visible here.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
