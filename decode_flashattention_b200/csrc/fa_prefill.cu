@@ -377,27 +377,36 @@ __global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
                 for (int e = 0; e < kKeys; ++e) x[e] = key0 + e <= lim ? x[e] : -INFINITY;
             }
             // row max with independent chains, in base-2 units (scale > 0)
+            // row max: eight independent chains of three-input max
             float mxa[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mxa[e] = x[e];
+            for (int e = 0; e < 8; ++e) mxa[e] = fmaxf(x[2 * e], x[2 * e + 1]);
 #pragma unroll
-            for (int e = 8; e < kKeys; ++e) mxa[e & 7] = fmaxf(mxa[e & 7], x[e]);
-            const float mx = fmaxf(fmaxf(fmaxf(mxa[0], mxa[1]), fmaxf(mxa[2], mxa[3])),
-                                   fmaxf(fmaxf(mxa[4], mxa[5]), fmaxf(mxa[6], mxa[7]))) *
+            for (int e = 16; e < kKeys; e += 16)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mxa[c] = max3f(mxa[c], x[e + 2 * c], x[e + 2 * c + 1]);
+            const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]),
+                                   fmaxf(mxa[6], mxa[7])) *
                              p.scale_log2;
             const float mn = fmaxf(m, mx);
             const float base = mn == -INFINITY ? 0.f : mn;
             const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
-            // p = 2^(x * scale_log2 - base): one FFMA and one ex2 per score
-            float suma[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            // p = 2^(x * scale_log2 - base): one packed FMA per key pair and one
+            // ex2 per score; sums in four packed accumulators
+            const uint64_t sc2 = pack2f(p.scale_log2, p.scale_log2), nb2 = pack2f(-base, -base);
+            uint64_t sum2[4] = {pack2f(0.f, 0.f), pack2f(0.f, 0.f), pack2f(0.f, 0.f), pack2f(0.f, 0.f)};
             uint32_t pk[kKeys / 2];
 #pragma unroll
             for (int e = 0; e < kKeys; e += 2) {
-                const float p0 = fast_exp2(fmaf(x[e], p.scale_log2, -base));
-                const float p1 = fast_exp2(fmaf(x[e + 1], p.scale_log2, -base));
-                suma[(e >> 1) & 7] += p0 + p1;
+                float y0, y1;
+                unpack2f(ffma2(pack2f(x[e], x[e + 1]), sc2, nb2), y0, y1);
+                const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+                sum2[(e >> 1) & 3] = fadd2(sum2[(e >> 1) & 3], pack2f(p0, p1));
                 pk[e / 2] = Mma<T>::pack(p0, p1);
             }
+            float suma[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) unpack2f(sum2[q], suma[2 * q], suma[2 * q + 1]);
             const float sum = ((suma[0] + suma[1]) + (suma[2] + suma[3])) + ((suma[4] + suma[5]) + (suma[6] + suma[7]));
             l = l * alpha + sum;
             m = mn;
