@@ -419,10 +419,17 @@ def run_ours(args):
     fa.check_status()
 
     # --- e2e: through the public API from pinned host buffers -------------------------
-    hins = [t.cpu().pin_memory() for t in ins0]
+    # host buffers with the device tensors' own layout ([H, L, D] storage stays
+    # [H, L, D]), so each copy is one plain memcpy of the storage
+    def pinned_like(t):
+        h = torch.empty_strided(t.size(), t.stride(), dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    hins = [pinned_like(t) for t in ins0]
     hsl = sl0.pin_memory() if sl0 is not None else None
-    ho = torch.empty(outs[0].shape, dtype=w.dtype).pin_memory()
-    hl = torch.empty(lses[0].shape, dtype=torch.float32).pin_memory()
+    ho = torch.empty_strided(outs[0].size(), outs[0].stride(), dtype=w.dtype, pin_memory=True)
+    hl = torch.empty_strided(lses[0].size(), lses[0].stride(), dtype=torch.float32, pin_memory=True)
     dins = [torch.empty_like(t) for t in ins0]
     dsl = torch.empty_like(sl_dev) if sl_dev is not None else None
     h2d = sum(t.numel() * t.element_size() for t in hins) + (hsl.numel() * 4 if hsl is not None else 0)
