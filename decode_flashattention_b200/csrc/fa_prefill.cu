@@ -701,7 +701,10 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     for (int kk = 0; kk < kKeys / 16; ++kk)  // P_g(j): 16 keys = 8 TMEM columns per step
                         umma_ts(tmem + 2 * kKeys + g * kD, tmem + g * kKeys + kk * 8,
                                 dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(o_bar(g));
+                    // O_g is final after the last tile's PV; before that, the commit
+                    // of S_g(j + 1) (issued after PV_g(j), and a commit covers all of
+                    // this thread's earlier products) tells the softmax PV_g(j) is done
+                    if (j + 1 == ntiles) umma_commit(o_bar(g));
                     if (g == ngroups - 1) umma_commit(empty_bar(qv % kSlots));  // V(j) read by its products
                     if (more) {
                         if (g == 0) {
@@ -802,15 +805,9 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             float suma[4];
             unpack2f(sum2[0], suma[0], suma[1]);
             unpack2f(sum2[1], suma[2], suma[3]);
-            // O_g *= alpha where the max moved.  PV_g(j - 1) is complete (it ran
-            // before S_g(j)); the wait on its barrier makes that visible here.
+            // O_g *= alpha where the max moved.  PV_g(j - 1) is complete: S_g(j),
+            // whose barrier this warp waited on, was committed after it.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                ok = mbar_wait(o_bar(grp), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < kD / 64; ++h) {
                     uint32_t v0[32], v1[32];
@@ -832,8 +829,8 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_bar(grp));  // this warp's rows of P(j) are written
         }
-        if (ok && ntiles > 0) {
-            ok = mbar_wait(o_bar(grp), (ntiles - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+        if (ok && ntiles > 0) {  // the one commit of o_bar(grp): after the last PV
+            ok = mbar_wait(o_bar(grp), 0, abort_flag, p.status, kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }
