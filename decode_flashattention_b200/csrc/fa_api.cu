@@ -331,11 +331,16 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     int variant = choose_variant(s);
     // Calls with at least 128 packed rows (prefill-shaped) on dense K / V run on
     // the tcgen05 kernel: 128 rows fill its M side, and the whole key range is
-    // one CTA's work (no split, no combine).
-    const bool tc_shape = !kvcache && s.R >= 128 && s.Dqk == 128 && s.Dv == 128;
+    // one CTA's work (no split, no combine).  Its time is then one CTA's walk
+    // over the keys, so it needs enough CTAs to beat the split-KV kernel, which
+    // spreads the keys over every SM (measured with 64-dim heads: 2 CTAs lose at
+    // every key length, 32 CTAs win from 128 keys on, 128 CTAs win 4-8x).
+    const bool tc_dims = s.Dqk == s.Dv && (s.Dqk == 128 || s.Dqk == 64);
+    const int64_t tc_ctas = (int64_t)((s.R + 127) / 128) * s.Hkv * s.B;
+    const bool tc_shape = !kvcache && s.R >= 128 && tc_dims && tc_ctas >= 32;
     if (variant == FA_VARIANT_TCGEN05 || (g_force_variant.load() == FA_VARIANT_AUTO && tc_shape)) {
-        if (!tc_shape && (kvcache || s.Dqk != 128 || s.Dv != 128))
-            return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 128/128");
+        if (kvcache || !tc_dims)
+            return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 64/64 or 128/128");
         // Two 128-row tiles per CTA while that still gives every SM a CTA (the
         // tiles' softmax and products overlap); with fewer CTAs than SMs one
         // tile per CTA, in the MMA-warp pipeline for a single tile of rows.
@@ -343,10 +348,10 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
         if (form == FA_TCGEN05_AUTO) {
             const int64_t pairs = (int64_t)((s.R + 255) / 256) * s.Hkv * s.B;
             form = pairs >= dev->sms ? FA_TCGEN05_TWO_TILES
-                                     : (s.R <= 128 ? FA_TCGEN05_ONE_TILE_MMA : FA_TCGEN05_ONE_TILE);
+                                     : (s.R <= 128 || s.Dqk != 128 ? FA_TCGEN05_ONE_TILE_MMA : FA_TCGEN05_ONE_TILE);
         }
         if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, form, &pl->main))
-            return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d", s.dtype);
+            return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d, head dim %d, form %d", s.dtype, s.Dqk, form);
         if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
         pl->prefill = true;
         pl->row_blocks = (s.R + pl->main.rows - 1) / pl->main.rows;

@@ -534,27 +534,38 @@ namespace pf3 {
 constexpr int kKeys = 128;
 constexpr int kSlots = 3;
 constexpr int kBox = kKeys * 128;                // one 64-column box of 128 rows (bytes)
-constexpr int kSlotBytes = 2 * kBox;             // a K or V tile: 128 keys x 128 elements
-constexpr int OFF_Q = 0;                         // Q_A, Q_B
-constexpr int OFF_KV = OFF_Q + 2 * pf::kTileQ;
-constexpr int OFF_BAR = OFF_KV + kSlots * kSlotBytes;
 // full[kSlots], empty[kSlots], s_done[2], p_ready[2], o_done[2], q_ready, drain
 constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
-constexpr int OFF_MISC = OFF_BAR + NBAR * 8;     // tmem base, abort flag, 8 warp maxima
-constexpr int SMEM = OFF_MISC + 64 + 1024;       // + alignment slack
 constexpr int kThreads = 320;                    // an MMA warp, a producer warp, 8 softmax warps
 constexpr int kMmaWarp = 0, kProducerWarp = 1, kFirstSoftmaxWarp = 2;
 constexpr uint32_t kTmemCols = 512;              // S_A, S_B, O_A, O_B: 128 columns each
 constexpr float kLazyMax = 8.f;                  // log2 of the largest p before the max moves
-static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+// Shared-memory layout for head dim D (64 or 128): rows of Q, K and V are
+// D / 64 boxes of 64 columns.
+template <int D>
+struct Cfg3 {
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kTileQ = kBoxes * kBox;     // one 128-row query tile
+    static constexpr int kSlotBytes = kBoxes * kBox; // a K or V tile: 128 keys x D
+    static constexpr int OFF_Q = 0;                  // Q_A, Q_B
+    static constexpr int OFF_KV = OFF_Q + 2 * kTileQ;
+    static constexpr int OFF_BAR = OFF_KV + kSlots * kSlotBytes;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, 8 warp maxima
+    static constexpr int SMEM = OFF_MISC + 64 + 1024;    // + alignment slack
+    static_assert(D == 64 || D == 128, "head dims 64 and 128");
+    static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
+    static_assert(2 * kKeys + 2 * D <= (int)kTmemCols, "S_A, S_B, O_A, O_B fit TMEM");
+};
 }  // namespace pf3
 
-// TILES: query tiles per CTA (2; or 1 when two-tile CTAs would leave SMs idle).
-template <typename T, int TILES>
+// TILES: query tiles per CTA (2; or 1 when two-tile CTAs would leave SMs idle);
+// D: head dim (64 or 128, Dqk = Dv).
+template <typename T, int TILES, int D>
 __global__ void __launch_bounds__(pf3::kThreads, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
     using namespace pf;
     using namespace pf3;
+    using L = Cfg3<D>;
     constexpr int kCtaRows = TILES * kRows;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -564,7 +575,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
     // row blocks in reverse order: under a causal mask the late rows see the
     // most keys, so the longest CTAs start first
     const int rb = gridDim.x - 1 - blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
     auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
     auto empty_bar = [&](int s) { return smem_u32(&bars[kSlots + s]); };
     auto s_bar = [&](int g) { return smem_u32(&bars[2 * kSlots + g]); };
@@ -572,9 +583,9 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
     auto o_bar = [&](int g) { return smem_u32(&bars[2 * kSlots + 4 + g]); };
     const uint32_t q_bar = smem_u32(&bars[2 * kSlots + 6]);
     const uint32_t drain_bar = smem_u32(&bars[2 * kSlots + 7]);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-    int *warp_keys = reinterpret_cast<int *>(smem + OFF_MISC + 16);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
+    int *warp_keys = reinterpret_cast<int *>(smem + L::OFF_MISC + 16);
 
     // ---- softmax threads: group, row, head, query position, last visible key
     const bool softmax = warp >= kFirstSoftmaxWarp;
@@ -642,10 +653,11 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             for (int q = 0; q < 2 * ntiles; ++q) {
                 const int s = q % kSlots, use = q / kSlots;
                 if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
-                const uint32_t dst = sb + OFF_KV + s * kSlotBytes;
+                const uint32_t dst = sb + L::OFF_KV + s * L::kSlotBytes;
                 const CUtensorMap *map = (q & 1) ? &tmV : &tmK;
-                mbar_expect_tx(full_bar(s), kSlotBytes);
-                for (int c = 0; c < 2; ++c) tma_load_4d_plain(dst + c * kBox, map, full_bar(s), c * 64, (q >> 1) * kKeys, hkv, b);
+                mbar_expect_tx(full_bar(s), L::kSlotBytes);
+                for (int c = 0; c < L::kBoxes; ++c)
+                    tma_load_4d_plain(dst + c * kBox, map, full_bar(s), c * 64, (q >> 1) * kKeys, hkv, b);
                 mbar_arrive(full_bar(s));
                 issued = q + 1;
             }
@@ -661,22 +673,22 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         // ================================================= MMA issue (one thread)
         if (lane == 0) {
             const uint32_t idesc = instr_desc(bf16, kRows, kKeys, false);   // S: N = 128 keys, K-major K
-            const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);     // PV: N = 128 dims, MN-major V
+            const uint32_t idesc_o = instr_desc(bf16, kRows, D, true);     // PV: N = 128 dims, MN-major V
             // Operand descriptors: a base descriptor plus a constant offset in
             // 16-byte units (every shared address stays below 256 KB, so the sum
             // never carries out of the address field).
-            const uint64_t dq0 = smem_desc(sb + OFF_Q, 16, 1024);
-            const uint64_t dk0 = smem_desc(sb + OFF_KV, 16, 1024);        // a slot holding K
-            const uint64_t dv0 = smem_desc(sb + OFF_KV, kBox, 1024);      // a slot holding V
+            const uint64_t dq0 = smem_desc(sb + L::OFF_Q, 16, 1024);
+            const uint64_t dk0 = smem_desc(sb + L::OFF_KV, 16, 1024);        // a slot holding K
+            const uint64_t dv0 = smem_desc(sb + L::OFF_KV, kBox, 1024);      // a slot holding V
             auto wait = [&](uint32_t bar, uint32_t parity) {
                 return mbar_wait(bar, parity, abort_flag, p.status, kWaitLimitNs);
             };
             // S_g(j) = Q_g K(j)^T; K(j) is ring entry 2j
             auto issue_s = [&](int g, int j) {
-                const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * kSlotBytes) >> 4);
-                const uint64_t dq = dq0 + (uint64_t)((g * kTileQ) >> 4);
+                const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * L::kSlotBytes) >> 4);
+                const uint64_t dq = dq0 + (uint64_t)((g * L::kTileQ) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
+                for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (uint32_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
                     umma(tmem + g * kKeys, dq + off, dk + off, idesc, kk > 0);
                 }
@@ -691,7 +703,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             for (int j = 0; j < ntiles && ok; ++j) {
                 const int qv = 2 * j + 1, qk = 2 * j + 2;  // ring entries of V(j), K(j + 1)
                 const bool more = j + 1 < ntiles;
-                const uint64_t dv = dv0 + (uint64_t)(((qv % kSlots) * kSlotBytes) >> 4);
+                const uint64_t dv = dv0 + (uint64_t)(((qv % kSlots) * L::kSlotBytes) >> 4);
                 for (int g = 0; g < ngroups && ok; ++g) {
                     // P_g(j) written (S_g(j) read, O_g rescaled); V(j) landed
                     ok = wait(p_bar(g), j & 1) && (g > 0 || wait(full_bar(qv % kSlots), (qv / kSlots) & 1));
@@ -699,7 +711,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk)  // P_g(j): 16 keys = 8 TMEM columns per step
-                        umma_ts(tmem + 2 * kKeys + g * kD, tmem + g * kKeys + kk * 8,
+                        umma_ts(tmem + 2 * kKeys + g * D, tmem + g * kKeys + kk * 8,
                                 dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     // O_g is final after the last tile's PV; before that, the commit
                     // of S_g(j + 1) (issued after PV_g(j), and a commit covers all of
@@ -728,9 +740,9 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         {
             const T *qg = reinterpret_cast<const T *>(p.q);
             const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
-            for (int c = 0; c < kD / 8; ++c) {
+            for (int c = 0; c < D / 8; ++c) {
                 const uint32_t dst =
-                    sb + OFF_Q + grp * kTileQ + (c >> 3) * kBoxQ + trow * 128 + ((((c & 7) ^ (trow & 7))) << 4);
+                    sb + L::OFF_Q + grp * L::kTileQ + (c >> 3) * kBoxQ + trow * 128 + ((((c & 7) ^ (trow & 7))) << 4);
                 cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
@@ -739,7 +751,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             if (lane == 0) mbar_arrive(q_bar);
         }
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t t_s = tmem + grp * kKeys + lane_off, t_o = tmem + 2 * kKeys + grp * kD + lane_off;
+        const uint32_t t_s = tmem + grp * kKeys + lane_off, t_o = tmem + 2 * kKeys + grp * D + lane_off;
         float m = -INFINITY, l = 0.f;  // m in base-2 units of the scaled scores
         bool ok = grp < ngroups;  // a group without rows has nothing to do
         for (int j = 0; j < ntiles && ok; ++j) {
@@ -809,7 +821,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // whose barrier this warp waited on, was committed after it.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                for (int h = 0; h < kD / 64; ++h) {
+                for (int h = 0; h < D / 64; ++h) {
                     uint32_t v0[32], v1[32];
                     tmem_ld32(t_o + h * 64, v0);
                     tmem_ld32(t_o + h * 64 + 32, v1);
@@ -838,7 +850,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             const float inv = l > 0.f ? 1.f / l : 0.f;
             T *og = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)qi * p.o_sl + (long long)hq * p.o_sh;
 #pragma unroll
-            for (int c = 0; c < kD / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
                 if (ntiles > 0) {
                     tmem_ld32(t_o + c * 32, v);
@@ -886,11 +898,11 @@ static void fill(KernelInfo *out) {
 // overhead cancelling the second CTA's interleaving.)
 constexpr int kPrefillKeys = 128;
 
-template <typename T, int TILES>
+template <typename T, int TILES, int D>
 static void fill3(KernelInfo *out) {
-    out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES>);
+    out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES, D>);
     out->threads = pf3::kThreads;
-    out->smem = pf3::SMEM;
+    out->smem = pf3::Cfg3<D>::SMEM;
     out->tile_keys = pf3::kKeys;
     out->stages = pf3::kSlots;
     out->variant = 3;  // FA_VARIANT_TCGEN05
@@ -899,19 +911,31 @@ static void fill3(KernelInfo *out) {
 }
 
 bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out) {
-    if (dqk != 128 || dv != 128 || dtype < 0 || dtype > 1) return false;
+    if (dtype < 0 || dtype > 1 || dqk != dv || (dqk != 64 && dqk != 128)) return false;
+    const bool h = dtype == 0;
     switch (form) {
-    case FA_TCGEN05_ONE_TILE:
-        if (dtype == 0) fill<__half, kPrefillKeys>(out);
+    case FA_TCGEN05_ONE_TILE:  // head dim 128 only
+        if (dqk != 128) return false;
+        if (h) fill<__half, kPrefillKeys>(out);
         else fill<__nv_bfloat16, kPrefillKeys>(out);
         return true;
     case FA_TCGEN05_TWO_TILES:
-        if (dtype == 0) fill3<__half, 2>(out);
-        else fill3<__nv_bfloat16, 2>(out);
+        if (dqk == 64) {
+            if (h) fill3<__half, 2, 64>(out);
+            else fill3<__nv_bfloat16, 2, 64>(out);
+        } else {
+            if (h) fill3<__half, 2, 128>(out);
+            else fill3<__nv_bfloat16, 2, 128>(out);
+        }
         return true;
     case FA_TCGEN05_ONE_TILE_MMA:
-        if (dtype == 0) fill3<__half, 1>(out);
-        else fill3<__nv_bfloat16, 1>(out);
+        if (dqk == 64) {
+            if (h) fill3<__half, 1, 64>(out);
+            else fill3<__nv_bfloat16, 1, 64>(out);
+        } else {
+            if (h) fill3<__half, 1, 128>(out);
+            else fill3<__nv_bfloat16, 1, 128>(out);
+        }
         return true;
     default:
         return false;

@@ -97,7 +97,7 @@ typedef enum fa_variant {
     FA_VARIANT_AUTO = 0,
     FA_VARIANT_MMA = 1,     /* split-KV kernel, mma.sync tensor-core products */
     FA_VARIANT_SCALAR = 2,  /* split-KV kernel, fp32 FMA products (one packed row) */
-    FA_VARIANT_TCGEN05 = 3  /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 128/128) */
+    FA_VARIANT_TCGEN05 = 3  /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 64/64 or 128/128) */
 } fa_variant;
 
 typedef struct fa_dispatch_info {
@@ -290,10 +290,10 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      TMEM) on blocks of 128 or 256 packed query rows (see
  *                      fa_tcgen05_form), whole key range per CTA, no split
  *                      and no combine; dense fa_fwd calls with head dims
- *                      128/128.
+ *                      64/64 or 128/128.
  * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
- * least 128 packed rows (g * Lq >= 128) and head dims 128/128 (prefill-shaped
- * calls); FA_VARIANT_MMA otherwise -- measured on B200 it is faster than the
+ * least 128 packed rows (g * Lq >= 128) and head dims 64/64 or 128/128
+ * (prefill-shaped calls); FA_VARIANT_MMA otherwise -- measured on B200 it is faster than the
  * FMA variant even for one packed row.  A forced variant that does not
  * support the call's shapes makes the call fail with FA_ERR_UNSUPPORTED.
  */
@@ -304,14 +304,15 @@ FA_API fa_status fa_force_variant(int variant);
  * K / V tiles, accumulators in TMEM, the whole key range per CTA):
  *   FA_TCGEN05_ONE_TILE       one tile per CTA; the softmax warps issue the
  *                             products themselves and S is double-buffered, so
- *                             the next tile's QK^T runs during this tile's softmax;
+ *                             the next tile's QK^T runs during this tile's softmax
+ *                             (head dim 128 only);
  *   FA_TCGEN05_TWO_TILES      two tiles per CTA and a dedicated MMA warp: one
  *                             tile's products run while the other tile's
  *                             softmax does (S single-buffered per tile);
  *   FA_TCGEN05_ONE_TILE_MMA   the two-tile kernel's pipeline with one tile.
  * The library's choice: two tiles when that still gives every SM a CTA
  * (ceil(R / 256) * Hkv * B >= SMs), else the MMA-warp pipeline for calls of at
- * most 128 packed rows, else one tile per CTA.
+ * most 128 packed rows or head dim 64, else one tile per CTA.
  */
 typedef enum {
     FA_TCGEN05_AUTO = 0,

@@ -1,7 +1,8 @@
-"""GPU parity of the tcgen05 kernel (dense fa_fwd with >= 128 packed rows,
-head dims 128/128) against the oracle: ragged query and key lengths, causal
-bottom-right alignment including rows with no visible key, GQA packing,
-fp16 / bf16, several batches; full-size prefill on sampled rows."""
+"""GPU parity of the tcgen05 kernels (dense fa_fwd with >= 128 packed rows,
+head dims 128/128, and 64/64 in the two-tile kernel's forms) against the
+oracle: ragged query and key lengths, causal bottom-right alignment
+including rows with no visible key, GQA packing, fp16 / bf16, several
+batches; full-size prefill on sampled rows."""
 import numpy as np
 import pytest
 import torch
@@ -43,6 +44,7 @@ def test_tcgen05_parity(case, dt):
     w = wl.Workload("pf", "fwd", "blhd", dt, B=B, Lq=Lq, Hq=Hq, Hkv=Hkv, Lk=Lk, Dqk=128, Dv=128, causal=causal,
                     seed=Lq + Lk)
     q, k, v, _ = wl.make_inputs(w, DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)  # small calls would otherwise go to the split-KV kernel
     o, lse = fa.fa_fwd(q, k, v, causal=causal)
     torch.cuda.synchronize()
     assert fa.last_dispatch()["variant"] == fa.VARIANT_TCGEN05
@@ -104,14 +106,54 @@ def test_every_form_parity(form, case):
     compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 form {form}")
 
 
-def test_automatic_form_choice():
+def test_automatic_kernel_and_form_choice():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    for (B, Lq, Hq, Hkv), want in (((1, 4096, 32, 8), fa.TCGEN05_TWO_TILES),   # 64 x 8 two-tile CTAs
-                                   ((1, 300, 16, 16), fa.TCGEN05_ONE_TILE),    # 2 x 16 two-tile CTAs
-                                   ((2, 32, 32, 8), fa.TCGEN05_ONE_TILE_MMA)):  # 128 rows, 16 CTAs
-        assert ((B > 0) and ((Lq * Hq // Hkv + 255) // 256) * Hkv * B >= sms) == (want == fa.TCGEN05_TWO_TILES)
-        q = torch.zeros(B, Lq, Hq, 128, dtype=torch.bfloat16, device=DEV)
-        k = torch.zeros(B, 256, Hkv, 128, dtype=torch.bfloat16, device=DEV)
+    for (B, Lq, Hq, Hkv, D), (var, form) in (
+            ((1, 4096, 32, 8, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_TWO_TILES)),   # 64 x 8 two-tile CTAs
+            ((1, 300, 16, 16, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE)),    # 2 x 16 two-tile CTAs
+            ((4, 32, 32, 8, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),  # 128 rows, 32 CTAs
+            ((4, 32, 32, 8, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),   # the same with 64-dim heads
+            ((1, 300, 16, 16, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)), # 64-dim heads: no serial form
+            ((2, 32, 32, 8, 128), (fa.VARIANT_MMA, 0)),                            # 16 CTAs: split-KV kernel
+            ((1, 32, 8, 2, 64), (fa.VARIANT_MMA, 0))):                             # 2 CTAs (the 64-key prefill)
+        if form == fa.TCGEN05_TWO_TILES:
+            assert ((Lq * Hq // Hkv + 255) // 256) * Hkv * B >= sms
+        q = torch.zeros(B, Lq, Hq, D, dtype=torch.bfloat16, device=DEV)
+        k = torch.zeros(B, 256, Hkv, D, dtype=torch.bfloat16, device=DEV)
         fa.fa_fwd(q, k, k, causal=True)
         torch.cuda.synchronize()
-        assert fa.last_dispatch()["tcgen05_form"] == want
+        d = fa.last_dispatch()
+        assert (d["variant"], d["tcgen05_form"]) == (var, form), ((B, Lq, Hq, Hkv, D), d)
+
+
+HD64_CASES = [  # B, Lq, Hq, Hkv, Lk, causal
+    (1, 200, 2, 1, 300, True), (2, 130, 4, 2, 129, False), (1, 32, 8, 2, 128, True), (1, 300, 2, 1, 100, True),
+    (1, 1000, 4, 4, 2000, True),
+]
+
+
+@pytest.mark.parametrize("form", [fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA])
+@pytest.mark.parametrize("case", HD64_CASES, ids=[str(c) for c in HD64_CASES])
+def test_head_dim_64_parity(form, case):
+    B, Lq, Hq, Hkv, Lk, causal = case
+    dt = torch.float16 if (Lq + form) % 2 else torch.bfloat16
+    w = wl.Workload("pf64", "fwd", "blhd", dt, B=B, Lq=Lq, Hq=Hq, Hkv=Hkv, Lk=Lk, Dqk=64, Dv=64, causal=causal,
+                    seed=Lq + Lk + 64 * form)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)
+    fa.force_tcgen05_form(form)
+    o, lse = fa.fa_fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    d = fa.last_dispatch()
+    assert d["variant"] == fa.VARIANT_TCGEN05 and d["tcgen05_form"] == form
+    ro, rl = oracle_full(q, k, v, causal)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 hd64 form {form}")
+
+
+def test_head_dim_64_one_tile_form_is_refused():
+    q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16, device=DEV)
+    k = torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16, device=DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)
+    fa.force_tcgen05_form(fa.TCGEN05_ONE_TILE)
+    with pytest.raises(fa.FaError, match="tcgen05"):
+        fa.fa_fwd(q, k, k, causal=True)
