@@ -514,22 +514,23 @@ __global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
 }
 
 // ---------------------------------------------------------------------------
-// Two query tiles per CTA with 128-key K / V tiles: every tensor-core product
-// is M 128 x N 128, and per 128 keys the MMA warp issues 32 products, five
-// commits and two waits.  K and V tiles stream separately through a ring of
-// three 32 KB slots (K(j), V(j), K(j + 1), ...).  S is single-buffered per
-// group; per tile j the MMA warp issues, for group A then group B,
+// Two query tiles per CTA with 128-key K / V tiles (the kernel also runs
+// with one tile): every QK^T product is M 128 x N 128 x K 16, every PV product
+// M 128 x N D x K 16, and per 128 keys the MMA warp issues 32 products (16
+// for D = 64) with four commits and two waits.  K and V tiles stream
+// separately through a ring of three slots (K(j), V(j), K(j + 1), ...; 128
+// keys x D each).  S is single-buffered per group; per tile j the MMA warp
+// issues, for group A then group B,
 //   PV_g(j) once the group has written P_g(j) (so it has read S_g(j)),
-//   S_g(j + 1) right behind it (the tensor core runs them in order),
+//   S_g(j + 1) right behind it (the tensor core runs one thread's products
+//   in order),
 // so one group's products run while the other group's softmax does.  P stays
-// in TMEM: the softmax writes it (two 16-bit values per 32-bit column) over the
-// S columns it has just read, and PV_g(j) takes its A operand from there, so
-// P costs no shared-memory bandwidth (the S products already use all of it:
-// Q and K reads of 8 KB per 64-cycle M 128 x N 128 x K 16 product).  The
-// softmax keeps a
-// running max m that only moves when a tile's max exceeds it by more than
-// 2^8 (p = 2^(s - m) then stays below 256, exact in fp32 and representable
-// in the 16-bit P), so O is rescaled only on those tiles.
+// in TMEM: the softmax writes it (two 16-bit values per 32-bit column) over
+// the S columns it has just read, and PV_g(j) takes its A operand from there,
+// so P never goes through shared memory.  The softmax keeps a running max m
+// that only moves when a tile's max exceeds it by more than 2^8 (p = 2^(s - m)
+// then stays below 256, exact in fp32 and representable in the 16-bit P), so
+// O is rescaled only on those tiles.
 namespace pf3 {
 constexpr int kKeys = 128;
 constexpr int kSlots = 3;
@@ -538,7 +539,7 @@ constexpr int kBox = kKeys * 128;                // one 64-column box of 128 row
 constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
 constexpr int kThreads = 320;                    // an MMA warp, a producer warp, 8 softmax warps
 constexpr int kMmaWarp = 0, kProducerWarp = 1, kFirstSoftmaxWarp = 2;
-constexpr uint32_t kTmemCols = 512;              // S_A, S_B, O_A, O_B: 128 columns each
+constexpr uint32_t kTmemCols = 512;              // S_A, S_B (128 columns each), O_A, O_B (D each)
 constexpr float kLazyMax = 8.f;                  // log2 of the largest p before the max moves
 // Shared-memory layout for head dim D (64 or 128): rows of Q, K and V are
 // D / 64 boxes of 64 columns.
