@@ -343,12 +343,11 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
             return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 64/64 or 128/128");
         // Two 128-row tiles per CTA while that still gives every SM a CTA (the
         // tiles' softmax and products overlap); with fewer CTAs than SMs one
-        // tile per CTA, in the MMA-warp pipeline for a single tile of rows.
+        // tile per CTA, in the same MMA-warp pipeline with S double-buffered.
         int form = g_force_tc_form.load();
         if (form == FA_TCGEN05_AUTO) {
             const int64_t pairs = (int64_t)((s.R + 255) / 256) * s.Hkv * s.B;
-            form = pairs >= dev->sms ? FA_TCGEN05_TWO_TILES
-                                     : (s.R <= 128 || s.Dqk != 128 ? FA_TCGEN05_ONE_TILE_MMA : FA_TCGEN05_ONE_TILE);
+            form = pairs >= dev->sms ? FA_TCGEN05_TWO_TILES : FA_TCGEN05_ONE_TILE_MMA;
         }
         if (!fa::get_prefill_kernel(s.dtype, s.Dqk, s.Dv, form, &pl->main))
             return fail(FA_ERR_UNSUPPORTED, "no tcgen05 kernel for dtype %d, head dim %d, form %d", s.dtype, s.Dqk, form);

@@ -696,6 +696,54 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                 umma_commit(s_bar(g));
             };
             bool ok = ntiles > 0 && wait(q_bar, 0) && wait(full_bar(0), 0);
+            if constexpr (TILES == 1) {
+                // One tile: S double-buffered in TMEM columns [0, 128) and
+                // [128, 256) (the second tile's, unused), so S(j + 1) is issued as
+                // soon as K(j + 1) has landed and its softmax can start while PV(j)
+                // runs.  S(j + 1)'s buffer last held P(j - 1), read by PV(j - 1),
+                // which was issued before it.
+                auto issue_s1 = [&](int j) {
+                    const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * L::kSlotBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (uint32_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
+                        umma(tmem + (j & 1) * kKeys, dq0 + off, dk + off, idesc, kk > 0);
+                    }
+                    umma_commit(s_bar(j & 1));
+                };
+                if (ok) {
+                    tc_fence_after();
+                    issue_s1(0);
+                    umma_commit(empty_bar(0));
+                }
+                for (int j = 0; j < ntiles && ok; ++j) {
+                    const int qv = 2 * j + 1, qk = 2 * j + 2;  // ring entries of V(j), K(j + 1)
+                    bool next = j + 1 >= ntiles;
+                    if (!next && mbar_try_wait(full_bar(qk % kSlots), (qk / kSlots) & 1)) {
+                        tc_fence_after();
+                        issue_s1(j + 1);
+                        umma_commit(empty_bar(qk % kSlots));
+                        next = true;
+                    }
+                    ok = wait(p_bar(0), j & 1) && wait(full_bar(qv % kSlots), (qv / kSlots) & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint64_t dv = dv0 + (uint64_t)(((qv % kSlots) * L::kSlotBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < kKeys / 16; ++kk)
+                        umma_ts(tmem + 2 * kKeys, tmem + (j & 1) * kKeys + kk * 8, dv + (uint64_t)((kk * 2048) >> 4),
+                                idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(o_bar(0));  // every tile: the softmax's rescale and the epilogue wait on it
+                    umma_commit(empty_bar(qv % kSlots));
+                    if (!next) {
+                        ok = wait(full_bar(qk % kSlots), (qk / kSlots) & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s1(j + 1);
+                        umma_commit(empty_bar(qk % kSlots));
+                    }
+                }
+            } else {
             if (ok) {
                 tc_fence_after();
                 for (int g = 0; g < ngroups; ++g) issue_s(g, 0);
@@ -730,6 +778,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     }
                 }
             }
+            }
             // every product this thread issued is done before TMEM can be freed
             umma_commit(drain_bar);
             volatile int no_abort = 0;
@@ -752,11 +801,14 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             if (lane == 0) mbar_arrive(q_bar);
         }
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t t_s = tmem + grp * kKeys + lane_off, t_o = tmem + 2 * kKeys + grp * D + lane_off;
+        const uint32_t t_o = tmem + 2 * kKeys + grp * D + lane_off;
         float m = -INFINITY, l = 0.f;  // m in base-2 units of the scaled scores
         bool ok = grp < ngroups;  // a group without rows has nothing to do
         for (int j = 0; j < ntiles && ok; ++j) {
-            ok = mbar_wait(s_bar(grp), j & 1, abort_flag, p.status, kWaitLimitNs);
+            // this tile's S: the group's buffer (two tiles), or buffer j % 2 (one tile)
+            const uint32_t t_s = tmem + (TILES == 2 ? grp : (j & 1)) * kKeys + lane_off;
+            ok = TILES == 2 ? mbar_wait(s_bar(grp), j & 1, abort_flag, p.status, kWaitLimitNs)
+                            : mbar_wait(s_bar(j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -818,9 +870,18 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             float suma[4];
             unpack2f(sum2[0], suma[0], suma[1]);
             unpack2f(sum2[1], suma[2], suma[3]);
-            // O_g *= alpha where the max moved.  PV_g(j - 1) is complete: S_g(j),
-            // whose barrier this warp waited on, was committed after it.
+            // O_g *= alpha where the max moved.  With two tiles PV_g(j - 1) is
+            // complete: S_g(j), whose barrier this warp waited on, was committed
+            // after it; with one tile S(j) may have gone first, so wait for it.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if constexpr (TILES == 1) {
+                    ok = mbar_wait(o_bar(0), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                    if (!__all_sync(0xffffffffu, ok)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
 #pragma unroll
                 for (int h = 0; h < D / 64; ++h) {
                     uint32_t v0[32], v1[32];
@@ -842,8 +903,12 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(p_bar(grp));  // this warp's rows of P(j) are written
         }
-        if (ok && ntiles > 0) {  // the one commit of o_bar(grp): after the last PV
-            ok = mbar_wait(o_bar(grp), 0, abort_flag, p.status, kWaitLimitNs);
+        if (ok && ntiles > 0) {
+            // the last PV: with two tiles o_bar's one commit; with one tile the
+            // MMA thread's final (drain) commit -- up to two of o_bar's per-tile
+            // phases can still be open here, which a parity wait cannot tell apart
+            ok = TILES == 2 ? mbar_wait(o_bar(grp), 0, abort_flag, p.status, kWaitLimitNs)
+                            : mbar_wait(drain_bar, 0, abort_flag, p.status, kWaitLimitNs);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }

@@ -305,14 +305,15 @@ FA_API fa_status fa_force_variant(int variant);
  *   FA_TCGEN05_ONE_TILE       one tile per CTA; the softmax warps issue the
  *                             products themselves and S is double-buffered, so
  *                             the next tile's QK^T runs during this tile's softmax
- *                             (head dim 128 only);
+ *                             (head dim 128 only; an earlier design, kept for
+ *                             comparison -- the library no longer chooses it);
  *   FA_TCGEN05_TWO_TILES      two tiles per CTA and a dedicated MMA warp: one
  *                             tile's products run while the other tile's
  *                             softmax does (S single-buffered per tile);
- *   FA_TCGEN05_ONE_TILE_MMA   the two-tile kernel's pipeline with one tile.
+ *   FA_TCGEN05_ONE_TILE_MMA   the two-tile kernel's pipeline with one tile, S
+ *                             double-buffered.
  * The library's choice: two tiles when that still gives every SM a CTA
- * (ceil(R / 256) * Hkv * B >= SMs), else the MMA-warp pipeline for calls of at
- * most 128 packed rows or head dim 64, else one tile per CTA.
+ * (ceil(R / 256) * Hkv * B >= SMs), else FA_TCGEN05_ONE_TILE_MMA.
  */
 typedef enum {
     FA_TCGEN05_AUTO = 0,

@@ -110,7 +110,7 @@ def test_automatic_kernel_and_form_choice():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     for (B, Lq, Hq, Hkv, D), (var, form) in (
             ((1, 4096, 32, 8, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_TWO_TILES)),   # 64 x 8 two-tile CTAs
-            ((1, 300, 16, 16, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE)),    # 2 x 16 two-tile CTAs
+            ((1, 300, 16, 16, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),  # 2 x 16 two-tile CTAs
             ((4, 32, 32, 8, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),  # 128 rows, 32 CTAs
             ((4, 32, 32, 8, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),   # the same with 64-dim heads
             ((1, 300, 16, 16, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)), # 64-dim heads: no serial form
