@@ -21,13 +21,14 @@
 // the canonical K-major layout for K and the MN-major one for V), and
 // tcgen05.commit releases a stage once its products are done.  Two kernels:
 //
-//   prefill_kernel    one query tile per CTA; its four softmax warps issue
-//                     the products themselves; S is double-buffered in TMEM
-//                     (the next tile's QK^T runs during this tile's softmax);
-//                     P goes through shared memory
 //   prefill3_kernel   one or two query tiles per CTA, a dedicated MMA warp
 //                     and a TMA warp; with two tiles one tile's products run
-//                     during the other's softmax; P stays in TMEM
+//                     during the other's softmax, with one tile S is
+//                     double-buffered; P stays in TMEM (the library's choice)
+//   prefill_kernel    an earlier design kept for comparison (reached only by
+//                     forcing its form): one query tile per CTA whose four
+//                     softmax warps issue the products themselves, S
+//                     double-buffered in TMEM, P through shared memory
 //
 // Every wait is bounded; on a timeout the CTA records the error, waits
 // (bounded) for its last tensor-core work and copies, and frees its TMEM
