@@ -2,21 +2,29 @@
 attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--per-config all|none|names]
 
 One step = one full call of the public API (host plan, split-KV kernel and,
 when needed, the LSE combine kernel) over one batch of synthetic input
-already resident in HBM.  Inputs rotate over enough copies to exceed 4x the
-126 MB L2, so K/V bytes come from HBM.  The timed steps are replayed from
-CUDA graphs (captured calls of the same API) and timed with CUDA events on
-the launching stream; N > 1 runs independent replicas (one per GPU) and
-reports the max time over ranks.
+already resident in HBM.  The headline workload is the largest single-GPU
+configuration (MLA-shaped speculative decode, B8 qLen8 H128 192/128,
+16384 keys; --workload picks another).  Inputs rotate over enough copies to
+exceed 4x the 126 MB L2, so K/V bytes come from HBM.  The K timed steps are
+replayed from CUDA graphs (captured calls of the same API) and timed with
+CUDA events on the launching stream, a short spin kernel queued ahead so the
+host's submission is off the clock; the same graph is replayed again to
+give the spread (median, p10, p90) of µs/call.  N > 1 runs independent
+replicas (one per GPU) and reports the max time over ranks.
 
 Printed (rank 0, one JSON line): value = algorithmic K/V bytes of all ranks
-per second (TB/s); ms_per_step; roofline of the split-KV kernel (its own
-CUDA-event duration, measured in a second pass with the library's event
-profiling); e2e = the same metric through the public API with pinned host
-buffers and the host<->device copies inside the timed region; cpu_baseline =
-the fp64 oracle on the host cores over a bounded sample.
+per second (TB/s); ms_per_step; eager µs/call (calls issued one by one, the
+host side of each call on the clock); roofline of the split-KV kernel (the
+whole call's time charged to it, with each kernel's isolated CUDA-event
+duration for its share); e2e = the same metric through the public API with
+pinned host buffers and the host<->device copies inside the timed region;
+cpu_baseline = the fp64 oracle on the host cores over a bounded sample; and
+per_config = the same measurements for each of the five configurations
+C1-C5 (graphs of >= 100 calls, median / p10 / p90 over replays).
 """
 from __future__ import annotations
 
@@ -46,12 +54,19 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--num-splits", type=int, default=0)
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of graph replays")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="bound of the oracle CPU sample")
     ap.add_argument("--variant", choices=["auto", "mma", "scalar"], default="auto",
                     help="force the split-KV kernel's variant (tensor-core or fp32 FMA)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (a reduced case, e.g. for an ncu capture)")
+    ap.add_argument("--reps", type=int, default=10, help="extra replays of the timed graph (µs/call spread)")
+    ap.add_argument("--per-config", default="all",
+                    help="configurations timed into the per_config block: all (C1-C5), none, or names")
+    ap.add_argument("--config-calls", type=int, default=200, help="calls per timed replay of a per_config entry")
+    ap.add_argument("--config-reps", type=int, default=11, help="timed replays of a per_config entry")
+    ap.add_argument("--config-e2e-steps", type=int, default=2)
+    ap.add_argument("--config-cpu-seconds", type=float, default=3.0)
     return ap.parse_args()
 
 
@@ -285,6 +300,254 @@ def cpu_baseline(w, ins, seqlens, seconds: float):
 
 
 # ------------------------------------------------------------------ our arm
+class Case:
+    """One workload set up on the device: rotating input copies (together
+    more than 4x L2, so K/V bytes come from HBM on every call), outputs,
+    workspace, and the public call."""
+
+    def __init__(self, w, device, rank, num_splits):
+        import torch
+
+        import decode_flashattention_b200 as fa
+        from decode_flashattention_b200 import workloads as wl
+
+        self.w = w
+        self.device = device
+        self.num_splits = num_splits
+
+        def draw(seed):
+            if w.call == "paged":
+                q, kp, vp, bt, sl = wl.make_paged_inputs(w, device, seed=seed)
+                return (q, kp, vp, bt), sl
+            q, k, v, sl = wl.make_inputs(w, device, seed=seed)
+            return (q, k, v), sl
+
+        self.ins0, self.sl0 = draw(w.seed + 1000 * rank)
+        q0 = self.ins0[0]
+        self.per_copy = sum(t.numel() * t.element_size() for t in self.ins0)
+        self.n_copies = max(1, math.ceil(4 * L2_BYTES / max(self.per_copy, 1)))
+        self.copies = [self.ins0] + [draw(w.seed + 1000 * rank + c)[0] for c in range(1, self.n_copies)]
+        self.sl_dev = self.sl0.to(device) if self.sl0 is not None else None
+        self.outs = [wl.empty_output(w, q0) for _ in range(self.n_copies)]
+        self.lses = [torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device)
+                     for _ in range(self.n_copies)]
+        if w.call == "paged":
+            ws_bytes = fa.paged_workspace_size(q0, self.ins0[1], self.ins0[2], self.ins0[3].shape[1], num_splits)
+        elif w.call == "kvcache":
+            ws_bytes = fa.kvcache_workspace_size(*self.ins0, num_splits)
+        else:
+            ws_bytes = fa.fwd_workspace_size(*self.ins0, w.causal, num_splits)
+        self.ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+        self.bytes_per_step = wl.kv_bytes(w, self.sl0)
+        self.flops_per_step = wl.attn_flops(w, self.sl0)
+
+    def call(self, ins, sl, o, l):
+        import decode_flashattention_b200 as fa
+
+        w, ns, ws = self.w, self.num_splits, self.ws
+        if w.call == "paged":
+            return fa.fa_decode_kvcache_paged(*ins, sl, causal=w.causal, num_splits=ns, out=o, lse=l, workspace=ws)
+        if w.call == "kvcache":
+            return fa.fa_decode_kvcache(*ins, sl, causal=w.causal, num_splits=ns, out=o, lse=l, workspace=ws)
+        return fa.fa_fwd(*ins, causal=w.causal, num_splits=ns, out=o, lse=l, workspace=ws)
+
+    def step(self, i):
+        c = i % self.n_copies
+        self.call(self.copies[c], self.sl_dev, self.outs[c], self.lses[c])
+
+    def graphs(self, K):
+        """CUDA graphs replaying K calls of the public API (chunks of at most
+        2000 calls); returns (graphs, our kernel launches they hold)."""
+        import torch
+
+        import decode_flashattention_b200 as fa
+
+        out, launches, done = [], 0, 0
+        while done < K:
+            n = min(2000, K - done)
+            n0 = fa.launch_count()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(done, done + n):
+                    self.step(i)
+            launches += fa.launch_count() - n0
+            out.append(g)
+            done += n
+        for g in out:  # warm the graphs themselves
+            g.replay()
+        torch.cuda.synchronize()
+        return out, launches
+
+
+def lead_sleep():
+    """Queue ~0.2 ms of device work ahead of a timed region, so the host has
+    submitted the region's work before its first event fires: the events then
+    time the device, not the host's launch latency."""
+    import torch
+
+    torch.cuda._sleep(int(4e5))
+
+
+def replay_ms(graphs, stream):
+    """Device time of one replay of `graphs` (CUDA events on the stream)."""
+    import torch
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lead_sleep()
+    e0.record(stream)
+    for g in graphs:
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def pct(xs, q):
+    xs = sorted(xs)
+    if not xs:
+        return None
+    i = min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))
+    return xs[i]
+
+
+def e2e_measure(case, E, world, device):
+    """The metric through the public API from pinned host buffers: every step
+    copies its inputs host -> device, calls, and copies O and lse back."""
+    import torch
+
+    w = case.w
+
+    def pinned_like(t):
+        # the device tensor's own layout ([H, L, D] storage stays [H, L, D]),
+        # so each copy is one plain memcpy of the storage
+        h = torch.empty_strided(t.size(), t.stride(), dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    hins = [pinned_like(t) for t in case.ins0]
+    hsl = case.sl0.pin_memory() if case.sl0 is not None else None
+    o0, l0 = case.outs[0], case.lses[0]
+    ho = torch.empty_strided(o0.size(), o0.stride(), dtype=w.dtype, pin_memory=True)
+    hl = torch.empty_strided(l0.size(), l0.stride(), dtype=torch.float32, pin_memory=True)
+    dins = [torch.empty_like(t) for t in case.ins0]
+    dsl = torch.empty_like(case.sl_dev) if case.sl_dev is not None else None
+    h2d = sum(t.numel() * t.element_size() for t in hins) + (hsl.numel() * 4 if hsl is not None else 0)
+    d2h = ho.numel() * ho.element_size() + hl.numel() * 4
+    stream = torch.cuda.current_stream(device)
+
+    def e2e_step():
+        for d, h in zip(dins, hins):
+            d.copy_(h, non_blocking=True)
+        if dsl is not None:
+            dsl.copy_(hsl, non_blocking=True)
+        o, l = case.call(dins, dsl, o0, l0)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(l, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    x1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(x0.elapsed_time(x1), world, device)
+    total = sum_over_ranks(case.bytes_per_step * E, world, device)
+    del dins, hins
+    return {"value": round(total / (ms / 1e3) / 1e12, 5), "unit": "TB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": ms / E}
+
+
+def isolated_kernels(case, Kb):
+    """Each kernel's own duration: the library brackets its launches with CUDA
+    events on the call's stream (and launches them without programmatic
+    overlap, so each event pair times one kernel alone).  A spin kernel ahead
+    of the calls lets the host queue them all before the first runs, so no
+    host launch gap falls between an event and its kernel."""
+    import torch
+
+    import decode_flashattention_b200 as fa
+
+    fa.profile_enable(True)
+    torch.cuda._sleep(int(40e6))  # about 20 ms of device time
+    for i in range(Kb):
+        case.step(i)
+    torch.cuda.synchronize()
+    prof = fa.profile_read()
+    fa.profile_enable(False)
+    fa.check_status()
+    return prof
+
+
+def hbm_roofline(case, us_per_call, prof, peak, peak_kind, traffic):
+    b = case.bytes_per_step
+    achieved = b / (us_per_call / 1e6) / 1e9
+    main_iso = prof["main_ms"] / max(prof["main_launches"], 1)
+    comb_iso = prof["combine_ms"] / max(prof["main_launches"], 1)  # per step (0 when no combine ran)
+    share_main = main_iso / (main_iso + comb_iso) if main_iso + comb_iso > 0 else 1.0
+    return {
+        "bound": "hbm",
+        "kernel": "split-KV kernel, charged with the whole call (combine and boundaries included)",
+        "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+        "frac": round(achieved / peak, 4), "traffic": traffic, "algorithmic_bytes_per_launch": b,
+        "kernel_us": round(us_per_call, 3),
+        "duration_method": "CUDA events on the launching stream around the timed region / calls (whole call)",
+        "share": round(share_main, 4),
+        "isolated_us": {"splitkv": round(main_iso * 1e3, 3),
+                        "combine": round(prof["combine_ms"] / max(prof["combine_launches"], 1) * 1e3, 3)},
+        "isolated_launches": prof["main_launches"],
+    }
+
+
+def config_entry(w, world, rank, device, args, reuse=None):
+    """Per-config block: µs/call (median, p10, p90 over repeated timed
+    replays of a graph of >= 100 calls), TB/s, fraction of the measured peak,
+    ncu traffic, e2e and the oracle's CPU baseline."""
+    import torch
+
+    import decode_flashattention_b200 as fa
+
+    case = reuse if reuse is not None else Case(w, device, rank, args.num_splits)
+    for i in range(3):
+        case.step(i)
+    torch.cuda.synchronize()
+    fa.check_status()
+    dispatch = fa.last_dispatch()
+    stream = torch.cuda.current_stream(device)
+    calls = max(100, args.config_calls)
+    graphs, _ = case.graphs(calls)
+    reps = []
+    for _ in range(max(3, args.config_reps)):
+        barrier(world, device)
+        reps.append(max_over_ranks(replay_ms(graphs, stream), world, device) / calls * 1e3)
+    fa.check_status()
+    del graphs
+    med = pct(reps, 0.5)
+    peak, peak_kind = peaks()
+    tbs = case.bytes_per_step / (med / 1e6) / 1e12
+    ent = {
+        "workload": w.name, "description": w.description,
+        "us_per_call": round(med, 3), "us_p10": round(pct(reps, 0.1), 3), "us_p90": round(pct(reps, 0.9), 3),
+        "calls_per_rep": calls, "reps": len(reps),
+        "value": round(tbs * world, 4), "unit": "TB/s", "frac": round(tbs * 1e3 / peak, 4), "peak": peak,
+        "peak_kind": peak_kind, "kv_bytes_per_call": case.bytes_per_step,
+        "query_tokens_per_s": round(w.B * w.Lq * world / (med / 1e6), 1),
+        "traffic": recorded_traffic(w.name),
+        "dispatch": {k: dispatch[k] for k in ("variant", "grid", "rows_per_cta", "units", "combine_launched")},
+    }
+    if dispatch.get("variant") == fa.VARIANT_TCGEN05 or w.name == "gqa_prefill_fp16":
+        ent["note"] = "latency-bound (64 KB of K/V): parity and µs/call only" if w.name == "gqa_prefill_fp16" else None
+    ent["e2e"] = e2e_measure(case, max(1, args.config_e2e_steps), world, device)
+    ent["cpu_baseline"] = (cpu_baseline(w, case.ins0, case.sl0, args.config_cpu_seconds)
+                           if world == 1 else None)
+    if reuse is None:
+        del case
+        torch.cuda.empty_cache()
+    return ent
+
+
 def run_ours(args):
     import torch
 
@@ -298,50 +561,14 @@ def run_ours(args):
     fa.force_variant({"auto": fa.VARIANT_AUTO, "mma": fa.VARIANT_MMA, "scalar": fa.VARIANT_SCALAR}[args.variant])
     name = args.workload or wl.DEFAULT_BENCH
     w = workload_of(args)
-    def draw(seed):
-        # (inputs of one call, cache lengths): dense q, k, v or paged q, k_pages, v_pages, block_table
-        if w.call == "paged":
-            q, kp, vp, bt, sl = wl.make_paged_inputs(w, device, seed=seed)
-            return (q, kp, vp, bt), sl
-        q, k, v, sl = wl.make_inputs(w, device, seed=seed)
-        return (q, k, v), sl
-
-    ins0, sl0 = draw(w.seed + 1000 * rank)
-    q0 = ins0[0]
-    per_copy = sum(t.numel() * t.element_size() for t in ins0)
-    n_copies = max(1, math.ceil(4 * L2_BYTES / max(per_copy, 1)))
-    copies = [ins0] + [draw(w.seed + 1000 * rank + c)[0] for c in range(1, n_copies)]
-    sl_dev = sl0.to(device) if sl0 is not None else None
-    outs = [wl.empty_output(w, q0) for _ in range(n_copies)]
-    lses = [torch.empty((w.B, w.Hq, w.Lq), dtype=torch.float32, device=device) for _ in range(n_copies)]
-    if w.call == "paged":
-        ws_bytes = fa.paged_workspace_size(q0, ins0[1], ins0[2], ins0[3].shape[1], args.num_splits)
-    elif w.call == "kvcache":
-        ws_bytes = fa.kvcache_workspace_size(*ins0, args.num_splits)
-    else:
-        ws_bytes = fa.fwd_workspace_size(*ins0, w.causal, args.num_splits)
-    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
-    bytes_per_step = wl.kv_bytes(w, sl0)
-
-    def call(ins, sl, o, l):
-        if w.call == "paged":
-            return fa.fa_decode_kvcache_paged(*ins, sl, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
-                                              workspace=ws)
-        if w.call == "kvcache":
-            return fa.fa_decode_kvcache(*ins, sl, causal=w.causal, num_splits=args.num_splits, out=o, lse=l,
-                                        workspace=ws)
-        return fa.fa_fwd(*ins, causal=w.causal, num_splits=args.num_splits, out=o, lse=l, workspace=ws)
-
-    def step(i):
-        call(copies[i % n_copies], sl_dev, outs[i % n_copies], lses[i % n_copies])
-
+    case = Case(w, device, rank, args.num_splits)
     stream = torch.cuda.current_stream(device)
-    for i in range(max(args.warmup, 3)):
-        step(i)
+    W = max(args.warmup, 3)
+    for i in range(W):
+        case.step(i)
     torch.cuda.synchronize()
     fa.check_status()
     dispatch = fa.last_dispatch()
-    launches_per_step = 1 + dispatch["combine_launched"] if dispatch["grid"] > 0 else dispatch["combine_launched"]
 
     # steps: about 2 s of work unless given
     if args.steps > 0:
@@ -350,132 +577,95 @@ def run_ours(args):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(20):
-            step(i)
+            case.step(i)
         e1.record(stream)
         torch.cuda.synchronize()
         per = e0.elapsed_time(e1) / 20 / 1e3
-        K = int(min(200000, max(50, 2.0 / max(per, 1e-7))))
-        K = max_over_ranks(K, world, device) if world > 1 else K
-        K = int(K)
+        K = int(max_over_ranks(int(min(200000, max(50, 2.0 / max(per, 1e-7)))), world, device))
 
-    # --- pass A: value (graph replays of the public call) -----------------------------
-    graphs = []
+    # --- the timed region: exactly K calls, replayed from CUDA graphs of the
+    # public call, device time by CUDA events on the launching stream --------------
     use_graph = not args.no_graph
-    G = min(K, 2000)
     if use_graph:
-        n0 = fa.launch_count()
-        g_full = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_full):
-            for i in range(G):
-                step(i)
-        captured = fa.launch_count() - n0
-        rem = K % G
-        g_rem = None
-        if rem:
-            g_rem = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_rem):
-                for i in range(rem):
-                    step(i)
-        reps = K // G
-        launches = captured * reps + (launches_per_step * rem if rem else 0)
-        g_full.replay()  # warm the graph itself
-        torch.cuda.synchronize()
-    else:
-        launches = launches_per_step * K
-    barrier(world, device)
-    torch.cuda.synchronize()
+        graphs, launches = case.graphs(K)
     sampler = ClockSampler(device.index)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with sampler:
-        e0.record(stream)
+        barrier(world, device)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if use_graph:
-            for _ in range(K // G):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
+            lead_sleep()
+            e0.record(stream)
+            for g in graphs:
+                g.replay()
         else:
+            n0 = fa.launch_count()
+            e0.record(stream)
             for i in range(K):
-                step(i)
+                case.step(i)
+            launches = fa.launch_count() - n0
         e1.record(stream)
         torch.cuda.synchronize()
-    barrier(world, device)
-    ms_local = e0.elapsed_time(e1)
-    ms = max_over_ranks(ms_local, world, device)
+        barrier(world, device)
+        ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+        # the same K calls replayed again: the spread of µs/call over replays
+        reps = []
+        if use_graph:
+            for _ in range(max(3, args.reps)):
+                barrier(world, device)
+                reps.append(max_over_ranks(replay_ms(graphs, stream), world, device) / K * 1e3)
     fa.check_status()
+    if use_graph:
+        del graphs
 
-    # --- pass B: each kernel's own duration.  The library brackets its launches
-    # with CUDA events on the call's stream (and launches them without
-    # programmatic overlap, so each event pair times one kernel alone).  A
-    # spin kernel ahead of the calls lets the host queue them all before the
-    # first runs, so no host launch gap falls between an event and its kernel.
-    Kb = int(min(K, 200))
-    fa.profile_enable(True)
-    torch.cuda._sleep(int(40e6))  # about 20 ms of device time
-    for i in range(Kb):
-        step(i)
-    torch.cuda.synchronize()
-    prof = fa.profile_read()
-    fa.profile_enable(False)
-    fa.check_status()
-
-    # --- e2e: through the public API from pinned host buffers -------------------------
-    # host buffers with the device tensors' own layout ([H, L, D] storage stays
-    # [H, L, D]), so each copy is one plain memcpy of the storage
-    def pinned_like(t):
-        h = torch.empty_strided(t.size(), t.stride(), dtype=t.dtype, pin_memory=True)
-        h.copy_(t)
-        return h
-
-    hins = [pinned_like(t) for t in ins0]
-    hsl = sl0.pin_memory() if sl0 is not None else None
-    ho = torch.empty_strided(outs[0].size(), outs[0].stride(), dtype=w.dtype, pin_memory=True)
-    hl = torch.empty_strided(lses[0].size(), lses[0].stride(), dtype=torch.float32, pin_memory=True)
-    dins = [torch.empty_like(t) for t in ins0]
-    dsl = torch.empty_like(sl_dev) if sl_dev is not None else None
-    h2d = sum(t.numel() * t.element_size() for t in hins) + (hsl.numel() * 4 if hsl is not None else 0)
-    d2h = ho.numel() * 2 + hl.numel() * 4
-    E = max(1, args.e2e_steps)
-
-    def e2e_step():
-        for d, h in zip(dins, hins):
-            d.copy_(h, non_blocking=True)
-        if dsl is not None:
-            dsl.copy_(hsl, non_blocking=True)
-        o, l = call(dins, dsl, outs[0], lses[0])
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(l, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
+    # --- eager calls: the host side of each call (validation, plan, two tensor-map
+    # encodes, launches) is on the clock -------------------------------------------
+    Ke = min(K, 2000)
     barrier(world, device)
+    torch.cuda.synchronize()
     x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
     x0.record(stream)
-    for _ in range(E):
-        e2e_step()
+    for i in range(Ke):
+        case.step(i)
     x1.record(stream)
+    host_s = time.perf_counter() - t0
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(x0.elapsed_time(x1), world, device)
+    eager_ms = max_over_ranks(x0.elapsed_time(x1), world, device)
     fa.check_status()
 
-    total_bytes = sum_over_ranks(bytes_per_step * K, world, device)
+    prof = isolated_kernels(case, int(min(K, 200)))
+    e2e = e2e_measure(case, max(1, args.e2e_steps), world, device)
+
+    total_bytes = sum_over_ranks(case.bytes_per_step * K, world, device)
     value = total_bytes / (ms / 1e3) / 1e12
-    e2e_value = sum_over_ranks(bytes_per_step * E, world, device) / (e2e_ms / 1e3) / 1e12
     peak, peak_kind = peaks()
     tc = dispatch.get("variant") == fa.VARIANT_TCGEN05
+    us_call = ms / K * 1e3
+    traffic = recorded_traffic(name) if not args.batch else None
+    clocks = sampler.summary()
     # Roofline of the call.  Both kernels run back to back with programmatic
     # overlap, so no event pair can time one of them inside the timed region
     # without breaking that overlap; the achieved figure therefore charges the
     # split-KV kernel with the whole time per call (its combine and both kernel
-    # boundaries included) -- a lower bound on its own bandwidth.  Pass B's
-    # isolated per-kernel event times give the kernels' shares, reported beside
-    # it (the ncu launch list of the same command gives the same shares).
-    main_iso = prof["main_ms"] / max(prof["main_launches"], 1)
-    comb_iso = prof["combine_ms"] / max(prof["main_launches"], 1)  # per step (0 when no combine ran)
-    share_main = main_iso / (main_iso + comb_iso) if main_iso + comb_iso > 0 else 1.0
-    main_ms = ms / K
-    achieved = bytes_per_step / (main_ms / 1e3) / 1e9 if main_ms > 0 else None
-    traffic = recorded_traffic(name) if not args.batch else None
-    clocks = sampler.summary()
+    # boundaries included) -- a lower bound on its own bandwidth.  The isolated
+    # per-kernel event times give the kernels' shares, reported beside it (the
+    # ncu launch list of the same command gives the same shares).
+    roof = (tensor_roofline(w, case.sl0, ms / K, prof, traffic) if tc
+            else hbm_roofline(case, us_call, prof, peak, peak_kind, traffic))
+    cpu = cpu_baseline(w, case.ins0, case.sl0, args.cpu_seconds) if world == 1 else None
+
+    # --- every configuration of the metric, each timed the same way -------------------
+    per_config = {}
+    if args.per_config != "none":
+        names = wl.CONFIGS if args.per_config == "all" else args.per_config.split(",")
+        for cname in names:
+            wc = wl.WORKLOADS[cname]
+            key = next((k for k, v in wl.CONFIG_IDS.items() if v == cname), cname)
+            if cname == name and not args.batch:
+                per_config[key] = config_entry(wc, world, rank, device, args, reuse=case)
+            else:
+                per_config[key] = config_entry(wc, world, rank, device, args)
     if rank != 0:
         return
     res = {
@@ -484,9 +674,17 @@ def run_ours(args):
         "unit": "TB/s",
         "n_gpus": world,
         "steps": K,
-        "warmup": max(args.warmup, 3),
+        "warmup": W,
         "ms_per_step": ms / K,
-        "us_per_call": ms / K * 1e3,
+        "us_per_call": us_call,
+        "us_per_call_replays": {"median": round(pct(reps, 0.5), 3) if reps else None,
+                                "p10": round(pct(reps, 0.1), 3) if reps else None,
+                                "p90": round(pct(reps, 0.9), 3) if reps else None,
+                                "replays": len(reps), "calls_per_replay": K},
+        "eager": {"us_per_call": round(eager_ms / Ke * 1e3, 3), "calls": Ke,
+                  "host_us_per_call": round(host_s / Ke * 1e6, 3),
+                  "what": "calls issued one by one from Python through the C ABI (host validation, plan, "
+                          "two tensor-map encodes and the launches of each call on the clock)"},
         "pct_of_peak_per_gpu": round(100 * value / world * 1e3 / peak, 2),
         "query_tokens_per_s": round(wl.tokens_per_call(w) * K * world / (ms / 1e3), 1),
         "higher_is_better": True,
@@ -499,35 +697,21 @@ def run_ours(args):
             "batch_override": args.batch or None,
             "B": w.B, "Lq": w.Lq, "Hq": w.Hq, "Hkv": w.Hkv, "Lk": w.Lk, "Dqk": w.Dqk, "Dv": w.Dv,
             "causal": w.causal, "num_splits": args.num_splits or "auto", "variant": args.variant,
-            "kv_bytes_per_step": bytes_per_step,
-            "l2": f"inputs rotate over {n_copies} copies ({n_copies * per_copy / 1e6:.0f} MB > 4x L2)",
+            "kv_bytes_per_step": case.bytes_per_step,
+            "l2": f"inputs rotate over {case.n_copies} copies ({case.n_copies * case.per_copy / 1e6:.0f} MB > 4x L2)",
             "launch": "cuda_graph_replay" if use_graph else "eager",
+            "timing": "device time by CUDA events on the launching stream; a short spin kernel queued ahead of "
+                      "each timed region so the host's submission is off the clock",
             "parallelism": f"replicas{world}" if world > 1 else "single_gpu",
             "dispatch": dispatch,
         },
-        "roofline": tensor_roofline(w, sl0, ms / K, prof, traffic) if tc else {
-            "bound": "hbm",
-            "kernel": "split-KV kernel, charged with the whole call (combine and boundaries included)",
-            "achieved": round(achieved, 1) if achieved else None,
-            "peak": peak,
-            "peak_kind": peak_kind,
-            "unit": "GB/s",
-            "frac": round(achieved / peak, 4) if achieved else None,
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": bytes_per_step,
-            "kernel_us": round(main_ms * 1e3, 3),
-            "duration_method": "CUDA events around the timed region / steps (whole call)",
-            "share": round(share_main, 4),
-            "isolated_us": {"splitkv": round(main_iso * 1e3, 3),
-                            "combine": round(prof["combine_ms"] / max(prof["combine_launches"], 1) * 1e3, 3)},
-            "isolated_launches": prof["main_launches"],
-        },
-        "e2e": {"value": round(e2e_value, 5), "unit": "TB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E},
+        "roofline": roof,
+        "e2e": e2e,
         "gpu_launches": int(launches),
         "clocks": clocks,
+        "cpu_baseline": cpu,
+        "per_config": per_config,
     }
-    res["cpu_baseline"] = cpu_baseline(w, ins0, sl0, args.cpu_seconds) if world == 1 else None
     print(json.dumps(res), flush=True)
 
 

@@ -100,7 +100,7 @@ def load_library():
         "fa_profile_enable": (i32, [i32]),
         "fa_profile_read": (i32, [P(ctypes.c_double), P(ctypes.c_int64), P(ctypes.c_double),
                                   P(ctypes.c_int64)]),
-        "fa_schedule": (i32, [i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, P(ctypes.c_int64),
+        "fa_schedule": (i32, [i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, P(ctypes.c_int64),
                               P(ctypes.c_int64), vp, vp, vp, ctypes.c_int64]),
         "fa_launch_count": (ctypes.c_int64, []),
         "fa_version": (ctypes.c_char_p, []),
@@ -430,13 +430,14 @@ def profile_read() -> dict:
             "combine_launches": cn.value}
 
 
-def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2, tile_keys=128):
+def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2, tile_keys=128,
+             rows_per_cta=8):
     """Host copy of the kernels' work partition (see fa_schedule in include/fa.h).
     Returns dict(work_tiles, ctas_used, unit_tiles, unit_first_cta, unit_last_cta)."""
     import numpy as np
 
     g = Hq // Hkv
-    units = B * ((g * Lq + 7) // 8) * Hkv
+    units = B * ((g * Lq + rows_per_cta - 1) // rows_per_cta) * Hkv
     tiles = np.zeros(units, dtype=np.int32)
     first = np.zeros(units, dtype=np.int64)
     last = np.zeros(units, dtype=np.int64)
@@ -445,7 +446,7 @@ def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2
     _check(load_library().fa_schedule(
         int(B), int(Lq), int(Hq), int(Hkv), int(Lk), int(bool(causal)),
         ctypes.c_void_p(sl.ctypes.data if sl is not None else None), int(num_ctas), int(min_share),
-        int(tile_keys), ctypes.byref(W), ctypes.byref(P), ctypes.c_void_p(tiles.ctypes.data),
+        int(tile_keys), int(rows_per_cta), ctypes.byref(W), ctypes.byref(P), ctypes.c_void_p(tiles.ctypes.data),
         ctypes.c_void_p(first.ctypes.data), ctypes.c_void_p(last.ctypes.data), units))
     return {"work_tiles": W.value, "ctas_used": P.value, "unit_tiles": tiles,
             "unit_first_cta": first, "unit_last_cta": last}

@@ -159,6 +159,7 @@ fa_status check_tensor(const fa_tensor *t, const char *name) {
 struct Shapes {
     int dtype;
     int B, Lq, Hq, Lk, Hkv, Dqk, Dv, g, R, RB, BR;
+    int rpc;        // packed rows per row block: RB = ceil(R / rpc) row blocks per (batch, kv head)
     int KDqk, KDv;  // head dims of the kernel instance that runs the call (>= Dqk, Dv)
 };
 
@@ -179,6 +180,18 @@ fa_status kernel_dims(Shapes *s) {
     } else {
         s->KDqk = s->KDv = std::max(pad(s->Dqk), pad(s->Dv));
     }
+    return FA_OK;
+}
+
+// Row blocks of rpc packed rows: RB per (batch, kv head), BR = B * RB entries.
+fa_status set_row_blocks(Shapes *s, int rpc) {
+    s->rpc = rpc;
+    s->RB = (s->R + rpc - 1) / rpc;
+    const int64_t BR = (int64_t)s->B * s->RB;
+    if (BR > fa::kMaxPrefixEntries)
+        return fail(FA_ERR_UNSUPPORTED, "B * ceil(g * Lq / %d) = %lld exceeds %d", rpc, (long long)BR,
+                    fa::kMaxPrefixEntries);
+    s->BR = (int)BR;
     return FA_OK;
 }
 
@@ -250,12 +263,7 @@ fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
     int64_t R = (int64_t)s->g * s->Lq;
     if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * Lq too large");
     s->R = (int)R;
-    s->RB = (s->R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
-    int64_t BR = (int64_t)s->B * s->RB;
-    if (BR > fa::kMaxPrefixEntries)
-        return fail(FA_ERR_UNSUPPORTED, "B * ceil(g * Lq / 8) = %lld exceeds %d", (long long)BR, fa::kMaxPrefixEntries);
-    s->BR = (int)BR;
-    return FA_OK;
+    return set_row_blocks(s, fa::kRowsPerCta);
 }
 
 // ------------------------------------------------------------ planning
@@ -296,7 +304,7 @@ void host_schedule(const Shapes &s, int causal, int tile_shift, int P, int min_s
     std::vector<int> pre(s.BR + 1, 0);
     bool empty_unit = false;
     for (int x = 0; x < s.BR; ++x) {
-        int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, tile_shift);
+        int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, tile_shift, s.rpc);
         if (t == 0) empty_unit = true;
         pre[x + 1] = pre[x] + s.Hkv * t;
     }
@@ -324,7 +332,9 @@ int log2_exact(int v) {
     return k;
 }
 
-fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl) {
+// Plans the call; may change the row blocking of `s` (the tcgen05 split-KV
+// kernel takes row blocks of 16 to 64 packed rows).
+fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl) {
     DeviceState *dev = nullptr;
     fa_status st = device_state(&dev);
     if (st) return st;
@@ -416,8 +426,8 @@ fa_status make_plan(const Shapes &s, int causal, int num_splits, bool kvcache, i
     }
     pl->need_workspace = pl->need_combine;
     pl->pieces = (size_t)pl->P_param;  // one piece per CTA
-    const size_t o_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta * s.KDv : 0;
-    const size_t lse_floats = pl->need_workspace ? pl->pieces * 2 * fa::kRowsPerCta : 0;
+    const size_t o_floats = pl->need_workspace ? pl->pieces * 2 * s.rpc * s.KDv : 0;
+    const size_t lse_floats = pl->need_workspace ? pl->pieces * 2 * s.rpc : 0;
     pl->ws_o_off = 0;
     pl->ws_lse_off = pl->ws_o_off + ((o_floats * 4 + 255) & ~size_t(255));
     pl->ws_bytes = pl->need_workspace ? pl->ws_lse_off + ((lse_floats * 4 + 255) & ~size_t(255)) : 0;
@@ -501,7 +511,7 @@ fa_status prof_record(cudaEvent_t *ev, cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------ the call
-fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
+fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, fa_tensor *o,
               const int32_t *seqlens, float *lse, int causal, float scale, int num_splits, void *workspace,
               size_t workspace_bytes, cudaStream_t stream, const Paging *pg = nullptr,
               const fa::AppendParams *ap = nullptr, const Varlen *vl = nullptr) {
@@ -547,6 +557,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     p.g = s.g;
     p.R = s.R;
     p.RB = s.RB;
+    p.rpc = s.rpc;
     p.Lk = s.Lk;
     p.dqk = s.Dqk;
     p.dv = s.Dv;
@@ -706,7 +717,7 @@ fa_status run(const Shapes &s, const fa_tensor *q, const fa_tensor *k, const fa_
     d.smem_bytes = pl.main.smem;
     d.tile_keys = pl.main.tile_keys;
     d.stages = pl.main.stages;
-    d.rows_per_cta = pl.prefill ? pl.main.rows : fa::kRowsPerCta;
+    d.rows_per_cta = pl.prefill ? pl.main.rows : s.rpc;
     d.units = (int)((int64_t)s.B * s.RB * s.Hkv);
     d.min_share_tiles = pl.min_share;
     d.combine_launched = pl.need_combine ? 1 : 0;
@@ -900,13 +911,7 @@ fa_status check_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
     const int64_t R = (int64_t)s->g * s->Lq;
     if (R > INT32_MAX / 2) return fail(FA_ERR_UNSUPPORTED, "g * max_seqlen_q too large");
     s->R = (int)R;
-    s->RB = (s->R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
-    const int64_t BR = (int64_t)s->B * s->RB;
-    if (BR > fa::kMaxPrefixEntries)
-        return fail(FA_ERR_UNSUPPORTED, "batch * ceil(g * max_seqlen_q / 8) = %lld exceeds %d", (long long)BR,
-                    fa::kMaxPrefixEntries);
-    s->BR = (int)BR;
-    return FA_OK;
+    return set_row_blocks(s, fa::kRowsPerCta);
 }
 
 fa_status fa_fwd_varlen(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v, const int32_t *cu_seqlens_q,
@@ -1027,12 +1032,13 @@ fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double *combi
 }
 
 fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens, int num_ctas,
-                      int min_share, int tile_keys, int64_t *work_tiles, int64_t *ctas_used, int32_t *unit_tiles,
-                      int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units) {
+                      int min_share, int tile_keys, int rows_per_cta, int64_t *work_tiles, int64_t *ctas_used,
+                      int32_t *unit_tiles, int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units) {
     if (B < 0 || Lq < 0 || Hq <= 0 || Hkv <= 0 || Lk < 0 || Hq % Hkv || num_ctas < 1 || min_share < 1 ||
-        tile_keys < 1 || (tile_keys & (tile_keys - 1)) || max_units < 0)
+        tile_keys < 1 || (tile_keys & (tile_keys - 1)) || max_units < 0 || rows_per_cta < 1 ||
+        rows_per_cta > fa::kMaxRowsPerCta)
         return fail(FA_ERR_INVALID_ARG, "fa_schedule: inconsistent sizes");
-    const int g = Hq / Hkv, R = g * Lq, RB = (R + fa::kRowsPerCta - 1) / fa::kRowsPerCta;
+    const int g = Hq / Hkv, R = g * Lq, RB = (R + rows_per_cta - 1) / rows_per_cta;
     const int shift = log2_exact(tile_keys);
     const int64_t BR = (int64_t)B * RB;
     if (BR * Hkv * (((int64_t)Lk + tile_keys - 1) / tile_keys) >= (int64_t(1) << 31) - 1)
@@ -1041,7 +1047,7 @@ fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const 
     std::vector<int32_t> tx(BR, 0);
     for (int64_t x = 0; x < BR; ++x) {
         int n = fa::batch_keys(seqlens, (int)(x / RB), Lk);
-        tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, shift);
+        tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, shift, rows_per_cta);
         pre[x + 1] = pre[x] + Hkv * tx[x];
     }
     const int W = pre[BR];

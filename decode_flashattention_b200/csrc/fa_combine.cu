@@ -69,9 +69,9 @@ __global__ void __launch_bounds__(kCombineThreads)
             b = (int)(row / ((long long)p.Lq * p.Hq));
             r = (hq % p.g) * p.Lq + i;
         }
-        rr = r % kRowsPerCta;
+        rr = r % p.rpc;
         hkv = hq / p.g;
-        x = b * p.RB + r / kRowsPerCta;
+        x = b * p.RB + r / p.rpc;
     };
     if (!p.cu_q) locate();
 
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kCombineThreads)
             nparts = piece_of(pt, u0 + t - 1) - cf + 1;
             const int c = cf + lane;
             if (lane < PPP && lane < nparts)
-                base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr;
+                base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * p.rpc + rr;
         }
     };
     if (uniform_batches(p) && live) plan();
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kCombineThreads)
                 const bool has = lane < PPP && j0 + lane < np;
                 const long long base =
                     j0 == 0 ? b0
-                            : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * kRowsPerCta + rr : 0);
+                            : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * p.rpc + rr : 0);
                 const int cnt = np - j0 < PPP ? np - j0 : PPP;
                 const float ls = has ? ws_lse[base] : -INFINITY;
                 float v[PPP][EPL];

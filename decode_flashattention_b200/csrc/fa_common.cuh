@@ -12,9 +12,12 @@
 namespace fa {
 
 // Query rows packed into one CTA: the g*Lq rows of a GQA group that share a
-// kv head are laid out as r = h_local * Lq + i and cut into blocks of 8
-// (the N extent of one m16n8k16 MMA when keys are the M operand).
+// kv head are laid out as r = h_local * Lq + i and cut into row blocks of
+// Params::rpc rows.  The mma.sync kernel takes blocks of 8 (the N extent of
+// one m16n8k16 MMA when keys are the M operand); the tcgen05 split-KV kernel
+// takes 16, 32 or 64 (the N extent of its products).
 constexpr int kRowsPerCta = 8;
+constexpr int kMaxRowsPerCta = 64;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
 constexpr int kMaxPrefixEntries = 8192;              // B * row-blocks bound
@@ -32,6 +35,7 @@ struct Params {
     const int *seqlens;    // [B] or null (then every batch has Lk keys)
     unsigned *status;      // device status word (timeouts)
     int B, Lq, Hq, Hkv, g, R, RB, Lk;
+    int rpc;               // packed rows per row block (unit), RB = ceil(R / rpc)
     int dqk, dv;           // the call's head dims (the kernel's DQK / DV may be larger: columns past them are zero)
     unsigned long long wait_limit_ns;  // bound of every wait on a pipeline barrier
     int stall;             // test hook: the first CTA leaves its first stage empty
@@ -74,13 +78,13 @@ struct Params {
 // (normalised O and log2-sum-exp) per CTA touching it, in slot 0 if it is the
 // CTA's first segment and slot 1 otherwise, and the combine kernel merges them.
 
-__host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int Lq, int causal) {
-    if (n <= 0 || rb * kRowsPerCta >= R) return 0;  // no keys, or a row block past the batch's rows
+__host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int Lq, int causal, int rpc) {
+    if (n <= 0 || rb * rpc >= R) return 0;  // no keys, or a row block past the batch's rows
     if (!causal) return n;
     // rows r0 .. r0 + cnt - 1 hold query positions i = r % Lq; the largest one
     // is r0 % Lq + cnt - 1 unless the run wraps past Lq - 1.
-    const int r0 = rb * kRowsPerCta;
-    const int cnt = R - r0 < kRowsPerCta ? R - r0 : kRowsPerCta;
+    const int r0 = rb * rpc;
+    const int cnt = R - r0 < rpc ? R - r0 : rpc;
     const int a = r0 % Lq;
     const int maxi = (a + cnt - 1 >= Lq) ? Lq - 1 : a + cnt - 1;
     int k = maxi + n - Lq + 1;  // bottom-right: row i sees keys j <= i + n - Lq
@@ -127,8 +131,8 @@ __device__ __forceinline__ BatchGeom batch_geom(const Params &p, int b) {
 #endif
 
 // Tiles of tile_keys = 1 << tile_shift keys covering the visible keys.
-__host__ __device__ inline int unit_tiles(int n, int rb, int R, int Lq, int causal, int tile_shift) {
-    const int k = keys_visible_to_block(n, rb, R, Lq, causal);
+__host__ __device__ inline int unit_tiles(int n, int rb, int R, int Lq, int causal, int tile_shift, int rpc) {
+    const int k = keys_visible_to_block(n, rb, R, Lq, causal, rpc);
     return (k + (1 << tile_shift) - 1) >> tile_shift;
 }
 
@@ -424,7 +428,7 @@ __device__ __forceinline__ void store_row8<__nv_bfloat16>(__nv_bfloat16 *dst, co
 __device__ __forceinline__ int entry_tiles(const Params &p, int x) {
     const int b = x / p.RB, rb = x - b * p.RB;
     const BatchGeom G = batch_geom(p, b);
-    return unit_tiles(G.n, rb, G.R, G.Lq, p.causal, p.tile_shift);
+    return unit_tiles(G.n, rb, G.R, G.Lq, p.causal, p.tile_shift, p.rpc);
 }
 
 __device__ __forceinline__ int warp_sum(int v) {

@@ -55,6 +55,12 @@
  *
  * Thread safety: the compute calls may be issued from several host threads;
  * fa_last_error() and fa_last_dispatch() report the calling thread's last call.
+ *
+ * Device state: the library keeps, per device, the address of its status
+ * word (fa_check_status) and of the allocation-free call's scratch array,
+ * looked up on first use and cached for the life of the process.  A
+ * cudaDeviceReset (or any other end of the device's primary context) makes
+ * them stale: do not call the library on that device afterwards.
  */
 #ifndef FA_B200_H
 #define FA_B200_H
@@ -124,7 +130,15 @@ FA_API fa_status fa_fwd(const fa_tensor *q, const fa_tensor *k, const fa_tensor 
                  float *lse, int causal, float scale, int num_splits, void *workspace,
                  size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace fa_fwd needs for these shapes on the current device. */
+/*
+ * fa_fwd_workspace_size -- bytes of workspace fa_fwd needs for these shapes
+ * on the current device (0 when no key range is split between CTAs).  The
+ * first half of the two-phase call of "SmallQ FlashAttention for Ascend
+ * 910B", section "aclnn API 调用": a GetWorkspaceSize call sizes the scratch,
+ * the caller allocates it, then the compute call runs on the caller's
+ * stream.  Host only (no launch, no allocation); the arguments are those of
+ * the matching compute call (o and data pointers are not read).
+ */
 FA_API fa_status fa_fwd_workspace_size(const fa_tensor *q, const fa_tensor *k, const fa_tensor *v,
                                 int causal, int num_splits, size_t *bytes);
 
@@ -141,7 +155,13 @@ FA_API fa_status fa_decode_kvcache(const fa_tensor *q, const fa_tensor *k_cache,
                             int causal, float scale, void *workspace, size_t workspace_bytes,
                             void *stream);
 
-/* Bytes of workspace fa_decode_kvcache needs for these shapes on the current device. */
+/*
+ * fa_decode_kvcache_workspace_size -- bytes of workspace fa_decode_kvcache
+ * needs for these shapes on the current device: the GetWorkspaceSize phase
+ * of the aclnn two-phase call ("SmallQ FlashAttention for Ascend 910B",
+ * section "aclnn API 调用"), as for fa_fwd_workspace_size.  The size does not
+ * depend on the cache lengths (they live on the device).
+ */
 FA_API fa_status fa_decode_kvcache_workspace_size(const fa_tensor *q, const fa_tensor *k_cache,
                                            const fa_tensor *v_cache, int num_splits,
                                            size_t *bytes);
@@ -253,7 +273,11 @@ FA_API fa_status fa_fwd_varlen_workspace_size(const fa_tensor *q, const fa_tenso
  * before any stream capture.  All calls on a device share the array and it
  * keeps the last call's contents (nothing in it needs to start at zero), so
  * calls whose GPU work overlaps -- on different streams or from racing host
- * threads -- race on it and must be serialised by the caller.
+ * threads -- race on it and must be serialised by the caller.  The array's
+ * address is cached per device for the life of the process (as is the
+ * status word's, see fa_check_status): after cudaDeviceReset, or anything
+ * else that destroys the device's primary context, both are stale and this
+ * library must not be called again in that process.
  */
 FA_API fa_status fa_decode_kvcache_noalloc(const fa_tensor *q, const fa_tensor *k_cache,
                                            const fa_tensor *v_cache, const int32_t *cache_seqlens,
@@ -264,17 +288,29 @@ FA_API fa_status fa_decode_kvcache_noalloc(const fa_tensor *q, const fa_tensor *
 FA_API size_t fa_noalloc_scratch_bytes(void);
 
 /*
+ * fa_check_status -- this library's own addition; the pages have no
+ * counterpart (their calls report errors only through return codes).
  * Synchronises `stream`, then reports whether any kernel of this library on
  * the current device gave up waiting on its copy pipeline since the last
  * check (FA_ERR_TIMEOUT) and clears that record.  FA_ERR_CUDA if the stream
- * itself reports an error.
+ * itself reports an error.  The record is ONE word per device, shared by
+ * every stream and host thread: a check on one stream also reads (and
+ * clears) a timeout recorded by a kernel that another stream or thread
+ * launched, so a caller that must attribute a timeout to one stream has to
+ * serialise its checks with the other users of the device.
  */
 FA_API fa_status fa_check_status(void *stream);
 
 /* Message of the calling thread's last failed call ("" after success). */
 FA_API const char *fa_last_error(void);
 
-/* What the calling thread's last successful compute call launched. */
+/*
+ * fa_last_dispatch -- what the calling thread's last successful compute call
+ * launched (kernel variant, grid, split partition, whether the combine ran):
+ * the counterpart of get_last_dispatch_info() in the MXFlashAttn README
+ * (section "前向算子 API"), which reports the backend that served the last
+ * forward call.  Host only; the record is per host thread.
+ */
 FA_API void fa_last_dispatch(fa_dispatch_info *info);
 
 /*
@@ -357,18 +393,21 @@ FA_API fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double
  * fa_schedule -- host-side copy of the work partition the kernels compute on
  * the device (no device access; for inspection and tests).  Work is counted
  * in key tiles of `tile_keys` keys (a power of two); a unit is (batch, block
- * of 8 packed query rows, kv head), ordered batch-major, then row block, then
- * kv head, and owns ceil(visible keys / tile_keys) tiles.  The W tiles of all
- * units are laid end to end and cut into ctas_used = min(num_ctas,
- * ceil(W / min_share)) contiguous pieces, one per CTA, whose sizes differ by
- * at most one tile (the first W mod ctas_used pieces are the longer ones).
- * seqlens: HOST int32 [B] (NULL: every batch has Lk keys).  For each of the
- * first max_units units the call writes its tile count and the first and last
- * CTA whose piece holds its tiles (-1, -1 for a unit with no tiles).
- * FA_ERR_INVALID_ARG for inconsistent sizes.
+ * of `rows_per_cta` packed query rows, kv head) -- 8 for the mma.sync
+ * split-KV kernel, 16 / 32 / 64 for the tcgen05 one (fa_last_dispatch's
+ * rows_per_cta says which a call used) -- ordered batch-major, then row
+ * block, then kv head, and owns ceil(visible keys / tile_keys) tiles.  The W
+ * tiles of all units are laid end to end and cut into ctas_used =
+ * min(num_ctas, ceil(W / min_share)) contiguous pieces, one per CTA, whose
+ * sizes differ by at most one tile (the first W mod ctas_used pieces are the
+ * longer ones).  seqlens: HOST int32 [B] (NULL: every batch has Lk keys).
+ * For each of the first max_units units the call writes its tile count and
+ * the first and last CTA whose piece holds its tiles (-1, -1 for a unit with
+ * no tiles).  FA_ERR_INVALID_ARG for inconsistent sizes (rows_per_cta must
+ * be in [1, 64]).
  */
 FA_API fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens,
-                             int num_ctas, int min_share, int tile_keys, int64_t *work_tiles,
+                             int num_ctas, int min_share, int tile_keys, int rows_per_cta, int64_t *work_tiles,
                              int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta,
                              int64_t *unit_last_cta, int64_t max_units);
 

@@ -163,11 +163,11 @@ def test_empty_batch_is_a_no_op():
 
 # ------------------------------------------------------------------ work partition
 
-def visible_tiles(n, rb, R, Lq, causal, TK=128):
+def visible_tiles(n, rb, R, Lq, causal, TK=128, rpc=8):
     """Independent restatement of the tiles a row block needs (bottom-right)."""
     if n <= 0:
         return 0
-    rows = range(rb * 8, min(rb * 8 + 8, R))
+    rows = range(rb * rpc, min(rb * rpc + rpc, R))
     k = max(min(n, (r % Lq) + n - Lq + 1) if causal else n for r in rows)
     return max(0, math.ceil(max(k, 0) / TK))
 
@@ -186,20 +186,21 @@ CASES = [
 
 @pytest.mark.parametrize("c", CASES, ids=range(len(CASES)))
 @pytest.mark.parametrize("min_share", [1, 2, 5])
-def test_schedule_covers_balances_and_bounds_partials(c, min_share):
+@pytest.mark.parametrize("rpc", [8, 16, 64])
+def test_schedule_covers_balances_and_bounds_partials(c, min_share, rpc):
     c = dict(c)
     if c["seqlens"] == "rand":
         c["seqlens"] = np.random.default_rng(3).integers(1, c["Lk"] + 1, c["B"]).astype(np.int32)
     s = fa.schedule(c["B"], c["Lq"], c["Hq"], c["Hkv"], c["Lk"], c["causal"], c["seqlens"],
-                    num_ctas=c["num_ctas"], min_share=min_share, tile_keys=128)
+                    num_ctas=c["num_ctas"], min_share=min_share, tile_keys=128, rows_per_cta=rpc)
     g = c["Hq"] // c["Hkv"]
     R = g * c["Lq"]
-    RB = (R + 7) // 8
+    RB = (R + rpc - 1) // rpc
     want = []
     for b in range(c["B"]):
         n = c["Lk"] if c["seqlens"] is None else int(c["seqlens"][b])
         for rb in range(RB):
-            want += [visible_tiles(n, rb, R, c["Lq"], c["causal"])] * c["Hkv"]
+            want += [visible_tiles(n, rb, R, c["Lq"], c["causal"], rpc=rpc)] * c["Hkv"]
     tiles = s["unit_tiles"]
     assert tiles.tolist() == want
     W = int(tiles.sum())

@@ -5,9 +5,10 @@ synchronisation).  It takes its split-KV scratch from a fixed array compiled
 into the library instead of a caller workspace.
 
 The test calls it through the C ABI twice in a row, on different inputs, and
-checks each result against the regular fa_decode_kvcache (caller workspace)
-within the parity tolerances; a request needing more scratch than the array
-holds must be refused with a message.  This file is named to be collected
+checks each result against the fp64 oracle and against the regular
+fa_decode_kvcache (caller workspace), both within the parity tolerances; a
+request needing more scratch than the array holds must be refused with a
+message.  This file is named to be collected
 last, and it runs the same way alone in a fresh process.
 """
 import ctypes
@@ -19,7 +20,7 @@ import decode_flashattention_b200 as fa
 from decode_flashattention_b200 import FaTensor
 from decode_flashattention_b200 import workloads as wl
 
-from helpers import compare
+from helpers import compare, oracle_full
 
 pytestmark = pytest.mark.gpu
 
@@ -76,8 +77,10 @@ def test_noalloc_matches_regular_call_twice_in_a_row():
         ro, rl = fa.fa_decode_kvcache(q, k, v, sl, causal=w.causal)
         torch.cuda.synchronize()
         fa.check_status()
+        eo, el = oracle_full(q, k, v, w.causal, seqlens=sl)
+        compare(o.float().cpu().numpy(), lse.cpu().numpy(), eo, el, w.dtype, w.name + " vs oracle")
         compare(o.float().cpu().numpy(), lse.cpu().numpy(), ro.float().cpu().numpy(), rl.cpu().numpy(),
-                w.dtype, w.name)
+                w.dtype, w.name + " vs fa_decode_kvcache")
 
 
 def test_noalloc_refuses_scratch_beyond_its_array():
