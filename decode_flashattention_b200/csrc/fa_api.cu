@@ -376,8 +376,26 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
             return fail(FA_ERR_UNSUPPORTED, "grid too large for the tcgen05 variant");
         return FA_OK;
     }
-    bool ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.KDqk, s.KDv, &pl->main)
-                                           : fa::get_mma_kernel(s.dtype, s.KDqk, s.KDv, &pl->main);
+    // More than 8 packed rows (a GQA group with several query positions): the
+    // tcgen05 split-KV kernel takes them as one unit of up to 64 rows, so K / V
+    // are streamed once for the whole group instead of once per 8 rows.
+    const bool tcs_dims = s.KDv <= 128 && s.KDqk <= 192;
+    if (variant == FA_VARIANT_MMA && g_force_variant.load() == FA_VARIANT_AUTO && s.R > fa::kRowsPerCta && tcs_dims)
+        variant = FA_VARIANT_TCGEN05_SPLIT;
+    bool ok;
+    if (variant == FA_VARIANT_TCGEN05_SPLIT) {
+        const int nr = s.R <= 16 ? 16 : (s.R <= 32 ? 32 : 64);
+        const int tdqk = s.KDqk <= 128 ? 128 : 192;
+        ok = tcs_dims && fa::get_tc_split_kernel(s.dtype, tdqk, 128, nr, &pl->main);
+        if (ok) {
+            s.KDqk = tdqk;  // dims past the call's own read as zeros, as for the other instances
+            s.KDv = 128;
+            if ((st = set_row_blocks(&s, nr))) return st;
+        }
+    } else {
+        ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.KDqk, s.KDv, &pl->main)
+                                          : fa::get_mma_kernel(s.dtype, s.KDqk, s.KDv, &pl->main);
+    }
     if (variant == FA_VARIANT_SCALAR && ok && s.R != 1)
         return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
     if (!ok) return fail(FA_ERR_UNSUPPORTED, "no kernel for variant %d, dtype %d, head dims (%d, %d)", variant,
@@ -980,7 +998,7 @@ void fa_last_dispatch(fa_dispatch_info *info) {
 }
 
 fa_status fa_force_variant(int variant) {
-    if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_TCGEN05)
+    if (variant < FA_VARIANT_AUTO || variant > FA_VARIANT_TCGEN05_SPLIT)
         return fail(FA_ERR_INVALID_ARG, "unknown variant %d", variant);
     g_force_variant.store(variant);
     return FA_OK;

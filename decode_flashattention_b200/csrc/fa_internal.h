@@ -29,6 +29,10 @@ bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out);
 // Main split-KV kernel using fp32 FMA dot products (one packed row).
 bool get_scalar_kernel(int dtype, int dqk, int dv, KernelInfo *out);
 
+// Split-KV kernel on tcgen05 (fa_splitkv_tc.cu) for row blocks of nr = 16,
+// 32 or 64 packed rows; instances (dqk, dv) = (128, 128) and (192, 128).
+bool get_tc_split_kernel(int dtype, int dqk, int dv, int nr, KernelInfo *out);
+
 // KV append (fa_append.cu): new K / V rows [B, Lnew, Hkv, D] into a dense
 // cache [B, Lmax, Hkv, D] or a paged one [num_blocks, page, Hkv, D] at
 // positions cache_seqlens[b] + t.  Strides in elements ({batch or block, row,

@@ -90,6 +90,184 @@ struct SplitCfg {
 };
 
 
+// The producer warp's loop, shared by the split-KV kernels: walks the CTA's
+// piece of the key-tile space (the Partition) segment by segment and feeds the
+// STAGES-deep ring -- per tile the TMA loads of K and V (C::KBOX and C::VBOX
+// boxes of C::TK keys x 64 elements, 128-byte swizzle, L2 evict-first, no
+// multicast; a paged cache gathered page by page) and the stage header; at the
+// first tile of each segment q_write(s, seg, b, rb, hkv, G) (all 32 lanes)
+// stages the unit's query rows and returns false if a wait gave up.  full0 /
+// empty0: shared addresses of the stages' full / empty barriers (8 bytes
+// apart).  Ends with the end-of-work marker and a bounded wait for every copy
+// still in flight.  Must be called by all 32 lanes of the warp.
+// Tiles of a CTA's piece the producer asks L2 for before waiting on the
+// previous kernel (dense K / V).
+#ifndef FA_PREFETCH_TILES
+#define FA_PREFETCH_TILES 2
+#endif
+constexpr int kPrefetchTiles = FA_PREFETCH_TILES;
+
+template <class C, int STAGES, class QW>
+__device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CUtensorMap *tmV, const Params &p,
+                                                uint32_t smem_base, uint32_t full0, uint32_t empty0,
+                                                StageMeta *meta, volatile int *abort_flag, QW &&q_write) {
+    const int lane = threadIdx.x & 31;
+    auto full_bar = [&](int s) { return full0 + 8u * s; };
+    auto empty_bar = [&](int s) { return empty0 + 8u * s; };
+    // Dense inputs: the schedule needs only the kernel's parameters, so it
+    // is worked out before the wait and overlaps the previous kernel; cache
+    // or sequence lengths are read only after the wait.
+    Partition pt = {0, 1};
+    SegmentWalker wk;
+    bool active = false;
+    const int cta = blockIdx.x;
+    auto plan = [&]() {
+        pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
+        active = pt.W > 0 && cta < pt.P;
+        if (active) wk.init(p, piece_start(pt, cta), piece_end(pt, cta));
+    };
+    if (uniform_batches(p)) {
+        plan();
+        // While the previous kernel in the stream finishes, ask L2 for the
+        // first tiles of this CTA's piece (dense K / V only: the addresses
+        // need no memory reads).  A prefetch hands no data to this CTA --
+        // the loads below still run after the wait and read L2, where any
+        // write of the previous kernel lands -- so it cannot see stale data;
+        // it only moves the first HBM reads ahead, into the previous
+        // kernel's tail, where the memory system is mostly idle.
+        if (active && lane == 0 && !p.block_table) {
+            SegmentWalker pw = wk;
+            int n = 0;
+            for (; !pw.done() && n < kPrefetchTiles; pw.advance(p)) {
+                const BatchGeom G = batch_geom(p, pw.b(p));
+                const int kb = pw.b(p);
+                for (int tt = pw.pos - pw.u0; tt < pw.seg_end() - pw.u0 && n < kPrefetchTiles; ++tt, ++n) {
+#pragma unroll
+                    for (int c = 0; c < C::KBOX; ++c) tma_prefetch_4d(tmK, c * 64, G.k0 + tt * C::TK, pw.hkv, kb);
+#pragma unroll
+                    for (int c = 0; c < C::VBOX; ++c) tma_prefetch_4d(tmV, c * 64, G.k0 + tt * C::TK, pw.hkv, kb);
+                }
+            }
+        }
+        __syncwarp();
+    }
+    pdl_wait_primary();
+    // The combine kernel's CTAs may be scheduled now (they wait for this
+    // grid to complete before reading anything it writes).
+    pdl_launch_dependents();
+    if (!uniform_batches(p)) plan();
+
+    const uint64_t policy = l2_policy_evict_first();
+    int it = 0, seg = 0;
+    bool stop = !active;
+    const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
+    for (; active && !wk.done() && !stop; wk.advance(p), ++seg) {
+        const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
+        const BatchGeom G = batch_geom(p, b);
+        const int kb = p.cu_q ? 0 : b;  // K / V batch coordinate (packed inputs: one batch of tokens)
+        const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
+        const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
+        const int slot = (wk.pos == lo) ? 0 : 1;
+        for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
+            const int s = it % STAGES, use = it / STAGES;
+            // test hook: the first CTA leaves its first stage empty (no copy,
+            // no arrival), so its consumers' wait on it runs out
+            if (p.stall && cta == 0 && it == 0) continue;
+            const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+            if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's control flow uniform
+                stop = true;
+                break;
+            }
+            const uint32_t kdst = smem_base + s * C::STAGE_BYTES;
+            const uint32_t vdst = kdst + C::KBOX * C::BOX_BYTES;
+            // (one piece per CTA: the piece's last tile is the CTA's last tile)
+            const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
+                              (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
+            const int j = tt * C::TK;
+            if (!p.block_table) {
+                if (lane == 0) {
+                    mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::KBOX; ++c)
+                        tma_load_4d(kdst + c * C::BOX_BYTES, tmK, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
+#pragma unroll
+                    for (int c = 0; c < C::VBOX; ++c)
+                        tma_load_4d(vdst + c * C::BOX_BYTES, tmV, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
+                }
+            } else {
+                // Paged K/V: the tile is gathered page by page.  A page of at
+                // least TK keys gives one box of TK rows; a smaller page gives
+                // TK / page boxes of `page` rows, stacked in the stage exactly
+                // where one TK-row box would put them (a box of 8 or more rows
+                // starts on a 1024-byte swizzle period).  The lanes share the
+                // boxes; a page past the table or an invalid block number
+                // reads as zeros (out-of-range coordinates).
+                if (lane == 0) mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
+                __syncwarp();
+                const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
+                const int nsub = C::TK >> sub_shift;
+                for (int idx = lane; idx < (C::KBOX + C::VBOX) * nsub; idx += 32) {
+                    const int c = idx / nsub, sub = idx - c * nsub;
+                    const int key = j + (sub << sub_shift);
+                    const int page = key >> p.page_shift;
+                    int blk = p.num_blocks;
+                    if (page < p.max_pages) {
+                        const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
+                        if (e >= 0 && e < p.num_blocks) blk = e;
+                    }
+                    const int row = key & ((1 << p.page_shift) - 1);
+                    const uint32_t off = (uint32_t)(sub << sub_shift) * 128u;
+                    if (c < C::KBOX)
+                        tma_load_4d(kdst + c * C::BOX_BYTES + off, tmK, full_bar(s), c * 64, row, hkv, blk, policy);
+                    else
+                        tma_load_4d(vdst + (c - C::KBOX) * C::BOX_BYTES + off, tmV, full_bar(s), (c - C::KBOX) * 64,
+                                    row, hkv, blk, policy);
+                }
+            }
+            if (lane == 0) {
+                StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
+                meta[s] = m;
+            }
+            const bool qok = !(flags & kMetaFirst) || __all_sync(0xffffffffu, q_write(s, seg, b, rb, hkv, G));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full_bar(s));
+            if (!qok) {  // a wait gave up (the CTA is aborting): the stage still completes, then stop
+                stop = true;
+                ++it;
+                break;
+            }
+        }
+    }
+    // end-of-work marker in the next stage (its previous load was consumed:
+    // the empty barrier says so)
+    const int s_done = it % STAGES;
+    bool done_sent = false;
+    {
+        const int use = it / STAGES;
+        bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (lane == 0) {
+            StageMeta m = {0, 0, 0, 0, kMetaDone, 0, 0, 0};
+            meta[s_done] = m;
+        }
+        __syncwarp();
+        if (lane == 0 && ok) mbar_arrive(full_bar(s_done));
+        done_sent = ok;
+    }
+    // Never leave the CTA with copies in flight: wait (bounded, whatever
+    // the abort state) for the last load issued into each stage.  The
+    // marker's stage needs no wait once the marker went out.
+    if (lane == 0) {
+        for (int s = 0; s < STAGES && s < it; ++s) {
+            if (s == s_done && done_sent) continue;
+            const int last_use = (it - 1 - s) / STAGES;
+            volatile int no_abort = 0;
+            mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
+        }
+    }
+}
+
+
 template <typename T, int DQK, int DV, int STAGES, bool FMA, int KB = 2>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -130,146 +308,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kConsumerWarps) {
         // ============================================================ producer warp
-        // Dense inputs: the schedule needs only the kernel's parameters, so it
-        // is worked out before the wait and overlaps the previous kernel; cache
-        // or sequence lengths are read only after the wait.
-        Partition pt = {0, 1};
-        SegmentWalker wk;
-        bool active = false;
-        const int cta = blockIdx.x;
-        auto plan = [&]() {
-            pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
-            active = pt.W > 0 && cta < pt.P;
-            if (active) wk.init(p, piece_start(pt, cta), piece_end(pt, cta));
-        };
-        if (uniform_batches(p)) plan();
-        pdl_wait_primary();
-        // The combine kernel's CTAs may be scheduled now (they wait for this
-        // grid to complete before reading anything it writes).
-        pdl_launch_dependents();
-        if (!uniform_batches(p)) plan();
-
+        // At the first tile of a segment the unit's 8 packed query rows (rows
+        // past g*Lq are zero) go into the stage's Q slot, copied
+        // asynchronously and counted on the same stage barrier.
         const T *__restrict__ qg = reinterpret_cast<const T *>(p.q);
-        const uint64_t policy = l2_policy_evict_first();
-        int it = 0;
-        bool stop = !active;
-        const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
-        for (; active && !wk.done() && !stop; wk.advance(p)) {
-            const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
-            const BatchGeom G = batch_geom(p, b);
-            const int kb = p.cu_q ? 0 : b;  // K / V batch coordinate (packed inputs: one batch of tokens)
-            const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
-            const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
-            const int slot = (wk.pos == lo) ? 0 : 1;
-            for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
-                const int s = it % STAGES, use = it / STAGES;
-                // test hook: the first CTA leaves its first stage empty (no copy,
-                // no arrival), so its consumers' wait on it runs out
-                if (p.stall && cta == 0 && it == 0) continue;
-                const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
-                if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's control flow uniform
-                    stop = true;
-                    break;
+        auto q_write = [&](int s, int seg, int b, int rb, int hkv, const BatchGeom &G) {
+            (void)seg;
+            const uint32_t qs = smem_base + C::OFF_Q + s * C::Q_BYTES;
+            for (int idx = lane; idx < kRowsPerCta * (DQK / 8); idx += 32) {
+                const int r = idx / (DQK / 8), c = idx % (DQK / 8);
+                const int rq = rb * kRowsPerCta + r;
+                const T *src = qg;
+                uint32_t nbytes = 0;
+                if (rq < G.R && c * 8 < p.dqk) {  // dims past the call's head dim stay zero
+                    const int hq = hkv * p.g + rq / G.Lq, i = rq % G.Lq;
+                    src = qg + b * p.q_sb + (long long)(G.q0 + i) * p.q_sl + (long long)hq * p.q_sh + c * 8;
+                    nbytes = 16;
                 }
-                const uint32_t kdst = smem_base + s * C::STAGE_BYTES;
-                const uint32_t vdst = kdst + C::KBOX * C::BOX_BYTES;
-                // (one piece per CTA: the piece's last tile is the CTA's last tile)
-                const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
-                                  (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
-                const int j = tt * C::TK;
-                if (!p.block_table) {
-                    if (lane == 0) {
-                        mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
-#pragma unroll
-                        for (int c = 0; c < C::KBOX; ++c)
-                            tma_load_4d(kdst + c * C::BOX_BYTES, &tmK, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
-#pragma unroll
-                        for (int c = 0; c < C::VBOX; ++c)
-                            tma_load_4d(vdst + c * C::BOX_BYTES, &tmV, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
-                    }
-                } else {
-                    // Paged K/V: the tile is gathered page by page.  A page of at
-                    // least TK keys gives one box of TK rows; a smaller page gives
-                    // TK / page boxes of `page` rows, stacked in the stage exactly
-                    // where one TK-row box would put them (a box of 8 or more rows
-                    // starts on a 1024-byte swizzle period).  The lanes share the
-                    // boxes; a page past the table or an invalid block number
-                    // reads as zeros (out-of-range coordinates).
-                    if (lane == 0) mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
-                    __syncwarp();
-                    const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
-                    const int nsub = C::TK >> sub_shift;
-                    for (int idx = lane; idx < (C::KBOX + C::VBOX) * nsub; idx += 32) {
-                        const int c = idx / nsub, sub = idx - c * nsub;
-                        const int key = j + (sub << sub_shift);
-                        const int page = key >> p.page_shift;
-                        int blk = p.num_blocks;
-                        if (page < p.max_pages) {
-                            const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
-                            if (e >= 0 && e < p.num_blocks) blk = e;
-                        }
-                        const int row = key & ((1 << p.page_shift) - 1);
-                        const uint32_t off = (uint32_t)(sub << sub_shift) * 128u;
-                        if (c < C::KBOX)
-                            tma_load_4d(kdst + c * C::BOX_BYTES + off, &tmK, full_bar(s), c * 64, row, hkv, blk, policy);
-                        else
-                            tma_load_4d(vdst + (c - C::KBOX) * C::BOX_BYTES + off, &tmV, full_bar(s), (c - C::KBOX) * 64,
-                                        row, hkv, blk, policy);
-                    }
-                }
-                if (lane == 0) {
-                    StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
-                    meta[s] = m;
-                }
-                if (flags & kMetaFirst) {
-                    // the unit's 8 packed query rows (rows past g*Lq are zero), copied
-                    // asynchronously and counted on the same stage barrier
-                    const uint32_t qs = smem_base + C::OFF_Q + s * C::Q_BYTES;
-                    for (int idx = lane; idx < kRowsPerCta * (DQK / 8); idx += 32) {
-                        const int r = idx / (DQK / 8), c = idx % (DQK / 8);
-                        const int rq = rb * kRowsPerCta + r;
-                        const T *src = qg;
-                        uint32_t nbytes = 0;
-                        if (rq < G.R && c * 8 < p.dqk) {  // dims past the call's head dim stay zero
-                            const int hq = hkv * p.g + rq / G.Lq, i = rq % G.Lq;
-                            src = qg + b * p.q_sb + (long long)(G.q0 + i) * p.q_sl + (long long)hq * p.q_sh + c * 8;
-                            nbytes = 16;
-                        }
-                        cp_async_16(qs + (r * C::Q_STRIDE + c * 8) * 2, src, nbytes);
-                    }
-                    cp_async_mbar_arrive(full_bar(s));
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full_bar(s));
+                cp_async_16(qs + (r * C::Q_STRIDE + c * 8) * 2, src, nbytes);
             }
-        }
-        // end-of-work marker in the next stage (its previous load was consumed:
-        // the empty barrier says so)
-        const int s_done = it % STAGES;
-        bool done_sent = false;
-        {
-            const int use = it / STAGES;
-            bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
-            ok = __all_sync(0xffffffffu, ok);
-            if (lane == 0) {
-                StageMeta m = {0, 0, 0, 0, kMetaDone, 0, 0, 0};
-                meta[s_done] = m;
-            }
-            __syncwarp();
-            if (lane == 0 && ok) mbar_arrive(full_bar(s_done));
-            done_sent = ok;
-        }
-        // Never leave the CTA with copies in flight: wait (bounded, whatever
-        // the abort state) for the last load issued into each stage.  The
-        // marker's stage needs no wait once the marker went out.
-        if (lane == 0) {
-            for (int s = 0; s < STAGES && s < it; ++s) {
-                if (s == s_done && done_sent) continue;
-                const int last_use = (it - 1 - s) / STAGES;
-                volatile int no_abort = 0;
-                mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
-            }
-        }
+            cp_async_mbar_arrive(full_bar(s));
+            return true;
+        };
+        splitkv_produce<C, STAGES>(&tmK, &tmV, p, smem_base, full_bar(0), empty_bar(0), meta, abort_flag, q_write);
         return;
     }
 

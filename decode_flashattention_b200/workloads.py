@@ -76,6 +76,14 @@ for _pg in (16, 256):
         description=f"batched GQA decode, paged cache ({_pg}-key blocks, shuffled) bf16 B64 Hq32 Hkv8 "
                     f"D128, seqlens U[1,16384]")
 
+# GQA 8 with 4 speculative query positions over a batched KV cache: 32 packed
+# rows per kv head, one unit of the tcgen05 split-KV kernel (GQA 2/4/8 in the
+# MXFlashAttn README's capability table; qLen 1-8 in the SmallQ README).
+WORKLOADS["gqa8_specdec_kvcache_bf16"] = Workload(
+    "gqa8_specdec_kvcache_bf16", "kvcache", "blhd", torch.bfloat16, B=64, Lq=4, Hq=64, Hkv=8, Lk=16384, Dqk=128,
+    Dv=128, causal=True, seed=1008, seqlen_lo=1, seqlen_hi=16384,
+    description="batched GQA-8 speculative decode kvcache bf16 B64 qLen4 Hq64 Hkv8 D128, seqlens U[1,16384], causal")
+
 # Head dim 256 (the SmallQ README's validation shapes include hd 256): GQA 4
 # decode over an 8K context.
 WORKLOADS["gqa_decode_hd256_bf16"] = Workload(

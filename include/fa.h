@@ -103,7 +103,8 @@ typedef enum fa_variant {
     FA_VARIANT_AUTO = 0,
     FA_VARIANT_MMA = 1,     /* split-KV kernel, mma.sync tensor-core products */
     FA_VARIANT_SCALAR = 2,  /* split-KV kernel, fp32 FMA products (one packed row) */
-    FA_VARIANT_TCGEN05 = 3  /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 64/64 or 128/128) */
+    FA_VARIANT_TCGEN05 = 3, /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 64/64 or 128/128) */
+    FA_VARIANT_TCGEN05_SPLIT = 4 /* split-KV kernel on tcgen05 + TMEM: row blocks of 16 / 32 / 64 packed rows */
 } fa_variant;
 
 typedef struct fa_dispatch_info {
@@ -327,11 +328,21 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      fa_tcgen05_form), whole key range per CTA, no split
  *                      and no combine; dense fa_fwd calls with head dims
  *                      64/64 or 128/128.
+ *   FA_VARIANT_TCGEN05_SPLIT  the split-KV kernel on the 5th-gen tensor
+ *                      cores: a unit is a block of up to 64 packed query rows
+ *                      (16, 32 or 64: the g * Lq rows of a GQA group with
+ *                      their speculative positions), so K / V are streamed
+ *                      once for all of them; S^T = K Q^T with the 128 keys of
+ *                      a tile as the M side and the rows as N, O^T = V^T P^T,
+ *                      both accumulated in TMEM; head dims up to 192 / 128
+ *                      (every call API: dense, kvcache, paged, varlen, append).
  * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
  * least 128 packed rows (g * Lq >= 128) and head dims 64/64 or 128/128
- * (prefill-shaped calls); FA_VARIANT_MMA otherwise -- measured on B200 it is faster than the
- * FMA variant even for one packed row.  A forced variant that does not
- * support the call's shapes makes the call fail with FA_ERR_UNSUPPORTED.
+ * (prefill-shaped calls); FA_VARIANT_TCGEN05_SPLIT for more than 8 packed
+ * rows (g * Lq > 8) with Dqk <= 192 and Dv <= 128; FA_VARIANT_MMA otherwise --
+ * measured on B200 it is faster than the FMA variant even for one packed row.
+ * A forced variant that does not support the call's shapes makes the call
+ * fail with FA_ERR_UNSUPPORTED.
  */
 FA_API fa_status fa_force_variant(int variant);
 
