@@ -334,7 +334,10 @@ int log2_exact(int v) {
 
 // Plans the call; may change the row blocking of `s` (the tcgen05 split-KV
 // kernel takes row blocks of 16 to 64 packed rows).
-fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl) {
+// rows_override: the number of output rows when it is not B * Hq * Lq (packed
+// variable-length inputs: Hq * total_q).
+fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t max_keys, Plan *pl,
+                    int64_t rows_override = -1) {
     DeviceState *dev = nullptr;
     fa_status st = device_state(&dev);
     if (st) return st;
@@ -400,7 +403,7 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
         return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
     if (!ok) return fail(FA_ERR_UNSUPPORTED, "no kernel for variant %d, dtype %d, head dims (%d, %d)", variant,
                          s.dtype, s.Dqk, s.Dv);
-    if (!fa::get_combine_kernel(s.dtype, s.KDv, &pl->comb))
+    if (!fa::get_combine_kernel(s.dtype, s.KDv, s.rpc, &pl->comb))
         return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.KDv);
     if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
     pl->comb_smem = 0;
@@ -449,8 +452,13 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     pl->ws_o_off = 0;
     pl->ws_lse_off = pl->ws_o_off + ((o_floats * 4 + 255) & ~size_t(255));
     pl->ws_bytes = pl->need_workspace ? pl->ws_lse_off + ((lse_floats * 4 + 255) & ~size_t(255)) : 0;
-    int64_t rows = (int64_t)s.B * s.Hq * s.Lq;
-    pl->comb_grid = (int)((rows + 3) / 4);
+    // the combine kernel: a warp per output row, or one to four per unit
+    const int64_t nunits = (int64_t)s.B * s.RB * s.Hkv;
+    const int64_t nrows = rows_override >= 0 ? rows_override : (int64_t)s.B * s.Hq * s.Lq;
+    if (nunits > INT32_MAX || nrows > 4 * (int64_t)INT32_MAX)
+        return fail(FA_ERR_UNSUPPORTED, "too many work units (%lld) or rows (%lld)", (long long)nunits,
+                    (long long)nrows);
+    pl->comb_grid = fa::combine_grid(nrows, nunits, s.rpc, s.R);
     return FA_OK;
 }
 
@@ -538,9 +546,9 @@ fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor 
         return FA_OK;
     }
     Plan pl;
-    fa_status st = make_plan(s, causal, num_splits, seqlens != nullptr || vl != nullptr, s.Lk, &pl);
+    fa_status st = make_plan(s, causal, num_splits, seqlens != nullptr || vl != nullptr, s.Lk, &pl,
+                             vl ? (int64_t)s.Hq * vl->total_q : -1);
     if (st) return st;
-    if (vl) pl.comb_grid = (int)(((int64_t)s.Hq * vl->total_q + 3) / 4);
     if (workspace_bytes < pl.ws_bytes)
         return fail(FA_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes,
                     pl.ws_bytes);

@@ -19,8 +19,10 @@ struct KernelInfo {
 
 // Main split-KV kernel using mma.sync (keys as M, packed rows as N).
 bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
-// LSE-weighted combine of split partials.
-bool get_combine_kernel(int dtype, int dv, KernelInfo *out);
+// LSE-weighted combine of split partials for row blocks of rpc rows, and its
+// grid for `rows` output rows in `units` units (R packed rows per kv head).
+bool get_combine_kernel(int dtype, int dv, int rpc, KernelInfo *out);
+int combine_grid(long long rows, long long units, int rpc, int R);
 
 // Dense attention on tcgen05 for calls with many packed rows (fa_prefill.cu).
 // form: an fa_tcgen05_form other than FA_TCGEN05_AUTO.

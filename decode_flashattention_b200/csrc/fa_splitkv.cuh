@@ -90,30 +90,88 @@ struct SplitCfg {
 };
 
 
-// The producer warp's loop, shared by the split-KV kernels: walks the CTA's
-// piece of the key-tile space (the Partition) segment by segment and feeds the
-// STAGES-deep ring -- per tile the TMA loads of K and V (C::KBOX and C::VBOX
-// boxes of C::TK keys x 64 elements, 128-byte swizzle, L2 evict-first, no
-// multicast; a paged cache gathered page by page) and the stage header; at the
-// first tile of each segment q_write(s, seg, b, rb, hkv, G) (all 32 lanes)
-// stages the unit's query rows and returns false if a wait gave up.  full0 /
-// empty0: shared addresses of the stages' full / empty barriers (8 bytes
-// apart).  Ends with the end-of-work marker and a bounded wait for every copy
-// still in flight.  Must be called by all 32 lanes of the warp.
 // Tiles of a CTA's piece the producer asks L2 for before waiting on the
 // previous kernel (dense K / V).
 #ifndef FA_PREFETCH_TILES
 #define FA_PREFETCH_TILES 2
 #endif
 constexpr int kPrefetchTiles = FA_PREFETCH_TILES;
+// Tile-by-tile cursor over a piece: a SegmentWalker plus the tile within the
+// current segment (device code, any single lane).
+struct TileCursor {
+    SegmentWalker w;
+    int tt, t1;
+    __device__ __forceinline__ void start(const SegmentWalker &wk) {
+        w = wk;
+        tt = w.done() ? 0 : w.pos - w.u0;
+        t1 = w.done() ? 0 : w.seg_end() - w.u0;
+    }
+    __device__ __forceinline__ bool done() const { return w.done(); }
+    __device__ __forceinline__ void next(const Params &p) {
+        if (++tt < t1) return;
+        w.advance(p);
+        if (!w.done()) {
+            tt = w.pos - w.u0;
+            t1 = w.seg_end() - w.u0;
+        }
+    }
+};
 
-template <class C, int STAGES, class QW>
+// L2 prefetch of the K and V boxes of the cursor's tile (dense K / V).
+template <class C>
+__device__ __forceinline__ void prefetch_tile(const CUtensorMap *tmK, const CUtensorMap *tmV, const Params &p,
+                                              const TileCursor &pc) {
+    const int b = pc.w.b(p);
+    const BatchGeom G = batch_geom(p, b);
+    const int kb = p.cu_q ? 0 : b;
+    const int key = G.k0 + pc.tt * C::TK;
+#pragma unroll
+    for (int c = 0; c < C::KBOX; ++c) tma_prefetch_4d(tmK, c * 64, key, pc.w.hkv, kb);
+#pragma unroll
+    for (int c = 0; c < C::VBOX; ++c) tma_prefetch_4d(tmV, c * 64, key, pc.w.hkv, kb);
+}
+
+// The producer warp's loop, shared by the split-KV kernels: walks the CTA's
+// piece of the key-tile space (the Partition) segment by segment and feeds the
+// copy ring(s) -- per tile the TMA loads of K and V (C::KBOX and C::VBOX
+// boxes of C::TK keys x 64 elements, 128-byte swizzle, L2 evict-first, no
+// multicast; a paged cache gathered page by page) and the tile header (in
+// meta[stage], or meta[it % kMetaRing] with separate rings); at the first tile of each segment q_write(s, seg, b, rb, hkv,
+// G) (all 32 lanes, s the K slot) stages the unit's query rows and returns
+// false if a wait gave up.  Ends with the end-of-work marker and a bounded
+// wait for every copy still in flight.  Must be called by all 32 lanes of the
+// warp.
+//
+// Where a tile's K and V go.  Joint stages (VS == 0 in splitkv_produce): K
+// and V of tile it share stage it % KS (V right after K) and its full / empty
+// barriers.  Separate rings (VS > 0): K goes to K slot it % KS and V to V slot
+// it % VS, each with its own full / empty barriers, so K can be released as
+// soon as the products that read it are done while V waits for its own.
+// With separate rings the tile headers have a ring of their own,
+// meta[it % kMetaRing]: the producer can run at most KS tiles ahead of the S
+// products and those at most two tiles ahead of the softmax, so a header is
+// read before its entry comes round again as long as KS + 3 <= kMetaRing.
+constexpr int kMetaRing = 8;
+
+struct RingLayout {
+    uint32_t k_base, k_stride;  // shared address of K slot 0, bytes between slots
+    uint32_t v_base, v_stride;  // V slot 0 (joint: stage 0's V boxes), bytes between slots
+    uint32_t kfull0, kempty0;   // barrier arrays of the K slots / joint stages (8 bytes apart)
+    uint32_t vfull0, vempty0;   // barrier arrays of the V slots (separate rings only)
+};
+
+template <class C, int KS, int VS, class QW>
 __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CUtensorMap *tmV, const Params &p,
-                                                uint32_t smem_base, uint32_t full0, uint32_t empty0,
-                                                StageMeta *meta, volatile int *abort_flag, QW &&q_write) {
+                                                const RingLayout &R, StageMeta *meta, volatile int *abort_flag,
+                                                QW &&q_write) {
+    constexpr bool kJoint = VS == 0;
+    static_assert(kJoint || KS + 3 <= kMetaRing, "header ring deep enough for the K ring");
+    constexpr uint32_t kKBytes = C::KBOX * C::BOX_BYTES, kVBytes = C::VBOX * C::BOX_BYTES;
     const int lane = threadIdx.x & 31;
-    auto full_bar = [&](int s) { return full0 + 8u * s; };
-    auto empty_bar = [&](int s) { return empty0 + 8u * s; };
+    auto kfull = [&](int s) { return R.kfull0 + 8u * s; };
+    auto kempty = [&](int s) { return R.kempty0 + 8u * s; };
+    auto vfull = [&](int s) { return R.vfull0 + 8u * s; };
+    auto vempty = [&](int s) { return R.vempty0 + 8u * s; };
     // Dense inputs: the schedule needs only the kernel's parameters, so it
     // is worked out before the wait and overlaps the previous kernel; cache
     // or sequence lengths are read only after the wait.
@@ -136,18 +194,9 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
         // it only moves the first HBM reads ahead, into the previous
         // kernel's tail, where the memory system is mostly idle.
         if (active && lane == 0 && !p.block_table) {
-            SegmentWalker pw = wk;
-            int n = 0;
-            for (; !pw.done() && n < kPrefetchTiles; pw.advance(p)) {
-                const BatchGeom G = batch_geom(p, pw.b(p));
-                const int kb = pw.b(p);
-                for (int tt = pw.pos - pw.u0; tt < pw.seg_end() - pw.u0 && n < kPrefetchTiles; ++tt, ++n) {
-#pragma unroll
-                    for (int c = 0; c < C::KBOX; ++c) tma_prefetch_4d(tmK, c * 64, G.k0 + tt * C::TK, pw.hkv, kb);
-#pragma unroll
-                    for (int c = 0; c < C::VBOX; ++c) tma_prefetch_4d(tmV, c * 64, G.k0 + tt * C::TK, pw.hkv, kb);
-                }
-            }
+            TileCursor pc;
+            pc.start(wk);
+            for (int n = 0; n < kPrefetchTiles && !pc.done(); ++n, pc.next(p)) prefetch_tile<C>(tmK, tmV, p, pc);
         }
         __syncwarp();
     }
@@ -158,111 +207,154 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
     if (!uniform_batches(p)) plan();
 
     const uint64_t policy = l2_policy_evict_first();
-    int it = 0, seg = 0;
+    // Issues the boxes of one tile's K (V_PART false) or V (true) -- or both,
+    // for joint stages -- completing on `bar`.  Paged K / V: the tile is
+    // gathered page by page.  A page of at least TK keys gives one box of TK
+    // rows; a smaller page gives TK / page boxes of `page` rows, stacked in
+    // the slot exactly where one TK-row box would put them (a box of 8 or more
+    // rows starts on a 1024-byte swizzle period).  The lanes share the boxes;
+    // a page past the table or an invalid block number reads as zeros
+    // (out-of-range coordinates).
+    auto issue = [&](bool do_k, bool do_v, uint32_t kdst, uint32_t vdst, uint32_t bar, int b, int hkv,
+                     const BatchGeom &G, int j) {
+        const int kb = p.cu_q ? 0 : b;  // K / V batch coordinate (packed inputs: one batch of tokens)
+        if (lane == 0) mbar_expect_tx(bar, (do_k ? kKBytes : 0u) + (do_v ? kVBytes : 0u));
+        if (!p.block_table) {
+            if (lane == 0) {
+                if (do_k) {
+#pragma unroll
+                    for (int c = 0; c < C::KBOX; ++c)
+                        tma_load_4d(kdst + c * C::BOX_BYTES, tmK, bar, c * 64, G.k0 + j, hkv, kb, policy);
+                }
+                if (do_v) {
+#pragma unroll
+                    for (int c = 0; c < C::VBOX; ++c)
+                        tma_load_4d(vdst + c * C::BOX_BYTES, tmV, bar, c * 64, G.k0 + j, hkv, kb, policy);
+                }
+            }
+        } else {
+            __syncwarp();
+            const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
+            const int nsub = C::TK >> sub_shift;
+            const int c0 = do_k ? 0 : C::KBOX, c1 = do_v ? C::KBOX + C::VBOX : C::KBOX;
+            for (int idx = lane; idx < (c1 - c0) * nsub; idx += 32) {
+                const int c = c0 + idx / nsub, sub = idx % nsub;
+                const int key = j + (sub << sub_shift);
+                const int page = key >> p.page_shift;
+                int blk = p.num_blocks;
+                if (page < p.max_pages) {
+                    const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
+                    if (e >= 0 && e < p.num_blocks) blk = e;
+                }
+                const int row = key & ((1 << p.page_shift) - 1);
+                const uint32_t off = (uint32_t)(sub << sub_shift) * 128u;
+                if (c < C::KBOX)
+                    tma_load_4d(kdst + c * C::BOX_BYTES + off, tmK, bar, c * 64, row, hkv, blk, policy);
+                else
+                    tma_load_4d(vdst + (c - C::KBOX) * C::BOX_BYTES + off, tmV, bar, (c - C::KBOX) * 64, row, hkv,
+                                blk, policy);
+            }
+        }
+    };
+    int it = 0, itv = 0, seg = 0;  // tiles whose K (joint: K and V) / separate V were issued
     bool stop = !active;
     const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
     for (; active && !wk.done() && !stop; wk.advance(p), ++seg) {
         const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
         const BatchGeom G = batch_geom(p, b);
-        const int kb = p.cu_q ? 0 : b;  // K / V batch coordinate (packed inputs: one batch of tokens)
         const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
         const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
         const int slot = (wk.pos == lo) ? 0 : 1;
         for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
-            const int s = it % STAGES, use = it / STAGES;
-            // test hook: the first CTA leaves its first stage empty (no copy,
-            // no arrival), so its consumers' wait on it runs out
-            if (p.stall && cta == 0 && it == 0) continue;
-            const bool ok = use == 0 || mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+            const int s = it % KS, use = it / KS;
+            // test hook: the first CTA leaves its first tile's slots empty (no
+            // copy, no arrival), so the consumers' wait on it runs out
+            if (p.stall && cta == 0 && it == 0) {
+                if (!kJoint) ++itv;
+                continue;
+            }
+            bool ok = use == 0 || mbar_wait(kempty(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) {  // keep the warp's control flow uniform
                 stop = true;
                 break;
             }
-            const uint32_t kdst = smem_base + s * C::STAGE_BYTES;
-            const uint32_t vdst = kdst + C::KBOX * C::BOX_BYTES;
+            const uint32_t kdst = R.k_base + s * R.k_stride;
             // (one piece per CTA: the piece's last tile is the CTA's last tile)
             const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
                               (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
             const int j = tt * C::TK;
-            if (!p.block_table) {
-                if (lane == 0) {
-                    mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::KBOX; ++c)
-                        tma_load_4d(kdst + c * C::BOX_BYTES, tmK, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
-#pragma unroll
-                    for (int c = 0; c < C::VBOX; ++c)
-                        tma_load_4d(vdst + c * C::BOX_BYTES, tmV, full_bar(s), c * 64, G.k0 + j, hkv, kb, policy);
-                }
-            } else {
-                // Paged K/V: the tile is gathered page by page.  A page of at
-                // least TK keys gives one box of TK rows; a smaller page gives
-                // TK / page boxes of `page` rows, stacked in the stage exactly
-                // where one TK-row box would put them (a box of 8 or more rows
-                // starts on a 1024-byte swizzle period).  The lanes share the
-                // boxes; a page past the table or an invalid block number
-                // reads as zeros (out-of-range coordinates).
-                if (lane == 0) mbar_expect_tx(full_bar(s), C::STAGE_BYTES);
-                __syncwarp();
-                const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
-                const int nsub = C::TK >> sub_shift;
-                for (int idx = lane; idx < (C::KBOX + C::VBOX) * nsub; idx += 32) {
-                    const int c = idx / nsub, sub = idx - c * nsub;
-                    const int key = j + (sub << sub_shift);
-                    const int page = key >> p.page_shift;
-                    int blk = p.num_blocks;
-                    if (page < p.max_pages) {
-                        const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
-                        if (e >= 0 && e < p.num_blocks) blk = e;
-                    }
-                    const int row = key & ((1 << p.page_shift) - 1);
-                    const uint32_t off = (uint32_t)(sub << sub_shift) * 128u;
-                    if (c < C::KBOX)
-                        tma_load_4d(kdst + c * C::BOX_BYTES + off, tmK, full_bar(s), c * 64, row, hkv, blk, policy);
-                    else
-                        tma_load_4d(vdst + (c - C::KBOX) * C::BOX_BYTES + off, tmV, full_bar(s), (c - C::KBOX) * 64,
-                                    row, hkv, blk, policy);
-                }
-            }
+            issue(true, kJoint, kdst, R.v_base + s * R.v_stride, kfull(s), b, hkv, G, j);
             if (lane == 0) {
                 StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
-                meta[s] = m;
+                meta[kJoint ? s : it % kMetaRing] = m;
             }
             const bool qok = !(flags & kMetaFirst) || __all_sync(0xffffffffu, q_write(s, seg, b, rb, hkv, G));
             __syncwarp();
-            if (lane == 0) mbar_arrive(full_bar(s));
-            if (!qok) {  // a wait gave up (the CTA is aborting): the stage still completes, then stop
+            if (lane == 0) mbar_arrive(kfull(s));
+            if (!qok) {  // a wait gave up (the CTA is aborting): the slot still completes, then stop
                 stop = true;
                 ++it;
                 break;
             }
+            if constexpr (!kJoint) {
+                const int vs = itv % VS, vuse = itv / VS;
+                ok = vuse == 0 || mbar_wait(vempty(vs), (vuse - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    stop = true;
+                    ++it;
+                    break;
+                }
+                issue(false, true, 0u, R.v_base + vs * R.v_stride, vfull(vs), b, hkv, G, j);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(vfull(vs));
+                ++itv;
+            }
         }
     }
-    // end-of-work marker in the next stage (its previous load was consumed:
-    // the empty barrier says so)
-    const int s_done = it % STAGES;
-    bool done_sent = false;
+    // end-of-work marker in the next K slot / stage (its previous load was
+    // consumed: the empty barrier says so); with separate rings it completes
+    // the next V slot's phase as well, since consumers may take the tile
+    // header from either ring's barrier
+    const int s_done = it % KS, v_done = itv % (kJoint ? 1 : VS);
+    bool done_sent = false, vdone_sent = false;
     {
-        const int use = it / STAGES;
-        bool ok = use == 0 || mbar_wait(empty_bar(s_done), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+        const int use = it / KS;
+        bool ok = use == 0 || mbar_wait(kempty(s_done), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+        bool vok = kJoint;
+        if constexpr (!kJoint) {
+            const int vuse = itv / VS;
+            vok = ok && (vuse == 0 || mbar_wait(vempty(v_done), (vuse - 1) & 1, abort_flag, p.status, p.wait_limit_ns));
+        }
         ok = __all_sync(0xffffffffu, ok);
+        vok = __all_sync(0xffffffffu, vok);
         if (lane == 0) {
             StageMeta m = {0, 0, 0, 0, kMetaDone, 0, 0, 0};
-            meta[s_done] = m;
+            meta[kJoint ? s_done : it % kMetaRing] = m;
         }
         __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(full_bar(s_done));
+        if (lane == 0 && ok) mbar_arrive(kfull(s_done));
+        if constexpr (!kJoint) {
+            if (lane == 0 && vok) mbar_arrive(vfull(v_done));
+        }
         done_sent = ok;
+        vdone_sent = !kJoint && vok;
     }
     // Never leave the CTA with copies in flight: wait (bounded, whatever
-    // the abort state) for the last load issued into each stage.  The
-    // marker's stage needs no wait once the marker went out.
+    // the abort state) for the last load issued into each slot.  The
+    // marker's slot needs no wait once the marker went out.
     if (lane == 0) {
-        for (int s = 0; s < STAGES && s < it; ++s) {
+        volatile int no_abort = 0;
+        for (int s = 0; s < KS && s < it; ++s) {
             if (s == s_done && done_sent) continue;
-            const int last_use = (it - 1 - s) / STAGES;
-            volatile int no_abort = 0;
-            mbar_wait(full_bar(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
+            const int last_use = (it - 1 - s) / KS;
+            mbar_wait(kfull(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
+        }
+        if constexpr (!kJoint) {
+            for (int s = 0; s < VS && s < itv; ++s) {
+                if (s == v_done && vdone_sent) continue;
+                const int last_use = (itv - 1 - s) / VS;
+                mbar_wait(vfull(s), last_use & 1, &no_abort, p.status, p.wait_limit_ns / 8);
+            }
         }
     }
 }
@@ -330,7 +422,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             cp_async_mbar_arrive(full_bar(s));
             return true;
         };
-        splitkv_produce<C, STAGES>(&tmK, &tmV, p, smem_base, full_bar(0), empty_bar(0), meta, abort_flag, q_write);
+        const RingLayout ring = {smem_base, (uint32_t)C::STAGE_BYTES, smem_base + C::KBOX * C::BOX_BYTES,
+                                 (uint32_t)C::STAGE_BYTES, full_bar(0), empty_bar(0), 0u, 0u};
+        splitkv_produce<C, STAGES, 0>(&tmK, &tmV, p, ring, meta, abort_flag, q_write);
         return;
     }
 

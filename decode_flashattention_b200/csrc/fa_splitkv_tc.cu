@@ -57,50 +57,55 @@ constexpr uint32_t kTmemCols = 256;  // S^T buffers at columns 0 and 64, O^T at 
 constexpr int kPvN = 64;             // N of the PV products (rows, zero padded)
 }  // namespace tcd
 
-template <int DQK, int DV, int NR, int STAGES>
+template <int DQK, int DV, int NR, int KS, int VS>
 struct TcCfg {
     static constexpr int TK = 128;
     static constexpr int TK_SHIFT = 7;
     static constexpr int KBOX = DQK / 64;
     static constexpr int VBOX = DV / 64;
     static constexpr int BOX_BYTES = TK * 128;                      // 128 keys x 64 elements
-    static constexpr int STAGE_BYTES = (KBOX + VBOX) * BOX_BYTES;   // K and V of one tile
+    static constexpr int K_BYTES = KBOX * BOX_BYTES;                // K of one tile
+    static constexpr int V_BYTES = VBOX * BOX_BYTES;                // V of one tile
     static constexpr int Q_BOX = NR * 128;                          // NR rows x 64 elements
     static constexpr int Q_BYTES = KBOX * Q_BOX;
     static constexpr int P_BYTES = TK * 128;                        // P^T: 128 keys x 64 rows
-    static constexpr int OFF_Q = STAGES * STAGE_BYTES;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + KS * K_BYTES;
+    static constexpr int OFF_Q = OFF_V + VS * V_BYTES;
     static constexpr int OFF_P = OFF_Q + Q_BYTES;
     static constexpr int OFF_META = OFF_P + P_BYTES;
-    static constexpr int NBARS = 2 * STAGES + 10;
-    static constexpr int OFF_BAR = OFF_META + STAGES * (int)sizeof(StageMeta);
+    static constexpr int NBARS = 2 * KS + 2 * VS + 10;
+    static constexpr int OFF_BAR = OFF_META + kMetaRing * (int)sizeof(StageMeta);
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;            // tmem base, abort flag, tile flags [2][4]
     static constexpr int OFF_M = (OFF_MISC + 48 + 15) & ~15;        // running max per row [NR]
     static constexpr int OFF_A = OFF_M + NR * 4;                    // rescale factors / row sums [NR]
     static constexpr int OFF_LIM = OFF_A + NR * 4;                  // last visible key per row [NR]
-    static constexpr int OFF_RED = OFF_LIM + NR * 4;                // per-warp row maxima / sums [4][NR]
+    static constexpr int OFF_RED = OFF_LIM + NR * 4;                // per-warp row maxima [4][NR]
     static constexpr int SMEM_USED = OFF_RED + 4 * NR * 4;
     // the dynamic shared memory base is at least 16-byte aligned, so 1008
     // bytes of slack always reach the next 1024-byte boundary
     static constexpr int SMEM = SMEM_USED + 1008;
     static_assert(DQK % 64 == 0 && DV == 128, "instances: head dims (128 | 192, 128)");
     static_assert(NR % 16 == 0 && NR >= 16 && NR <= tcd::kPvN, "16 to 64 packed rows (N of the S products)");
-    static_assert(Q_BOX % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms on 1024-byte boundaries");
+    static_assert(Q_BOX % 1024 == 0 && OFF_V % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_P % 1024 == 0,
+                  "swizzle atoms on 1024-byte boundaries");
     static_assert(SMEM <= 232448, "fits the 227 KB per-CTA shared memory limit");
 };
 
-template <typename T>
-__device__ __forceinline__ T from_float(float x);
-template <>
-__device__ __forceinline__ __half from_float<__half>(float x) { return __float2half_rn(x); }
-template <>
-__device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+// Maximum over the warp's 32 lanes (sm_100 warp reduction on fp32; NaN inputs
+// are ignored, -inf is the identity).
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
 
-template <typename T, int DQK, int DV, int NR, int STAGES>
+template <typename T, int DQK, int DV, int NR, int KS, int VS>
 __global__ void __launch_bounds__(tcd::kThreads, 1)
     splitkv_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const Params p) {
     using namespace pf;
-    using C = TcCfg<DQK, DV, NR, STAGES>;
+    using C = TcCfg<DQK, DV, NR, KS, VS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -109,12 +114,18 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
 
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
-    const uint32_t full0 = bar(0), empty0 = bar(STAGES);
-    auto full_bar = [&](int s) { return full0 + 8u * s; };
-    auto empty_bar = [&](int s) { return empty0 + 8u * s; };
-    const uint32_t sfull0 = bar(2 * STAGES), sfree0 = bar(2 * STAGES + 2);
-    const uint32_t pready = bar(2 * STAGES + 4), pdone = bar(2 * STAGES + 5), ofree = bar(2 * STAGES + 6);
-    const uint32_t qfree = bar(2 * STAGES + 7), drain = bar(2 * STAGES + 8), syncb = bar(2 * STAGES + 9);
+    // K slots: kfull (TMA bytes + the producer's arrival), kempty (the S
+    // products' commit); V slots: vfull, vempty (the PV products' commit); the
+    // tile headers are in their own ring, meta[it % kMetaRing]
+    const uint32_t kfull0 = bar(0), kempty0 = bar(KS), vfull0 = bar(2 * KS), vempty0 = bar(2 * KS + VS);
+    auto kfull = [&](int s) { return kfull0 + 8u * s; };
+    auto kempty = [&](int s) { return kempty0 + 8u * s; };
+    auto vfull = [&](int s) { return vfull0 + 8u * s; };
+    auto vempty = [&](int s) { return vempty0 + 8u * s; };
+    constexpr int B0 = 2 * KS + 2 * VS;
+    const uint32_t sfull0 = bar(B0), sfree0 = bar(B0 + 2);
+    const uint32_t pready = bar(B0 + 4), pdone = bar(B0 + 5), ofree = bar(B0 + 6);
+    const uint32_t qfree = bar(B0 + 7), drain = bar(B0 + 8), syncb = bar(B0 + 9);
     StageMeta *meta = reinterpret_cast<StageMeta *>(smem + C::OFF_META);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
@@ -125,9 +136,13 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
     float *red_sh = reinterpret_cast<float *>(smem + C::OFF_RED);
 
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);  // one tcgen05.commit after the tile's PV products
+        for (int s = 0; s < KS; ++s) {
+            mbar_init(kfull(s), 1);
+            mbar_init(kempty(s), 1);
+        }
+        for (int s = 0; s < VS; ++s) {
+            mbar_init(vfull(s), 1);
+            mbar_init(vempty(s), 1);  // one tcgen05.commit after the tile's PV products
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(sfull0 + 8u * b, 1);
@@ -197,53 +212,56 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
             fence_proxy_async_smem();  // the tensor core reads the slot through the async proxy
             return true;
         };
-        splitkv_produce<C, STAGES>(&tmK, &tmV, p, sb, full0, empty0, meta, abort_flag, q_write);
+        const RingLayout ring = {sb + C::OFF_K, (uint32_t)C::K_BYTES, sb + C::OFF_V, (uint32_t)C::V_BYTES,
+                                 kfull0, kempty0, vfull0, vempty0};
+        splitkv_produce<C, KS, VS>(&tmK, &tmV, p, ring, meta, abort_flag, q_write);
     } else if (warp == tcd::kMmaWarp) {
         // ============================================================ MMA issue (one thread)
         if (lane == 0) {
             const uint32_t idesc_s = instr_desc(bf16, 128, NR, false, false);        // S^T: K-major K and Q
             const uint32_t idesc_o = instr_desc(bf16, 128, tcd::kPvN, true, true);    // O^T: MN-major V and P^T
             const uint64_t dq0 = smem_desc(sb + C::OFF_Q, 16, 1024);
-            const uint64_t dk0 = smem_desc(sb, 16, 1024);                                   // stage 0's K
-            const uint64_t dv0 = smem_desc(sb + C::KBOX * C::BOX_BYTES, C::BOX_BYTES, 1024);  // stage 0's V
+            const uint64_t dk0 = smem_desc(sb + C::OFF_K, 16, 1024);                // K slot 0
+            const uint64_t dv0 = smem_desc(sb + C::OFF_V, C::BOX_BYTES, 1024);      // V slot 0
             const uint64_t dp0 = smem_desc(sb + C::OFF_P, C::BOX_BYTES, 1024);
             auto wait = [&](uint32_t b, uint32_t parity) {
                 return mbar_wait(b, parity, abort_flag, p.status, p.wait_limit_ns);
             };
             // tile j's PV products (P^T(j) written, the O^T of its segment free)
-            int pv_s = 0, pv_seg = 0;
+            int pv_seg = 0;
             bool pv_first = false, pending = false;
             auto issue_pv = [&](int j) {
-                if (!wait(pready, j & 1)) return false;
+                const int vs = j % VS;
+                if (!wait(pready, j & 1) || !wait(vfull(vs), (j / VS) & 1)) return false;
                 if (pv_first && pv_seg > 0 && !wait(ofree, (pv_seg - 1) & 1)) return false;
                 tc_fence_after();
-                const uint64_t dv = dv0 + (uint64_t)((pv_s * C::STAGE_BYTES) >> 4);
+                const uint64_t dv = dv0 + (uint64_t)((vs * C::V_BYTES) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < C::TK / 16; ++ks)
                     umma(tmem + 128, dv + (uint64_t)((ks * 2048) >> 4), dp0 + (uint64_t)((ks * 2048) >> 4), idesc_o,
                          (pv_first && ks == 0) ? 0u : 1u);
                 umma_commit(pdone);
-                umma_commit(empty_bar(pv_s));  // K and V of the tile are read
+                umma_commit(vempty(vs));  // the tile's V is read
                 return true;
             };
             int it = 0, seg = -1;
             bool ok = true;
             for (;; ++it) {
-                const int s = it % STAGES, use = it / STAGES;
-                // while this tile's copies are still landing, the previous
-                // tile's PV can go first (it frees a stage sooner)
-                if (pending && !mbar_try_wait(full_bar(s), use & 1)) {
+                const int s = it % KS, use = it / KS;
+                // while this tile's K is still landing, the previous tile's PV
+                // can go first (it frees a V slot sooner)
+                if (pending && !mbar_try_wait(kfull(s), use & 1)) {
                     if (!(ok = issue_pv(it - 1))) break;
                     pending = false;
                 }
-                if (!(ok = wait(full_bar(s), use & 1))) break;
-                const StageMeta md = meta[s];
+                if (!(ok = wait(kfull(s), use & 1))) break;
+                const StageMeta md = meta[it % kMetaRing];
                 if (md.flags & kMetaDone) break;
                 if (md.flags & kMetaFirst) ++seg;
                 // S^T(it) into buffer it & 1, last read by the softmax of tile it - 2
                 if (it >= 2 && !(ok = wait(sfree0 + 8u * (it & 1), ((it >> 1) - 1) & 1))) break;
                 tc_fence_after();
-                const uint64_t dk = dk0 + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                const uint64_t dk = dk0 + (uint64_t)((s * C::K_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
                     const uint32_t ok_ = (uint32_t)(((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4);
@@ -251,10 +269,10 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
                     umma(tmem + (uint32_t)((it & 1) * 64), dk + ok_, dq0 + oq, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(sfull0 + 8u * (it & 1));
+                umma_commit(kempty(s));  // the tile's K is read once its S products are done
                 if (md.flags & kMetaLast) umma_commit(qfree);  // the segment's last read of the Q slot
                 if (pending && !(ok = issue_pv(it - 1))) break;
                 pending = true;
-                pv_s = s;
                 pv_seg = seg;
                 pv_first = (md.flags & kMetaFirst) != 0;
             }
@@ -277,10 +295,13 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
         int minlim = 0, rreal = 0;
         BatchGeom G = {0, 0, 0, 0, 0};
         for (int it = 0;; ++it) {
-            const int s = it % STAGES;
-            bool ok = mbar_wait(full_bar(s), (it / STAGES) & 1, abort_flag, p.status, p.wait_limit_ns);
+            // The tile header (and V) through the V slot's barrier: a V slot is
+            // refilled only after this tile's PV, which needs this group's P, so
+            // the wait can never fall a whole phase behind -- unlike a K slot,
+            // which the S products free two tiles ahead of the softmax.
+            bool ok = mbar_wait(vfull(it % VS), (it / VS) & 1, abort_flag, p.status, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
-            const StageMeta md = meta[s];
+            const StageMeta md = meta[it % kMetaRing];
             if (md.flags & kMetaDone) break;
             const bool first = (md.flags & kMetaFirst) != 0;
             if (first) {
@@ -342,12 +363,11 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
             if (!csync()) break;
             const int fb = (it & 1) * 4;
             if (flag_sh[fb] | flag_sh[fb + 1] | flag_sh[fb + 2] | flag_sh[fb + 3]) {
-                // per-row max over this warp's 32 keys, then over the 4 warps
+                // per-row max over this warp's 32 keys (one warp reduction per
+                // row), then over the 4 warps
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
-                    float v = x[r];
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                    const float v = warp_max_f32(x[r]);
                     if (lane == (r & 31)) red_sh[warp * NR + r] = v;
                 }
                 if (!csync()) break;
@@ -386,8 +406,8 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
             }
             // ---- cache slots at or beyond the batch's length may hold anything
             // (NaN included): zero this key's V row so 0 * V stays 0
-            if ((p.seqlens || p.cu_q) && key >= G.n) {
-                const uint32_t vrow = sb + s * C::STAGE_BYTES + C::KBOX * C::BOX_BYTES + tid * 128;
+            if ((p.seqlens || p.cu_q) && key >= G.n) {  // (this tile's V has landed: vfull above)
+                const uint32_t vrow = sb + C::OFF_V + (it % VS) * C::V_BYTES + tid * 128;
 #pragma unroll
                 for (int c = 0; c < C::VBOX * 8; ++c) {
                     const uint32_t a = vrow + (c >> 3) * C::BOX_BYTES + (c & 7) * 16;
@@ -424,57 +444,93 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
             if (!(md.flags & kMetaLast)) continue;
 
             // ================================================ segment epilogue
-            ok = mbar_wait(pdone, it & 1, abort_flag, p.status, p.wait_limit_ns);  // the last PV
+            // The last PV is done, so the P^T buffer is free until this warp
+            // group writes the next segment's first P: it stages the row sums
+            // and O (32 rows at a time), which lets every loop over rows stay
+            // rolled -- the epilogue runs once per segment and its code would
+            // otherwise be fetched cold each time.
+            ok = mbar_wait(pdone, it & 1, abort_flag, p.status, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            // row sums over the 128 keys
-#pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                float v = l[r];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == (r & 31)) red_sh[warp * NR + r] = v;
-            }
-            if (!csync()) break;
-            if (tid < NR) a_sh[tid] = (red_sh[tid] + red_sh[NR + tid]) + (red_sh[2 * NR + tid] + red_sh[3 * NR + tid]);
-            if (!csync()) break;
-            // O^T: this thread's TMEM lane is head dim tid
-            uint32_t ov[NR / 16][16];
-#pragma unroll
-            for (int c = 0; c < NR / 16; ++c) tmem_ld16(tmem + 128u + (uint32_t)(c * 16) + lane_off, ov[c]);
-            tmem_wait_ld();
+            float *stg = reinterpret_cast<float *>(smem + C::OFF_P);  // [32 rows][128] fp32
             const bool whole = (md.flags & kMetaWhole) != 0;
             const long long wbase = ((long long)md.piece * 2 + md.slot) * NR;
+            bool eok = true;
 #pragma unroll
-            for (int r = 0; r < NR; ++r) {
-                if (r < rreal) {
-                    const float L = a_sh[r];
-                    const float o = __uint_as_float(ov[r >> 4][r & 15]) * (L > 0.f ? 1.f / L : 0.f);
+            for (int h = 0; h < NR; h += 32) {
+                constexpr int RC = NR < 32 ? NR : 32;  // rows per chunk
+                // row sums over the 128 keys: column tid of the table, then one
+                // warp per row
+#pragma unroll
+                for (int r = 0; r < RC; ++r) stg[r * 128 + tid] = l[h + r];
+                if (!(eok = csync())) break;
+#pragma unroll 1
+                for (int r = warp; r < RC; r += tcd::kSoftmaxWarps) {
+                    float v = (stg[r * 128 + lane] + stg[r * 128 + lane + 32]) +
+                              (stg[r * 128 + lane + 64] + stg[r * 128 + lane + 96]);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    if (lane == 0) a_sh[h + r] = v;
+                }
+                if (!(eok = csync())) break;
+                // O^T columns [h, h + RC): this thread's TMEM lane is head dim tid
+                {
+                    uint32_t ov[RC / 16][16];
+#pragma unroll
+                    for (int c = 0; c < RC / 16; ++c)
+                        tmem_ld16(tmem + 128u + (uint32_t)(h + c * 16) + lane_off, ov[c]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int r = 0; r < RC; ++r) stg[r * 128 + tid] = __uint_as_float(ov[r >> 4][r & 15]);
+                }
+                if (!(eok = csync())) break;
+                // one warp per row, four head dims per lane
+                const int rows = rreal - h < RC ? rreal - h : RC;
+#pragma unroll 1
+                for (int r = warp; r < rows; r += tcd::kSoftmaxWarps) {
+                    const float L = a_sh[h + r];
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    const float4 o4 = *reinterpret_cast<const float4 *>(stg + r * 128 + lane * 4);
+                    const float o[4] = {o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv};
                     if (whole) {
-                        if (tid < p.dv) {
-                            const int rg = md.rb * NR + r;
+                        if (lane * 4 < p.dv) {
+                            const int rg = md.rb * NR + h + r;
                             const int hq = md.hkv * p.g + rg / G.Lq, i = rg % G.Lq;
-                            og[md.b * p.o_sb + (long long)(G.q0 + i) * p.o_sl + (long long)hq * p.o_sh + tid] =
-                                from_float<T>(o);
+                            T *dst = og + md.b * p.o_sb + (long long)(G.q0 + i) * p.o_sl + (long long)hq * p.o_sh +
+                                     lane * 4;
+                            *reinterpret_cast<uint2 *>(dst) = make_uint2(Mma<T>::pack(o[0], o[1]), Mma<T>::pack(o[2], o[3]));
                         }
                     } else {
-                        p.ws_o[(wbase + r) * DV + tid] = o;
+                        *reinterpret_cast<float4 *>(p.ws_o + (wbase + h + r) * DV + lane * 4) =
+                            make_float4(o[0], o[1], o[2], o[3]);
                     }
                 }
+                if (!(eok = csync())) break;  // the table is rewritten by the next chunk / segment
             }
-            if (tid < rreal) {
-                const float L = a_sh[tid];
-                const float lse2 = L > 0.f ? m_sh[tid] + log2f(L) : -INFINITY;
+            if (!eok) break;
+#pragma unroll 1
+            for (int r = tid; r < rreal; r += 128) {
+                const float L = a_sh[r];
+                const float lse2 = L > 0.f ? m_sh[r] + log2f(L) : -INFINITY;
                 if (whole) {
                     if (p.lse) {
-                        const int rg = md.rb * NR + tid;
+                        const int rg = md.rb * NR + r;
                         const int hq = md.hkv * p.g + rg / G.Lq, i = rg % G.Lq;
                         p.lse[md.b * p.lse_sb + (long long)hq * p.lse_sh + G.q0 + i] =
                             L > 0.f ? lse2 * 0.69314718055994531f : -INFINITY;
                     }
                 } else {
-                    p.ws_lse[wbase + tid] = lse2;
+                    p.ws_lse[wbase + r] = lse2;
                 }
+            }
+            if constexpr (NR < tcd::kPvN) {
+                // the staging overwrote P^T's zero padding rows: restore this key's
+#pragma unroll
+                for (int c = NR / 8; c < 8; ++c) {
+                    const uint32_t a = prow + ((c ^ (tid & 7)) << 4);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                }
+                fence_proxy_async_smem();
             }
             tc_fence_before();
             __syncwarp();
@@ -492,31 +548,32 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
     }
 }
 
-template <typename T, int DQK, int DV, int NR, int STAGES>
+template <typename T, int DQK, int DV, int NR, int KS, int VS>
 static void fill_tc(KernelInfo *out) {
-    using C = TcCfg<DQK, DV, NR, STAGES>;
-    out->fn = reinterpret_cast<const void *>(&splitkv_tc_kernel<T, DQK, DV, NR, STAGES>);
+    using C = TcCfg<DQK, DV, NR, KS, VS>;
+    out->fn = reinterpret_cast<const void *>(&splitkv_tc_kernel<T, DQK, DV, NR, KS, VS>);
     out->threads = tcd::kThreads;
     out->smem = C::SMEM;
     out->tile_keys = C::TK;
-    out->stages = STAGES;
+    out->stages = VS;
     out->variant = FA_VARIANT_TCGEN05_SPLIT;
     out->rows = NR;
     out->form = 0;
 }
 
+// K slots are released as soon as their S products are done, V slots only
+// after the PV products: two K slots, and as many V slots as fit beside the Q
+// slot and P^T.
 template <typename T>
 static bool fill_tc_dims(int dqk, int nr, KernelInfo *out) {
     if (dqk == 128) {
-        // K + V stages of 64 KB: three fit beside a Q slot of up to 32 rows,
-        // two beside one of 64 rows
-        if (nr == 16) { fill_tc<T, 128, 128, 16, 3>(out); return true; }
-        if (nr == 32) { fill_tc<T, 128, 128, 32, 3>(out); return true; }
-        if (nr == 64) { fill_tc<T, 128, 128, 64, 2>(out); return true; }
+        if (nr == 16) { fill_tc<T, 128, 128, 16, 2, 4>(out); return true; }
+        if (nr == 32) { fill_tc<T, 128, 128, 32, 2, 4>(out); return true; }
+        if (nr == 64) { fill_tc<T, 128, 128, 64, 2, 3>(out); return true; }
     } else if (dqk == 192) {
-        if (nr == 16) { fill_tc<T, 192, 128, 16, 2>(out); return true; }
-        if (nr == 32) { fill_tc<T, 192, 128, 32, 2>(out); return true; }
-        if (nr == 64) { fill_tc<T, 192, 128, 64, 2>(out); return true; }
+        if (nr == 16) { fill_tc<T, 192, 128, 16, 2, 3>(out); return true; }
+        if (nr == 32) { fill_tc<T, 192, 128, 32, 2, 3>(out); return true; }
+        if (nr == 64) { fill_tc<T, 192, 128, 64, 2, 2>(out); return true; }
     }
     return false;
 }

@@ -3,7 +3,9 @@ pipeline stage of the split-KV kernel empty (a barrier phase nothing
 completes) and bounds the call's waits by 20 ms.  The waiting warps give up,
 record FA_ERR_TIMEOUT in the device status word and return; the host reads it
 with check_status, and the next call on the same context runs normally and
-matches the oracle."""
+matches the oracle.  Covered for the mma.sync kernel, its fp32 FMA form and
+the tcgen05 split-KV kernel (whose abort path must also wait for its tensor-core
+work and free its tensor memory before the next call can allocate it)."""
 import time
 
 import pytest
@@ -36,11 +38,14 @@ def _call(variant, w, q, k, v, sl):
     return fa.fa_decode_kvcache(q, k, v, sl.to(DEV), causal=w.causal)
 
 
-@pytest.mark.parametrize("variant", [fa.VARIANT_MMA, fa.VARIANT_SCALAR])
+@pytest.mark.parametrize("variant", [fa.VARIANT_MMA, fa.VARIANT_SCALAR, fa.VARIANT_TCGEN05_SPLIT])
 def test_timeout_is_reported_and_the_context_stays_usable(variant):
     if variant == fa.VARIANT_SCALAR:  # one packed row
         w = wl.Workload("stall_sc", "fwd", "blhd", torch.float16, B=1, Lq=1, Hq=4, Hkv=4, Lk=3000, Dqk=128, Dv=128,
                         causal=False, seed=31)
+    elif variant == fa.VARIANT_TCGEN05_SPLIT:  # 16 packed rows per kv head
+        w = wl.Workload("stall_tc", "kvcache", "blhd", torch.bfloat16, B=6, Lq=4, Hq=8, Hkv=2, Lk=3000, Dqk=128,
+                        Dv=128, causal=True, seed=33, seqlen_lo=1, seqlen_hi=3000)
     else:
         w = wl.Workload("stall_kv", "kvcache", "blhd", torch.bfloat16, B=6, Lq=2, Hq=8, Hkv=2, Lk=3000, Dqk=128,
                         Dv=128, causal=True, seed=32, seqlen_lo=1, seqlen_hi=3000)
