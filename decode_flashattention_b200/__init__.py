@@ -101,7 +101,7 @@ def load_library():
         "fa_profile_enable": (i32, [i32]),
         "fa_profile_read": (i32, [P(ctypes.c_double), P(ctypes.c_int64), P(ctypes.c_double),
                                   P(ctypes.c_int64)]),
-        "fa_schedule": (i32, [i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, P(ctypes.c_int64),
+        "fa_schedule": (i32, [i32, i32, i32, i32, i32, i32, vp, i32, i32, i32, i32, i32, P(ctypes.c_int64),
                               P(ctypes.c_int64), vp, vp, vp, ctypes.c_int64]),
         "fa_launch_count": (ctypes.c_int64, []),
         "fa_version": (ctypes.c_char_p, []),
@@ -432,7 +432,7 @@ def profile_read() -> dict:
 
 
 def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2, tile_keys=128,
-             rows_per_cta=8):
+             rows_per_cta=8, seg_cost=0):
     """Host copy of the kernels' work partition (see fa_schedule in include/fa.h).
     Returns dict(work_tiles, ctas_used, unit_tiles, unit_first_cta, unit_last_cta)."""
     import numpy as np
@@ -447,7 +447,8 @@ def schedule(B, Lq, Hq, Hkv, Lk, causal, seqlens=None, num_ctas=148, min_share=2
     _check(load_library().fa_schedule(
         int(B), int(Lq), int(Hq), int(Hkv), int(Lk), int(bool(causal)),
         ctypes.c_void_p(sl.ctypes.data if sl is not None else None), int(num_ctas), int(min_share),
-        int(tile_keys), int(rows_per_cta), ctypes.byref(W), ctypes.byref(P), ctypes.c_void_p(tiles.ctypes.data),
+        int(tile_keys), int(rows_per_cta), int(seg_cost), ctypes.byref(W), ctypes.byref(P),
+        ctypes.c_void_p(tiles.ctypes.data),
         ctypes.c_void_p(first.ctypes.data), ctypes.c_void_p(last.ctypes.data), units))
     return {"work_tiles": W.value, "ctas_used": P.value, "unit_tiles": tiles,
             "unit_first_cta": first, "unit_last_cta": last}

@@ -34,6 +34,16 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int kDefaultMinShare = 2;
+// K / V bytes of re-reads (mma.sync kernel, blocks of 8 rows) the tcgen05
+// split-KV kernel must save before the library chooses it.
+constexpr int64_t kTcSplitMinSavedBytes = int64_t(128) << 20;
+// Extra partition positions (in tiles) per unit for the tcgen05 split-KV
+// kernel: its segment epilogue and the next segment's first tile take about
+// this many tiles' worth of streaming time.
+#ifndef FA_TC_SEG_COST
+#define FA_TC_SEG_COST 4
+#endif
+constexpr int kTcSegCost = FA_TC_SEG_COST;
 
 thread_local std::string t_err;
 thread_local fa_dispatch_info t_disp = {};
@@ -282,6 +292,7 @@ struct Plan {
     int comb_smem;
     int comb_grid;
     bool prefill = false;  // the tcgen05 kernel: one CTA per (block of 128 rows, kv head, batch), no combine
+    int seg_cost = 0;      // partition positions per unit beyond its tiles
     int row_blocks = 0;
 };
 
@@ -299,14 +310,14 @@ int choose_variant(const Shapes &) {
 // Host copy of the device partition for dense inputs (every batch has Lk keys):
 // returns W and the partition, and whether some unit is cut between pieces
 // or has no tiles (then the combine kernel has work).
-void host_schedule(const Shapes &s, int causal, int tile_shift, int P, int min_share, int *W_out,
+void host_schedule(const Shapes &s, int causal, int tile_shift, int seg_cost, int P, int min_share, int *W_out,
                    fa::Partition *pt_out, bool *need_combine) {
     std::vector<int> pre(s.BR + 1, 0);
     bool empty_unit = false;
     for (int x = 0; x < s.BR; ++x) {
         int t = fa::unit_tiles(s.Lk, x % s.RB, s.R, s.Lq, causal, tile_shift, s.rpc);
         if (t == 0) empty_unit = true;
-        pre[x + 1] = pre[x] + s.Hkv * t;
+        pre[x + 1] = pre[x] + s.Hkv * fa::unit_weight(t, seg_cost);
     }
     const int W = pre[s.BR];
     const fa::Partition pt = fa::make_partition(W, P, min_share);
@@ -318,8 +329,11 @@ void host_schedule(const Shapes &s, int causal, int tile_shift, int P, int min_s
             int mid = (lo + hi + 1) / 2;
             if (pre[mid] <= pos) lo = mid; else hi = mid - 1;
         }
-        const int t = (pre[lo + 1] - pre[lo]) / s.Hkv;
-        if (t > 0 && (pos - pre[lo]) % t != 0) split = true;
+        const int w = (pre[lo + 1] - pre[lo]) / s.Hkv;  // positions per unit of the entry
+        if (w > 0) {
+            const int off = (pos - pre[lo]) % w;  // a boundary strictly inside a unit's tiles splits it
+            if (off > 0 && off < w - seg_cost) split = true;
+        }
     }
     *W_out = W;
     *pt_out = pt;
@@ -381,10 +395,18 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     }
     // More than 8 packed rows (a GQA group with several query positions): the
     // tcgen05 split-KV kernel takes them as one unit of up to 64 rows, so K / V
-    // are streamed once for the whole group instead of once per 8 rows.
+    // are streamed once for the whole group instead of once per 8 rows.  Its
+    // fixed cost per call is higher (measured on GQA-8, qLen 4: 12.5 vs 4.0 us
+    // at 128 keys, 28 vs 20 us at 8K keys, while at 32K keys or batch 4 x 8K
+    // it wins 47 vs 59-67 us and at batch 16 x 8K 117 vs 303 us), so it is
+    // chosen once the re-reads it saves reach kTcSplitMinSavedBytes.
     const bool tcs_dims = s.KDv <= 128 && s.KDqk <= 192;
-    if (variant == FA_VARIANT_MMA && g_force_variant.load() == FA_VARIANT_AUTO && s.R > fa::kRowsPerCta && tcs_dims)
-        variant = FA_VARIANT_TCGEN05_SPLIT;
+    if (variant == FA_VARIANT_MMA && g_force_variant.load() == FA_VARIANT_AUTO && s.R > fa::kRowsPerCta && tcs_dims) {
+        const int nr = s.R <= 16 ? 16 : (s.R <= 32 ? 32 : 64);
+        const int64_t kv = (int64_t)s.B * s.Lk * s.Hkv * (s.Dqk + s.Dv) * 2;  // cache capacity for kvcache calls
+        const int64_t saved = ((int64_t)(s.R + fa::kRowsPerCta - 1) / fa::kRowsPerCta - (s.R + nr - 1) / nr) * kv;
+        if (saved >= kTcSplitMinSavedBytes) variant = FA_VARIANT_TCGEN05_SPLIT;
+    }
     bool ok;
     if (variant == FA_VARIANT_TCGEN05_SPLIT) {
         const int nr = s.R <= 16 ? 16 : (s.R <= 32 ? 32 : 64);
@@ -403,7 +425,8 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
         return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
     if (!ok) return fail(FA_ERR_UNSUPPORTED, "no kernel for variant %d, dtype %d, head dims (%d, %d)", variant,
                          s.dtype, s.Dqk, s.Dv);
-    if (!fa::get_combine_kernel(s.dtype, s.KDv, s.rpc, &pl->comb))
+    const bool comb_unit = fa::combine_per_unit((int64_t)s.B * s.RB * s.Hkv, s.rpc, dev->sms);
+    if (!fa::get_combine_kernel(s.dtype, s.KDv, comb_unit, &pl->comb))
         return fail(FA_ERR_UNSUPPORTED, "no combine kernel for dtype %d, Dv %d", s.dtype, s.KDv);
     if ((st = prepare_fn(pl->main.fn, pl->main.threads, pl->main.smem, &pl->occupancy))) return st;
     pl->comb_smem = 0;
@@ -414,7 +437,11 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     const int tile_shift = log2_exact(TK);
     const int64_t units = (int64_t)s.B * s.RB * s.Hkv;
     // every tile position must fit in 32 bits
-    const int64_t max_tiles = units * (((int64_t)s.Lk + TK - 1) / TK);
+    // the tcgen05 kernel's segment epilogue and the next segment's start cost
+    // about kTcSegCost tiles of streaming: its units are weighted by that much
+    // more in the partition (the mma.sync kernel's by nothing)
+    pl->seg_cost = pl->main.variant == FA_VARIANT_TCGEN05_SPLIT ? kTcSegCost : 0;
+    const int64_t max_tiles = units * (((int64_t)s.Lk + TK - 1) / TK + pl->seg_cost);
     if (max_tiles >= (int64_t(1) << 31) - 1)
         return fail(FA_ERR_UNSUPPORTED, "problem too large: %lld key tiles", (long long)max_tiles);
     int64_t P;
@@ -432,10 +459,10 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
         int W;
         fa::Partition pt;
         bool need;
-        host_schedule(s, causal, tile_shift, (int)P, pl->min_share, &W, &pt, &need);
+        host_schedule(s, causal, tile_shift, pl->seg_cost, (int)P, pl->min_share, &W, &pt, &need);
         if (num_splits <= 0 && W <= P) {  // small problem: one tile per CTA, as many CTAs as tiles
             pl->min_share = 1;
-            host_schedule(s, causal, tile_shift, (int)P, pl->min_share, &W, &pt, &need);
+            host_schedule(s, causal, tile_shift, pl->seg_cost, (int)P, pl->min_share, &W, &pt, &need);
         }
         pl->W = W;
         pl->P = W > 0 ? pt.P : 0;  // W == 0: nothing to stream, the combine writes every row
@@ -458,7 +485,7 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     if (nunits > INT32_MAX || nrows > 4 * (int64_t)INT32_MAX)
         return fail(FA_ERR_UNSUPPORTED, "too many work units (%lld) or rows (%lld)", (long long)nunits,
                     (long long)nrows);
-    pl->comb_grid = fa::combine_grid(nrows, nunits, s.rpc, s.R);
+    pl->comb_grid = fa::combine_grid(nrows, nunits, s.rpc, s.R, comb_unit);
     return FA_OK;
 }
 
@@ -602,6 +629,7 @@ fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor 
     p.min_share = pl.min_share;
     p.tile_keys = pl.main.tile_keys;
     p.tile_shift = log2_exact(pl.main.tile_keys);
+    p.seg_cost = pl.seg_cost;
     p.lse_sb = (int64_t)s.Hq * s.Lq;
     p.lse_sh = s.Lq;
     if (vl) {
@@ -1058,23 +1086,24 @@ fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double *combi
 }
 
 fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens, int num_ctas,
-                      int min_share, int tile_keys, int rows_per_cta, int64_t *work_tiles, int64_t *ctas_used,
-                      int32_t *unit_tiles, int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units) {
+                      int min_share, int tile_keys, int rows_per_cta, int seg_cost, int64_t *work_tiles,
+                      int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta, int64_t *unit_last_cta,
+                      int64_t max_units) {
     if (B < 0 || Lq < 0 || Hq <= 0 || Hkv <= 0 || Lk < 0 || Hq % Hkv || num_ctas < 1 || min_share < 1 ||
         tile_keys < 1 || (tile_keys & (tile_keys - 1)) || max_units < 0 || rows_per_cta < 1 ||
-        rows_per_cta > fa::kMaxRowsPerCta)
+        rows_per_cta > fa::kMaxRowsPerCta || seg_cost < 0 || seg_cost > 1024)
         return fail(FA_ERR_INVALID_ARG, "fa_schedule: inconsistent sizes");
     const int g = Hq / Hkv, R = g * Lq, RB = (R + rows_per_cta - 1) / rows_per_cta;
     const int shift = log2_exact(tile_keys);
     const int64_t BR = (int64_t)B * RB;
-    if (BR * Hkv * (((int64_t)Lk + tile_keys - 1) / tile_keys) >= (int64_t(1) << 31) - 1)
+    if (BR * Hkv * (((int64_t)Lk + tile_keys - 1) / tile_keys + seg_cost) >= (int64_t(1) << 31) - 1)
         return fail(FA_ERR_UNSUPPORTED, "fa_schedule: problem too large");
     std::vector<int> pre(BR + 1, 0);
     std::vector<int32_t> tx(BR, 0);
     for (int64_t x = 0; x < BR; ++x) {
         int n = fa::batch_keys(seqlens, (int)(x / RB), Lk);
         tx[x] = fa::unit_tiles(n, (int)(x % RB), R, Lq, causal, shift, rows_per_cta);
-        pre[x + 1] = pre[x] + Hkv * tx[x];
+        pre[x + 1] = pre[x] + Hkv * fa::unit_weight(tx[x], seg_cost);
     }
     const int W = pre[BR];
     const fa::Partition pt = fa::make_partition(W, num_ctas, min_share);
@@ -1083,7 +1112,7 @@ fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const 
     int64_t u = 0;
     for (int64_t x = 0; x < BR && u < max_units; ++x)
         for (int h = 0; h < Hkv && u < max_units; ++h, ++u) {
-            const int u0 = pre[x] + h * tx[x];
+            const int u0 = pre[x] + h * fa::unit_weight(tx[x], seg_cost);
             if (unit_tiles) unit_tiles[u] = tx[x];
             const bool has = tx[x] > 0;
             if (unit_first_cta) unit_first_cta[u] = has ? fa::piece_of(pt, u0) : -1;

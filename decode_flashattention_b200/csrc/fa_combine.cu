@@ -37,7 +37,7 @@ __host__ __device__ inline int combine_warps_per_unit(int rpc, int R) {
 // row rl of the unit whose tiles start at u0 (slot 0 when the piece starts
 // inside the unit, else slot 1).
 __device__ __forceinline__ long long partial_base(const Params &p, const Partition &pt, int c, int u0, int rl) {
-    return ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * p.rpc + rl;
+    return ((long long)c * 2 + (piece_start(pt, c) >= u0 - p.seg_cost ? 0 : 1)) * p.rpc + rl;
 }
 
 // Merges the np partials (pieces cf .. cf + np - 1) of one output row -- row
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     auto plan = [&]() {
         pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
         t = entry_tiles(p, x);
-        u0 = warp_entry_begin(p, x) + hkv * t;
+        u0 = warp_entry_begin(p, x) + hkv * unit_weight(t, p.seg_cost);
         nparts = 0;
         base0 = 0;
         if (t > 0) {
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kCombineThreads)
             nparts = piece_of(pt, u0 + t - 1) - cf + 1;
             const int c = cf + lane;
             if (lane < PPP && lane < nparts)
-                base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * p.rpc + rr;
+                base0 = ((long long)c * 2 + (piece_start(pt, c) >= u0 - p.seg_cost ? 0 : 1)) * p.rpc + rr;
         }
     };
     if (uniform_batches(p) && live) plan();
@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kCombineThreads)
                 const bool has = lane < PPP && j0 + lane < np;
                 const long long base =
                     j0 == 0 ? b0
-                            : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 ? 0 : 1)) * p.rpc + rr : 0);
+                            : (has ? ((long long)c * 2 + (piece_start(pt, c) >= u0 - p.seg_cost ? 0 : 1)) * p.rpc + rr : 0);
                 const int cnt = np - j0 < PPP ? np - j0 : PPP;
                 const float ls = has ? ws_lse[base] : -INFINITY;
                 float v[PPP][EPL];
@@ -332,7 +332,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     auto plan = [&]() {
         pt = make_partition(warp_total_tiles(p), p.P, p.min_share);
         t = entry_tiles(p, x);
-        u0 = warp_entry_begin(p, x) + hkv * t;
+        u0 = warp_entry_begin(p, x) + hkv * unit_weight(t, p.seg_cost);
         nparts = 0;
         if (t > 0) {
             cf = piece_of(pt, u0);
@@ -370,18 +370,23 @@ __global__ void __launch_bounds__(kCombineThreads)
     }
 }
 
+// Which form: per unit for wide row blocks when the units are many (the
+// per-row form would repeat the partition arithmetic for every row), per row
+// otherwise (few units: their rows merge in parallel).
+bool combine_per_unit(long long units, int rpc, int sms) { return rpc > kRowsPerCta && units >= 2LL * sms; }
+
 // CTAs of the combine kernel: rows / 4 for the per-row form, units / (units
 // per CTA) for the per-unit form.
-int combine_grid(long long rows, long long units, int rpc, int R) {
-    if (rpc <= kRowsPerCta) return (int)((rows + kCombineWarps - 1) / kCombineWarps);
+int combine_grid(long long rows, long long units, int rpc, int R, bool per_unit) {
+    if (!per_unit) return (int)((rows + kCombineWarps - 1) / kCombineWarps);
     const int per_cta = kCombineWarps / combine_warps_per_unit(rpc, R);
     return (int)((units + per_cta - 1) / per_cta);
 }
 
 template <typename T, int DV>
-static void fill(KernelInfo *out, int rpc) {
-    out->fn = rpc <= kRowsPerCta ? reinterpret_cast<const void *>(&combine_rows_kernel<T, DV>)
-                                 : reinterpret_cast<const void *>(&combine_units_kernel<T, DV>);
+static void fill(KernelInfo *out, bool per_unit) {
+    out->fn = per_unit ? reinterpret_cast<const void *>(&combine_units_kernel<T, DV>)
+                       : reinterpret_cast<const void *>(&combine_rows_kernel<T, DV>);
     out->threads = kCombineThreads;
     out->smem = 0;
     out->tile_keys = 0;
@@ -389,15 +394,15 @@ static void fill(KernelInfo *out, int rpc) {
     out->variant = 0;
 }
 
-bool get_combine_kernel(int dtype, int dv, int rpc, KernelInfo *out) {
+bool get_combine_kernel(int dtype, int dv, bool per_unit, KernelInfo *out) {
     if (dtype == 0) {
-        if (dv == 64) { fill<__half, 64>(out, rpc); return true; }
-        if (dv == 128) { fill<__half, 128>(out, rpc); return true; }
-        if (dv == 256) { fill<__half, 256>(out, rpc); return true; }
+        if (dv == 64) { fill<__half, 64>(out, per_unit); return true; }
+        if (dv == 128) { fill<__half, 128>(out, per_unit); return true; }
+        if (dv == 256) { fill<__half, 256>(out, per_unit); return true; }
     } else if (dtype == 1) {
-        if (dv == 64) { fill<__nv_bfloat16, 64>(out, rpc); return true; }
-        if (dv == 128) { fill<__nv_bfloat16, 128>(out, rpc); return true; }
-        if (dv == 256) { fill<__nv_bfloat16, 256>(out, rpc); return true; }
+        if (dv == 64) { fill<__nv_bfloat16, 64>(out, per_unit); return true; }
+        if (dv == 128) { fill<__nv_bfloat16, 128>(out, per_unit); return true; }
+        if (dv == 256) { fill<__nv_bfloat16, 256>(out, per_unit); return true; }
     }
     return false;
 }

@@ -46,6 +46,7 @@ struct Params {
     int W_host;            // total tiles when known on the host (dense inputs), else -1
     int tile_keys;         // keys per tile (TK), a power of two
     int tile_shift;        // log2(tile_keys)
+    int seg_cost;          // positions a unit occupies in the partition beyond its tiles (see below)
     // Paged K/V (block_table non-null): K and V are [num_blocks, page, Hkv, D]
     // and key j of batch b lives in block block_table[b * bt_stride + j / page]
     // at row j % page.
@@ -69,14 +70,19 @@ struct Params {
 
 // ------------------------------------------------------------------ schedule
 // Work is counted in key tiles.  A unit is (batch b, row block rb, kv head
-// hkv); unit u = (b * RB + rb) * Hkv + hkv owns ceil(kmax / TK) tiles, kmax
-// being the number of leading keys any of its rows can see.  The units' tiles
-// are laid end to end (W tiles in total) and cut into P_eff equal contiguous
-// ranges, one per CTA, so every CTA streams the same number of tiles however
-// ragged the per-batch lengths are.  A unit that falls inside one range is
-// finished by that CTA; a unit cut by range boundaries leaves one partial
-// (normalised O and log2-sum-exp) per CTA touching it, in slot 0 if it is the
-// CTA's first segment and slot 1 otherwise, and the combine kernel merges them.
+// hkv); unit u = (b * RB + rb) * Hkv + hkv owns t = ceil(kmax / TK) tiles,
+// kmax being the number of leading keys any of its rows can see.  In the
+// partition a unit with tiles occupies t + seg_cost positions: its tiles, then
+// seg_cost positions that stand for the fixed cost of starting and finishing a
+// unit (0 for the mma.sync kernel, whose segment epilogue is short).  The
+// units' positions are laid end to end (W in total) and cut into P_eff equal
+// contiguous ranges, one per CTA, so every CTA gets the same work however
+// ragged the per-batch lengths are.  A range starting inside a unit's trailing
+// positions begins with the next unit.  A unit whose tiles fall inside one
+// range is finished by that CTA; a unit whose tiles are cut by range
+// boundaries leaves one partial (normalised O and log2-sum-exp) per CTA
+// touching them, in slot 0 if it is the CTA's first segment and slot 1
+// otherwise, and the combine kernel merges them.
 
 __host__ __device__ inline int keys_visible_to_block(int n, int rb, int R, int Lq, int causal, int rpc) {
     if (n <= 0 || rb * rpc >= R) return 0;  // no keys, or a row block past the batch's rows
@@ -334,13 +340,14 @@ struct Mma<__nv_bfloat16> {
     }
 };
 
-// 16-bit element(s) to fp32 (exact).
+// 16-bit element(s) to fp32 (exact), and fp32 to 16-bit (round to nearest even).
 template <typename T>
 struct Cvt;
 
 template <>
 struct Cvt<__half> {
     __device__ __forceinline__ static float f1(__half x) { return __half2float(x); }
+    __device__ __forceinline__ static __half from(float x) { return __float2half_rn(x); }
     __device__ __forceinline__ static float2 f2(uint32_t x) {
         return __half22float2(*reinterpret_cast<const __half2 *>(&x));
     }
@@ -349,6 +356,7 @@ struct Cvt<__half> {
 template <>
 struct Cvt<__nv_bfloat16> {
     __device__ __forceinline__ static float f1(__nv_bfloat16 x) { return __bfloat162float(x); }
+    __device__ __forceinline__ static __nv_bfloat16 from(float x) { return __float2bfloat16_rn(x); }
     __device__ __forceinline__ static float2 f2(uint32_t x) {
         return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x));
     }
@@ -440,17 +448,20 @@ __device__ __forceinline__ int entry_tiles(const Params &p, int x) {
     return unit_tiles(G.n, rb, G.R, G.Lq, p.causal, p.tile_shift, p.rpc);
 }
 
+// Partition positions of one unit with t tiles.
+__host__ __device__ __forceinline__ int unit_weight(int t, int seg_cost) { return t > 0 ? t + seg_cost : 0; }
+
 __device__ __forceinline__ int warp_sum(int v) {
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
     return v;
 }
 
-// Tiles of all units of entries [x0, x1), counted Hkv times (one per kv head).
+// Positions of all units of entries [x0, x1), counted Hkv times (one per kv head).
 __device__ __forceinline__ int warp_entry_tiles(const Params &p, int x0, int x1) {
     const int lane = threadIdx.x & 31;
     int acc = 0;
-    for (int x = x0 + lane; x < x1; x += 32) acc += entry_tiles(p, x);
+    for (int x = x0 + lane; x < x1; x += 32) acc += unit_weight(entry_tiles(p, x), p.seg_cost);
     return warp_sum(acc) * p.Hkv;
 }
 
@@ -458,14 +469,14 @@ __device__ __forceinline__ int warp_entry_tiles(const Params &p, int x0, int x1)
 // and the schedule needs no memory reads.
 __device__ __forceinline__ bool uniform_batches(const Params &p) { return !p.seqlens && !p.cu_q; }
 
-// Total tiles W.
+// Total positions W.
 __device__ __forceinline__ int warp_total_tiles(const Params &p) {
     if (p.W_host >= 0) return p.W_host;
     if (uniform_batches(p)) return warp_entry_tiles(p, 0, p.RB) * p.B;
     return warp_entry_tiles(p, 0, p.B * p.RB);
 }
 
-// First tile position of entry x's units.
+// First position of entry x's units.
 __device__ __forceinline__ int warp_entry_begin(const Params &p, int x) {
     if (uniform_batches(p)) {
         const int b = x / p.RB;
@@ -474,7 +485,7 @@ __device__ __forceinline__ int warp_entry_begin(const Params &p, int x) {
     return warp_entry_tiles(p, 0, x);
 }
 
-// Entry x holding tile position t (0 <= t < W); *x_begin receives the first
+// Entry x holding position t (0 <= t < W); *x_begin receives the first
 // position of x's units.
 __device__ __forceinline__ int warp_locate(const Params &p, int t, int *x_begin) {
     const int lane = threadIdx.x & 31;
@@ -488,7 +499,7 @@ __device__ __forceinline__ int warp_locate(const Params &p, int t, int *x_begin)
     }
     for (int c0 = x_lo; c0 < x_hi; c0 += 32) {
         const int x = c0 + lane;
-        const int tt = x < x_hi ? entry_tiles(p, x) * p.Hkv : 0;
+        const int tt = x < x_hi ? unit_weight(entry_tiles(p, x), p.seg_cost) * p.Hkv : 0;
         int incl = tt;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -508,12 +519,13 @@ __device__ __forceinline__ int warp_locate(const Params &p, int t, int *x_begin)
     return x_hi - 1;
 }
 
-// Walks the segments of one CTA's tile range [start, end): each segment is a
-// run of tiles of one unit.  Producer and consumers step identical copies.
+// Walks the segments of one CTA's range [start, end) of positions: each
+// segment is a run of tiles of one unit.  Producer and consumers step
+// identical copies.
 struct SegmentWalker {
     int x, hkv;   // current (b*RB + rb) entry and kv head
-    int u0;       // first tile position of the current unit
-    int t;        // tiles of the current unit
+    int u0;       // first position of the current unit (its first tile)
+    int t, w;     // tiles and positions of the current unit
     int pos, start, end;
 
     // Must be called by all 32 lanes of a warp (uses warp collectives).
@@ -524,29 +536,36 @@ struct SegmentWalker {
         int xb = 0;
         x = warp_locate(p, s, &xb);
         t = entry_tiles(p, x);
-        hkv = (s - xb) / t;
-        u0 = xb + hkv * t;
+        w = unit_weight(t, p.seg_cost);
+        hkv = (s - xb) / w;
+        u0 = xb + hkv * w;
+        // a range starting in a unit's trailing positions begins with the next unit
+        if (pos >= u0 + t) advance(p);
     }
     __device__ __forceinline__ bool done() const { return pos >= end; }
     __device__ __forceinline__ int b(const Params &p) const { return x / p.RB; }
     __device__ __forceinline__ int rb(const Params &p) const { return x % p.RB; }
+    // end (position) of the current segment's tiles
     __device__ __forceinline__ int seg_end() const {
         const int ue = u0 + t;
         return ue < end ? ue : end;
     }
-    // Move past the current segment.
+    // whether the current segment is the range's last (the next unit starts at
+    // or past the range's end)
+    __device__ __forceinline__ bool last_segment() const { return u0 + w >= end; }
+    // Move past the current unit.
     __device__ __forceinline__ void advance(const Params &p) {
-        pos = seg_end();
+        pos = u0 + w;
         if (pos >= end) return;
-        // pos is now the end of the current unit: step to the next unit with tiles
-        u0 += t;
+        u0 += w;
         if (++hkv < p.Hkv) return;
         hkv = 0;
         const int BR = p.B * p.RB;
         for (;;) {
             ++x;
-            if (x >= BR) { t = 1; return; }  // unreachable while pos < end
+            if (x >= BR) { t = 1; w = 1; return; }  // unreachable while pos < end
             t = entry_tiles(p, x);
+            w = unit_weight(t, p.seg_cost);
             if (t > 0) return;
         }
     }

@@ -19,10 +19,12 @@ struct KernelInfo {
 
 // Main split-KV kernel using mma.sync (keys as M, packed rows as N).
 bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
-// LSE-weighted combine of split partials for row blocks of rpc rows, and its
-// grid for `rows` output rows in `units` units (R packed rows per kv head).
-bool get_combine_kernel(int dtype, int dv, int rpc, KernelInfo *out);
-int combine_grid(long long rows, long long units, int rpc, int R);
+// LSE-weighted combine of split partials (per-row or per-unit form), the
+// choice of form for `units` units of row blocks of rpc rows on `sms` SMs, and
+// its grid for `rows` output rows (R packed rows per kv head).
+bool get_combine_kernel(int dtype, int dv, bool per_unit, KernelInfo *out);
+bool combine_per_unit(long long units, int rpc, int sms);
+int combine_grid(long long rows, long long units, int rpc, int R, bool per_unit);
 
 // Dense attention on tcgen05 for calls with many packed rows (fa_prefill.cu).
 // form: an fa_tcgen05_form other than FA_TCGEN05_AUTO.

@@ -258,13 +258,12 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
     };
     int it = 0, itv = 0, seg = 0;  // tiles whose K (joint: K and V) / separate V were issued
     bool stop = !active;
-    const int lo = active ? wk.start : 0, hi = active ? wk.end : 0;
     for (; active && !wk.done() && !stop; wk.advance(p), ++seg) {
         const int b = wk.b(p), rb = wk.rb(p), hkv = wk.hkv;
         const BatchGeom G = batch_geom(p, b);
         const int t0 = wk.pos - wk.u0, t1 = wk.seg_end() - wk.u0;
         const bool whole = (wk.pos == wk.u0) && (wk.seg_end() == wk.u0 + wk.t);
-        const int slot = (wk.pos == lo) ? 0 : 1;
+        const int slot = seg == 0 ? 0 : 1;  // partial slot: the CTA's first segment, or a later one
         for (int tt = t0; tt < t1 && !stop; ++tt, ++it) {
             const int s = it % KS, use = it / KS;
             // test hook: the first CTA leaves its first tile's slots empty (no
@@ -281,33 +280,37 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
             const uint32_t kdst = R.k_base + s * R.k_stride;
             // (one piece per CTA: the piece's last tile is the CTA's last tile)
             const int flags = (tt == t0 ? kMetaFirst : 0) | (tt == t1 - 1 ? kMetaLast : 0) |
-                              (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.seg_end() == hi ? kMetaFinal : 0);
+                              (whole ? kMetaWhole : 0) | (tt == t1 - 1 && wk.last_segment() ? kMetaFinal : 0);
             const int j = tt * C::TK;
             issue(true, kJoint, kdst, R.v_base + s * R.v_stride, kfull(s), b, hkv, G, j);
+            // separate rings: V's copy goes out too before the query rows are
+            // staged (a synchronous copy at a segment's first tile)
+            int vs = 0;
+            bool vok = true;
+            if constexpr (!kJoint) {
+                const int vuse = itv / VS;
+                vs = itv % VS;
+                vok = vuse == 0 || mbar_wait(vempty(vs), (vuse - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
+                vok = __all_sync(0xffffffffu, vok);
+                if (vok) issue(false, true, 0u, R.v_base + vs * R.v_stride, vfull(vs), b, hkv, G, j);
+            }
             if (lane == 0) {
                 StageMeta m = {b, rb, hkv, tt, flags, cta, slot, 0};
                 meta[kJoint ? s : it % kMetaRing] = m;
             }
-            const bool qok = !(flags & kMetaFirst) || __all_sync(0xffffffffu, q_write(s, seg, b, rb, hkv, G));
+            const bool qok = vok && (!(flags & kMetaFirst) || __all_sync(0xffffffffu, q_write(s, seg, b, rb, hkv, G)));
             __syncwarp();
             if (lane == 0) mbar_arrive(kfull(s));
-            if (!qok) {  // a wait gave up (the CTA is aborting): the slot still completes, then stop
+            if constexpr (!kJoint) {
+                if (vok) {
+                    if (lane == 0) mbar_arrive(vfull(vs));
+                    ++itv;
+                }
+            }
+            if (!qok) {  // a wait gave up (the CTA is aborting): the slots still complete, then stop
                 stop = true;
                 ++it;
                 break;
-            }
-            if constexpr (!kJoint) {
-                const int vs = itv % VS, vuse = itv / VS;
-                ok = vuse == 0 || mbar_wait(vempty(vs), (vuse - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    stop = true;
-                    ++it;
-                    break;
-                }
-                issue(false, true, 0u, R.v_base + vs * R.v_stride, vfull(vs), b, hkv, G, j);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(vfull(vs));
-                ++itv;
             }
         }
     }

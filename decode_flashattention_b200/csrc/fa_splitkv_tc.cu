@@ -80,8 +80,10 @@ struct TcCfg {
     static constexpr int OFF_M = (OFF_MISC + 48 + 15) & ~15;        // running max per row [NR]
     static constexpr int OFF_A = OFF_M + NR * 4;                    // rescale factors / row sums [NR]
     static constexpr int OFF_LIM = OFF_A + NR * 4;                  // last visible key per row [NR]
-    static constexpr int OFF_RED = OFF_LIM + NR * 4;                // per-warp row maxima [4][NR]
-    static constexpr int SMEM_USED = OFF_RED + 4 * NR * 4;
+    static constexpr int OFF_RED = OFF_LIM + NR * 4;                // per-warp row maxima / sums [4][NR]
+    static constexpr int OFF_OOFF = OFF_RED + 4 * NR * 4;           // output row offsets [NR] (elements)
+    static constexpr int OFF_LOFF = OFF_OOFF + NR * 8;              // lse offsets [NR] (-1: none)
+    static constexpr int SMEM_USED = OFF_LOFF + NR * 8;
     // the dynamic shared memory base is at least 16-byte aligned, so 1008
     // bytes of slack always reach the next 1024-byte boundary
     static constexpr int SMEM = SMEM_USED + 1008;
@@ -98,6 +100,25 @@ __device__ __forceinline__ float warp_max_f32(float v) {
     float r;
     asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
     return r;
+}
+
+// Row sums of 32 rows over the warp's 32 lanes (v[r]: this lane's part of row
+// r; v is consumed): a reduce-scatter butterfly -- at each step a lane keeps
+// one half of its rows and adds its partner's copy of that half -- after
+// which lane r holds the warp's sum of row r.  31 shuffles for 32 rows.
+__device__ __forceinline__ float warp_row_sums32(float (&v)[32]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int half = 16; half >= 1; half >>= 1) {
+        const bool up = (lane & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = up ? v[i] : v[i + half];
+            const float keep = up ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return v[0];
 }
 
 template <typename T, int DQK, int DV, int NR, int KS, int VS>
@@ -134,6 +155,8 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
     float *a_sh = reinterpret_cast<float *>(smem + C::OFF_A);
     int *lim_sh = reinterpret_cast<int *>(smem + C::OFF_LIM);
     float *red_sh = reinterpret_cast<float *>(smem + C::OFF_RED);
+    long long *ooff_sh = reinterpret_cast<long long *>(smem + C::OFF_OOFF);
+    long long *loff_sh = reinterpret_cast<long long *>(smem + C::OFF_LOFF);
 
     if (tid == 0) {
         for (int s = 0; s < KS; ++s) {
@@ -312,14 +335,20 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
                 if (tid < NR) {
                     int lim = -1;
                     float m0 = tcd::kPadMax;
+                    long long oo = 0, lo = -1;
                     if (tid < rreal) {
-                        const int i = (md.rb * NR + tid) % G.Lq;
+                        const int rg = md.rb * NR + tid;
+                        const int i = rg % G.Lq, hq = md.hkv * p.g + rg / G.Lq;
                         lim = G.n - 1;
                         if (p.causal && i + G.n - G.Lq < lim) lim = i + G.n - G.Lq;
                         m0 = -INFINITY;
+                        oo = md.b * p.o_sb + (long long)(G.q0 + i) * p.o_sl + (long long)hq * p.o_sh;
+                        if (p.lse) lo = md.b * p.lse_sb + (long long)hq * p.lse_sh + G.q0 + i;
                     }
                     lim_sh[tid] = lim;
                     m_sh[tid] = m0;
+                    ooff_sh[tid] = oo;
+                    loff_sh[tid] = lo;
                 }
 #pragma unroll
                 for (int r = 0; r < NR; ++r) l[r] = 0.f;
@@ -444,93 +473,54 @@ __global__ void __launch_bounds__(tcd::kThreads, 1)
             if (!(md.flags & kMetaLast)) continue;
 
             // ================================================ segment epilogue
-            // The last PV is done, so the P^T buffer is free until this warp
-            // group writes the next segment's first P: it stages the row sums
-            // and O (32 rows at a time), which lets every loop over rows stay
-            // rolled -- the epilogue runs once per segment and its code would
-            // otherwise be fetched cold each time.
-            ok = mbar_wait(pdone, it & 1, abort_flag, p.status, p.wait_limit_ns);
+            // Row sums over the 128 keys (a reduce-scatter butterfly per warp,
+            // then the four warps' sums), then O^T read from TMEM -- this
+            // thread's lane is head dim tid, so each row of O is written by
+            // 128 consecutive threads -- scaled by 1 / sum; row offsets were
+            // worked out at the segment's start.
+            ok = mbar_wait(pdone, it & 1, abort_flag, p.status, p.wait_limit_ns);  // the last PV
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            float *stg = reinterpret_cast<float *>(smem + C::OFF_P);  // [32 rows][128] fp32
-            const bool whole = (md.flags & kMetaWhole) != 0;
-            const long long wbase = ((long long)md.piece * 2 + md.slot) * NR;
-            bool eok = true;
 #pragma unroll
             for (int h = 0; h < NR; h += 32) {
-                constexpr int RC = NR < 32 ? NR : 32;  // rows per chunk
-                // row sums over the 128 keys: column tid of the table, then one
-                // warp per row
+                float v[32];
 #pragma unroll
-                for (int r = 0; r < RC; ++r) stg[r * 128 + tid] = l[h + r];
-                if (!(eok = csync())) break;
-#pragma unroll 1
-                for (int r = warp; r < RC; r += tcd::kSoftmaxWarps) {
-                    float v = (stg[r * 128 + lane] + stg[r * 128 + lane + 32]) +
-                              (stg[r * 128 + lane + 64] + stg[r * 128 + lane + 96]);
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                    if (lane == 0) a_sh[h + r] = v;
-                }
-                if (!(eok = csync())) break;
-                // O^T columns [h, h + RC): this thread's TMEM lane is head dim tid
-                {
-                    uint32_t ov[RC / 16][16];
-#pragma unroll
-                    for (int c = 0; c < RC / 16; ++c)
-                        tmem_ld16(tmem + 128u + (uint32_t)(h + c * 16) + lane_off, ov[c]);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int r = 0; r < RC; ++r) stg[r * 128 + tid] = __uint_as_float(ov[r >> 4][r & 15]);
-                }
-                if (!(eok = csync())) break;
-                // one warp per row, four head dims per lane
-                const int rows = rreal - h < RC ? rreal - h : RC;
-#pragma unroll 1
-                for (int r = warp; r < rows; r += tcd::kSoftmaxWarps) {
-                    const float L = a_sh[h + r];
-                    const float inv = L > 0.f ? 1.f / L : 0.f;
-                    const float4 o4 = *reinterpret_cast<const float4 *>(stg + r * 128 + lane * 4);
-                    const float o[4] = {o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv};
-                    if (whole) {
-                        if (lane * 4 < p.dv) {
-                            const int rg = md.rb * NR + h + r;
-                            const int hq = md.hkv * p.g + rg / G.Lq, i = rg % G.Lq;
-                            T *dst = og + md.b * p.o_sb + (long long)(G.q0 + i) * p.o_sl + (long long)hq * p.o_sh +
-                                     lane * 4;
-                            *reinterpret_cast<uint2 *>(dst) = make_uint2(Mma<T>::pack(o[0], o[1]), Mma<T>::pack(o[2], o[3]));
-                        }
-                    } else {
-                        *reinterpret_cast<float4 *>(p.ws_o + (wbase + h + r) * DV + lane * 4) =
-                            make_float4(o[0], o[1], o[2], o[3]);
-                    }
-                }
-                if (!(eok = csync())) break;  // the table is rewritten by the next chunk / segment
+                for (int r = 0; r < 32; ++r) v[r] = h + r < NR ? l[h + r] : 0.f;
+                const float rs = warp_row_sums32(v);
+                if (h + lane < NR) red_sh[warp * NR + h + lane] = rs;
             }
-            if (!eok) break;
-#pragma unroll 1
-            for (int r = tid; r < rreal; r += 128) {
-                const float L = a_sh[r];
-                const float lse2 = L > 0.f ? m_sh[r] + log2f(L) : -INFINITY;
+            if (!csync()) break;
+            const bool whole = (md.flags & kMetaWhole) != 0;
+            const long long wbase = ((long long)md.piece * 2 + md.slot) * NR;
+            if (tid < rreal) {
+                const float L = (red_sh[tid] + red_sh[NR + tid]) + (red_sh[2 * NR + tid] + red_sh[3 * NR + tid]);
+                a_sh[tid] = L > 0.f ? 1.f / L : 0.f;
+                const float lse2 = L > 0.f ? m_sh[tid] + log2f(L) : -INFINITY;
                 if (whole) {
-                    if (p.lse) {
-                        const int rg = md.rb * NR + r;
-                        const int hq = md.hkv * p.g + rg / G.Lq, i = rg % G.Lq;
-                        p.lse[md.b * p.lse_sb + (long long)hq * p.lse_sh + G.q0 + i] =
-                            L > 0.f ? lse2 * 0.69314718055994531f : -INFINITY;
+                    if (loff_sh[tid] >= 0) p.lse[loff_sh[tid]] = L > 0.f ? lse2 * 0.69314718055994531f : -INFINITY;
+                } else {
+                    p.ws_lse[wbase + tid] = lse2;
+                }
+            }
+            if (!csync()) break;
+#pragma unroll
+            for (int c = 0; c < NR / 16; ++c) {  // 16 rows (TMEM columns) at a time
+                uint32_t ov[16];
+                tmem_ld16(tmem + 128u + (uint32_t)(c * 16) + lane_off, ov);
+                tmem_wait_ld();
+                if (whole) {
+                    if (tid < p.dv) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c * 16 + e < rreal)
+                                og[ooff_sh[c * 16 + e] + tid] = Cvt<T>::from(__uint_as_float(ov[e]) * a_sh[c * 16 + e]);
                     }
                 } else {
-                    p.ws_lse[wbase + r] = lse2;
-                }
-            }
-            if constexpr (NR < tcd::kPvN) {
-                // the staging overwrote P^T's zero padding rows: restore this key's
 #pragma unroll
-                for (int c = NR / 8; c < 8; ++c) {
-                    const uint32_t a = prow + ((c ^ (tid & 7)) << 4);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+                    for (int e = 0; e < 16; ++e)
+                        if (c * 16 + e < rreal)
+                            p.ws_o[(wbase + c * 16 + e) * DV + tid] = __uint_as_float(ov[e]) * a_sh[c * 16 + e];
                 }
-                fence_proxy_async_smem();
             }
             tc_fence_before();
             __syncwarp();

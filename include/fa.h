@@ -339,7 +339,10 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
  * least 128 packed rows (g * Lq >= 128) and head dims 64/64 or 128/128
  * (prefill-shaped calls); FA_VARIANT_TCGEN05_SPLIT for more than 8 packed
- * rows (g * Lq > 8) with Dqk <= 192 and Dv <= 128; FA_VARIANT_MMA otherwise --
+ * rows (g * Lq > 8) with Dqk <= 192 and Dv <= 128 once the K / V re-reads it
+ * saves over blocks of 8 rows reach 128 MB (B * Lk * Hkv * (Dqk + Dv) * 2
+ * bytes per block, Lk the cache capacity for the kvcache calls: below that its
+ * higher fixed cost per call loses); FA_VARIANT_MMA otherwise --
  * measured on B200 it is faster than the FMA variant even for one packed row.
  * A forced variant that does not support the call's shapes makes the call
  * fail with FA_ERR_UNSUPPORTED.
@@ -407,20 +410,24 @@ FA_API fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double
  * of `rows_per_cta` packed query rows, kv head) -- 8 for the mma.sync
  * split-KV kernel, 16 / 32 / 64 for the tcgen05 one (fa_last_dispatch's
  * rows_per_cta says which a call used) -- ordered batch-major, then row
- * block, then kv head, and owns ceil(visible keys / tile_keys) tiles.  The W
- * tiles of all units are laid end to end and cut into ctas_used =
- * min(num_ctas, ceil(W / min_share)) contiguous pieces, one per CTA, whose
- * sizes differ by at most one tile (the first W mod ctas_used pieces are the
- * longer ones).  seqlens: HOST int32 [B] (NULL: every batch has Lk keys).
- * For each of the first max_units units the call writes its tile count and
- * the first and last CTA whose piece holds its tiles (-1, -1 for a unit with
- * no tiles).  FA_ERR_INVALID_ARG for inconsistent sizes (rows_per_cta must
- * be in [1, 64]).
+ * block, then kv head, and owns t = ceil(visible keys / tile_keys) tiles.  In
+ * the partition a unit with t > 0 tiles occupies t + seg_cost positions (its
+ * tiles first; seg_cost stands for the fixed cost of a unit: 0 for the
+ * mma.sync kernel, 4 for the tcgen05 one).  The W positions of all units are
+ * laid end to end and cut into ctas_used = min(num_ctas, ceil(W / min_share))
+ * contiguous pieces, one per CTA, whose sizes differ by at most one position
+ * (the first W mod ctas_used pieces are the longer ones); a piece that starts
+ * in a unit's trailing positions starts with the next unit.  seqlens: HOST
+ * int32 [B] (NULL: every batch has Lk keys).  For each of the first max_units
+ * units the call writes its tile count and the first and last CTA whose piece
+ * holds its tiles (-1, -1 for a unit with no tiles).  FA_ERR_INVALID_ARG for
+ * inconsistent sizes (rows_per_cta must be in [1, 64], seg_cost in
+ * [0, 1024]).
  */
 FA_API fa_status fa_schedule(int B, int Lq, int Hq, int Hkv, int Lk, int causal, const int32_t *seqlens,
-                             int num_ctas, int min_share, int tile_keys, int rows_per_cta, int64_t *work_tiles,
-                             int64_t *ctas_used, int32_t *unit_tiles, int64_t *unit_first_cta,
-                             int64_t *unit_last_cta, int64_t max_units);
+                             int num_ctas, int min_share, int tile_keys, int rows_per_cta, int seg_cost,
+                             int64_t *work_tiles, int64_t *ctas_used, int32_t *unit_tiles,
+                             int64_t *unit_first_cta, int64_t *unit_last_cta, int64_t max_units);
 
 /* Kernels launched by this library in this process (both kinds). */
 FA_API int64_t fa_launch_count(void);

@@ -186,13 +186,14 @@ CASES = [
 
 @pytest.mark.parametrize("c", CASES, ids=range(len(CASES)))
 @pytest.mark.parametrize("min_share", [1, 2, 5])
-@pytest.mark.parametrize("rpc", [8, 16, 64])
-def test_schedule_covers_balances_and_bounds_partials(c, min_share, rpc):
+@pytest.mark.parametrize("rpc,seg_cost", [(8, 0), (16, 4), (64, 0), (32, 4), (8, 3)])
+def test_schedule_covers_balances_and_bounds_partials(c, min_share, rpc, seg_cost):
     c = dict(c)
     if c["seqlens"] == "rand":
         c["seqlens"] = np.random.default_rng(3).integers(1, c["Lk"] + 1, c["B"]).astype(np.int32)
     s = fa.schedule(c["B"], c["Lq"], c["Hq"], c["Hkv"], c["Lk"], c["causal"], c["seqlens"],
-                    num_ctas=c["num_ctas"], min_share=min_share, tile_keys=128, rows_per_cta=rpc)
+                    num_ctas=c["num_ctas"], min_share=min_share, tile_keys=128, rows_per_cta=rpc,
+                    seg_cost=seg_cost)
     g = c["Hq"] // c["Hkv"]
     R = g * c["Lq"]
     RB = (R + rpc - 1) // rpc
@@ -203,14 +204,15 @@ def test_schedule_covers_balances_and_bounds_partials(c, min_share, rpc):
             want += [visible_tiles(n, rb, R, c["Lq"], c["causal"], rpc=rpc)] * c["Hkv"]
     tiles = s["unit_tiles"]
     assert tiles.tolist() == want
-    W = int(tiles.sum())
+    # a unit with tiles occupies its tiles, then seg_cost trailing positions
+    W = int(tiles.sum()) + seg_cost * int((tiles > 0).sum())
     assert s["work_tiles"] == W
     P = s["ctas_used"]
     assert P == max(1, min(c["num_ctas"], math.ceil(W / min_share)))
     if W == 0:
         assert np.all(s["unit_first_cta"] == -1)
         return
-    # P contiguous pieces; the first W % P are one tile longer
+    # P contiguous pieces; the first W % P are one position longer
     share, rem = divmod(W, P)
     starts = [cc * share + min(cc, rem) for cc in range(P)] + [W]
     sizes = np.diff(starts)
@@ -222,10 +224,10 @@ def test_schedule_covers_balances_and_bounds_partials(c, min_share, rpc):
     for t, f, l in zip(tiles[has], first, last):
         assert starts[f] <= pos < starts[f + 1]
         assert starts[l] <= pos + int(t) - 1 < starts[l + 1]
-        pos += int(t)
+        pos += int(t) + seg_cost
     assert pos == W
     assert np.all(np.diff(first) >= 0) and np.all(np.diff(last) >= 0)
-    assert first[0] == 0 and last[-1] == P - 1
+    assert first[0] == 0 and (last[-1] == P - 1 or seg_cost > 0)
     # a piece holds at most two partial units (its first and its last segment)
     partial_count = np.zeros(P, dtype=int)
     for f, l in zip(first, last):

@@ -3,7 +3,8 @@
 Each case draws a call (dense, kvcache, paged, append or varlen), head dims
 (the compiled kernels' and others that run zero-padded on them),
 element type, GQA ratio, query length 1-8, causal flag, split count and
-variant, with ragged lengths, and compares the result with the oracle
+variant (the library's choice, the fp32 FMA form for one packed row, or the
+tcgen05 split-KV kernel for more than 8), with ragged lengths, and compares the result with the oracle
 element by element.  The draws are fixed by the seed, so a failure names a
 reproducible case."""
 import numpy as np
@@ -42,6 +43,11 @@ def _draw(i):
     splits = int(r.choice([0, 0, 1, 2, 9]))
     variant = fa.VARIANT_SCALAR if (g * lq == 1 and not _runs_on_256(d) and r.random() < 0.5) else fa.VARIANT_AUTO
     page = int(r.choice([16, 32, 64, 128, 256]))
+    # more than 8 packed rows: half the cases forced onto the tcgen05 split-KV
+    # kernel (at these sizes the library itself keeps the 8-row blocks)
+    fits_tc = (d[1] <= 128 and d[0] <= 192) if not _runs_on_256(d) else False
+    if g * lq > 8 and fits_tc and r.random() < 0.5:
+        variant = fa.VARIANT_TCGEN05_SPLIT
     return call, d, dt, Hkv, g, lq, B, lk, causal, splits, variant, page, r
 
 

@@ -114,20 +114,21 @@ def test_scalar_variant(d):
 
 def test_prefill_shaped_call_on_the_split_kernel():
     # 256 packed rows with head dim 96: not a tcgen05 prefill shape, the split-KV kernel takes it
-    # (on the tensor cores, in row blocks of 64)
+    # (8-row blocks at this size; forced, the tcgen05 split-KV kernel's row blocks of 64)
     w = wl.Workload("hd_pf", "fwd", "blhd", torch.bfloat16, B=1, Lq=64, Hq=8, Hkv=2, Lk=500, Dqk=96, Dv=96,
                     causal=True, seed=77)
     q, k, v, _ = wl.make_inputs(w, DEV)
     o, lse = fa.fa_fwd(q, k, v, causal=True)
     torch.cuda.synchronize()
-    assert fa.last_dispatch()["variant"] == fa.VARIANT_TCGEN05_SPLIT
+    assert fa.last_dispatch()["variant"] == fa.VARIANT_MMA
     ro, rl = oracle_full(q, k, v, True)
     compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, torch.bfloat16, "prefill-shaped hd 96")
-    fa.force_variant(fa.VARIANT_MMA)  # and on the mma.sync kernel's 8-row blocks
+    fa.force_variant(fa.VARIANT_TCGEN05_SPLIT)  # and on the tcgen05 split-KV kernel's 64-row blocks
     o, lse = fa.fa_fwd(q, k, v, causal=True)
     torch.cuda.synchronize()
+    assert fa.last_dispatch()["rows_per_cta"] == 64
     fa.force_variant(fa.VARIANT_AUTO)
-    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, torch.bfloat16, "prefill-shaped hd 96, mma.sync")
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, torch.bfloat16, "prefill-shaped hd 96, tcgen05 split")
 
 
 def test_instance_dims_in_dispatch():

@@ -114,8 +114,8 @@ def test_automatic_kernel_and_form_choice():
             ((4, 32, 32, 8, 128), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),  # 128 rows, 32 CTAs
             ((4, 32, 32, 8, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)),   # the same with 64-dim heads
             ((1, 300, 16, 16, 64), (fa.VARIANT_TCGEN05, fa.TCGEN05_ONE_TILE_MMA)), # 64-dim heads: no serial form
-            ((2, 32, 32, 8, 128), (fa.VARIANT_TCGEN05_SPLIT, 0)),                  # 16 CTAs: split-KV kernel
-            ((1, 32, 8, 2, 64), (fa.VARIANT_TCGEN05_SPLIT, 0))):                   # 2 CTAs (the 64-key prefill)
+            ((2, 32, 32, 8, 128), (fa.VARIANT_MMA, 0)),                            # 16 CTAs: split-KV kernel
+            ((1, 32, 8, 2, 64), (fa.VARIANT_MMA, 0))):                             # 2 CTAs (the 64-key prefill)
         if form == fa.TCGEN05_TWO_TILES:
             assert ((Lq * Hq // Hkv + 255) // 256) * Hkv * B >= sms
         q = torch.zeros(B, Lq, Hq, D, dtype=torch.bfloat16, device=DEV)

@@ -30,8 +30,10 @@ DEV = "cuda"
 
 
 @pytest.fixture(autouse=True)
-def _auto_variant():
-    fa.force_variant(fa.VARIANT_AUTO)
+def _tc_variant():
+    # the shapes here are small, where the library itself would choose the
+    # mma.sync kernel: force the tcgen05 split-KV kernel
+    fa.force_variant(fa.VARIANT_TCGEN05_SPLIT)
     yield
     fa.force_variant(fa.VARIANT_AUTO)
     torch.cuda.synchronize()
@@ -182,11 +184,27 @@ def test_determinism_bitwise():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+def test_automatic_choice():
+    """The library's own choice: 8-row blocks while the re-reads they cost
+    stay small, the tcgen05 split-KV kernel from 128 MB of saved re-reads."""
+    fa.force_variant(fa.VARIANT_AUTO)
+    for (B, Lk, Hkv, g, lq), want in (((1, 128, 2, 4, 32), fa.VARIANT_MMA),       # 64 KB of K/V (C1's shape)
+                                      ((1, 8192, 8, 8, 4), fa.VARIANT_MMA),       # 33.5 MB, 3x re-read
+                                      ((4, 8192, 8, 8, 4), fa.VARIANT_TCGEN05_SPLIT),  # 134 MB, 3x re-read
+                                      ((1, 8192, 8, 8, 1), fa.VARIANT_MMA)):      # 8 rows: one block
+        q = torch.zeros(B, lq, g * Hkv, 128, dtype=torch.bfloat16, device=DEV)
+        k = torch.zeros(B, Lk, Hkv, 128, dtype=torch.bfloat16, device=DEV)
+        fa.fa_fwd(q, k, k, causal=True)
+        torch.cuda.synchronize()
+        assert fa.last_dispatch()["variant"] == want, (B, Lk, Hkv, g, lq, fa.last_dispatch())
+
+
 @pytest.mark.slow
 def test_gqa8_specdec_kvcache_full_size_sampled():
     """The batched GQA-8 speculative decode (B64, qLen 4, Hq 64 / Hkv 8, D128,
     cache lengths U[1, 16384]) in the bench's launch configuration, on
     sampled rows."""
+    fa.force_variant(fa.VARIANT_AUTO)  # the library's own choice at this size
     w = wl.WORKLOADS["gqa8_specdec_kvcache_bf16"]
     q, k, v, sl = wl.make_inputs(w, DEV)
     o, lse = fa.fa_decode_kvcache(q, k, v, sl.to(DEV), causal=w.causal)
