@@ -33,7 +33,7 @@ __all__ = [
     "last_dispatch", "force_variant", "force_tcgen05_form", "test_stall_next_call", "profile_enable", "profile_read", "launch_count",
     "library_path", "load_library", "schedule", "VARIANT_AUTO", "VARIANT_MMA", "VARIANT_SCALAR", "VARIANT_TCGEN05",
     "VARIANT_TCGEN05_SPLIT",
-    "TCGEN05_AUTO", "TCGEN05_ONE_TILE", "TCGEN05_TWO_TILES", "TCGEN05_ONE_TILE_MMA",
+    "TCGEN05_AUTO", "TCGEN05_TWO_TILES", "TCGEN05_ONE_TILE_MMA",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -41,7 +41,7 @@ _LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 _lib = None
 
 VARIANT_AUTO, VARIANT_MMA, VARIANT_SCALAR, VARIANT_TCGEN05, VARIANT_TCGEN05_SPLIT = 0, 1, 2, 3, 4
-TCGEN05_AUTO, TCGEN05_ONE_TILE, TCGEN05_TWO_TILES, TCGEN05_ONE_TILE_MMA = 0, 1, 2, 3
+TCGEN05_AUTO, TCGEN05_TWO_TILES, TCGEN05_ONE_TILE_MMA = 0, 2, 3  # form 1 is retired
 _STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_WORKSPACE",
            4: "FA_ERR_CUDA", 5: "FA_ERR_TIMEOUT"}
 _DTYPE = {torch.float16: 0, torch.bfloat16: 1}

@@ -44,6 +44,15 @@ constexpr int64_t kTcSplitMinSavedBytes = int64_t(128) << 20;
 #define FA_TC_SEG_COST 4
 #endif
 constexpr int kTcSegCost = FA_TC_SEG_COST;
+// The same for the mma.sync kernel: its epilogue at a unit boundary inside a
+// piece (the merge of the four warps' partials and the partial's write) costs
+// about one tile.  Measured on one B200 (µs per call, seg cost 0 / 1 / 2):
+// single-row decode 14.83 / 14.70 / 14.72, speculative decode 19.18 / 18.80 /
+// 18.99, batched kvcache 307.9 / 307.3 / 309.8.
+#ifndef FA_MMA_SEG_COST
+#define FA_MMA_SEG_COST 1
+#endif
+constexpr int kMmaSegCost = FA_MMA_SEG_COST;
 
 thread_local std::string t_err;
 thread_local fa_dispatch_info t_disp = {};
@@ -437,10 +446,10 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     const int tile_shift = log2_exact(TK);
     const int64_t units = (int64_t)s.B * s.RB * s.Hkv;
     // every tile position must fit in 32 bits
-    // the tcgen05 kernel's segment epilogue and the next segment's start cost
-    // about kTcSegCost tiles of streaming: its units are weighted by that much
-    // more in the partition (the mma.sync kernel's by nothing)
-    pl->seg_cost = pl->main.variant == FA_VARIANT_TCGEN05_SPLIT ? kTcSegCost : 0;
+    // a segment epilogue and the next segment's start cost about seg_cost
+    // tiles of streaming: every unit is weighted by that much more in the
+    // partition
+    pl->seg_cost = pl->main.variant == FA_VARIANT_TCGEN05_SPLIT ? kTcSegCost : kMmaSegCost;
     const int64_t max_tiles = units * (((int64_t)s.Lk + TK - 1) / TK + pl->seg_cost);
     if (max_tiles >= (int64_t(1) << 31) - 1)
         return fail(FA_ERR_UNSUPPORTED, "problem too large: %lld key tiles", (long long)max_tiles);
@@ -616,11 +625,9 @@ fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor 
     p.dv = s.Dv;
     p.wait_limit_ns = kWaitLimitNs;
     p.stall = 0;
-    if (!pl.prefill) {  // the hook acts on the split-KV kernel
-        if (const unsigned long long lim = g_stall_next.exchange(0)) {
-            p.wait_limit_ns = lim;
-            p.stall = 1;
-        }
+    if (const unsigned long long lim = g_stall_next.exchange(0)) {  // test hook, any kernel
+        p.wait_limit_ns = lim;
+        p.stall = 1;
     }
     p.causal = causal ? 1 : 0;
     float sc = scale > 0.f ? scale : 1.0f / std::sqrt((float)s.Dqk);
@@ -1048,8 +1055,8 @@ fa_status fa_test_stall_next_call(unsigned long long wait_limit_ns) {
 }
 
 fa_status fa_force_tcgen05_form(int form) {
-    if (form < FA_TCGEN05_AUTO || form > FA_TCGEN05_ONE_TILE_MMA)
-        return fail(FA_ERR_INVALID_ARG, "unknown tcgen05 form %d", form);
+    if (form < FA_TCGEN05_AUTO || form > FA_TCGEN05_ONE_TILE_MMA || form == FA_TCGEN05_ONE_TILE)
+        return fail(FA_ERR_INVALID_ARG, "unknown or retired tcgen05 form %d", form);
     g_force_tc_form.store(form);
     return FA_OK;
 }

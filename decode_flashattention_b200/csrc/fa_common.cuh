@@ -74,7 +74,7 @@ struct Params {
 // kmax being the number of leading keys any of its rows can see.  In the
 // partition a unit with tiles occupies t + seg_cost positions: its tiles, then
 // seg_cost positions that stand for the fixed cost of starting and finishing a
-// unit (0 for the mma.sync kernel, whose segment epilogue is short).  The
+// unit (1 for the mma.sync kernel, 4 for the tcgen05 one).  The
 // units' positions are laid end to end (W in total) and cut into P_eff equal
 // contiguous ranges, one per CTA, so every CTA gets the same work however
 // ragged the per-batch lengths are.  A range starting inside a unit's trailing

@@ -19,16 +19,10 @@
 // Cube / Vector split of the ops-transformer walkthrough mapped onto the
 // tensor core and the CUDA cores).  K and V arrive by TMA (128-byte swizzle,
 // the canonical K-major layout for K and the MN-major one for V), and
-// tcgen05.commit releases a stage once its products are done.  Two kernels:
-//
-//   prefill3_kernel   one or two query tiles per CTA, a dedicated MMA warp
-//                     and a TMA warp; with two tiles one tile's products run
-//                     during the other's softmax, with one tile S is
-//                     double-buffered; P stays in TMEM (the library's choice)
-//   prefill_kernel    an earlier design kept for comparison (reached only by
-//                     forcing its form): one query tile per CTA whose four
-//                     softmax warps issue the products themselves, S
-//                     double-buffered in TMEM, P through shared memory
+// tcgen05.commit releases a slot once its products are done.  The kernel,
+// prefill3_kernel, takes one or two query tiles per CTA with a dedicated MMA
+// warp and a TMA warp; with two tiles one tile's products run during the
+// other's softmax, with one tile S is double-buffered; P stays in TMEM.
 //
 // Every wait is bounded; on a timeout the CTA records the error, waits
 // (bounded) for its last tensor-core work and copies, and frees its TMEM
@@ -43,364 +37,9 @@
 namespace fa {
 
 namespace pf {
-
-constexpr int kRows = 128;       // packed query rows per CTA (MMA M)
-constexpr int kD = 128;          // head dim (both products)
-constexpr int kStages = 2;
-constexpr int kBoxQ = kRows * 128;                  // one 64-column box of 128 rows (bytes): Q and P
-constexpr int kTileQ = 2 * kBoxQ;                   // Q: 128 rows x 128 elements
-constexpr int NBAR = 2 * kStages + 4;               // full[2], empty[2], s_done[2], o_done, compute sync
-constexpr int kThreads = 160;                       // 4 compute warps (TMEM lanes 0-127) + 1 producer
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
-
-// Shared-memory layout for KEYS keys per tile.  KEYS = 128: one CTA per SM,
-// a 2-stage ring of 64 KB K + V stages, S double-buffered in TMEM (512 columns).
-// KEYS = 64: half the stage and P sizes, so two CTAs share an SM (their
-// softmax warps interleave on each sub-partition), 256 TMEM columns each; the
-// base must then already be 1024-byte aligned (checked at run time) since
-// there is no room for alignment slack.
-template <int KEYS>
-struct Cfg {
-    static constexpr int kKeys = KEYS;
-    static constexpr int kBoxKV = KEYS * 128;         // one 64-column box of K or V (bytes)
-    static constexpr int kTileKV = 2 * kBoxKV;        // K or V tile: KEYS rows x 128 elements
-    static constexpr int kStageBytes = 2 * kTileKV;   // K + V
-    static constexpr int kPBytes = kRows * KEYS * 2;  // P: 128 rows x KEYS keys
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_P = OFF_Q + kTileQ;
-    static constexpr int OFF_KV = OFF_P + kPBytes;
-    static constexpr int OFF_BAR = OFF_KV + kStages * kStageBytes;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, 4 warp maxima
-    static constexpr int SLACK = KEYS == 128 ? 1024 : 0;
-    static constexpr int SMEM = OFF_MISC + 64 + SLACK;
-    static constexpr uint32_t kTmemCols = KEYS == 128 ? 512 : 256;  // S x 2 [0, 2 KEYS), O [2 KEYS, 2 KEYS + 128)
-    static constexpr int kMinBlocks = KEYS == 128 ? 1 : 2;
-    static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
-    static_assert(KEYS == 128 || 2 * (SMEM + 1024) <= 233472, "two CTAs fit an SM");
-};
-
-
+constexpr int kRows = 128;           // packed query rows per query tile (MMA M)
+constexpr int kBoxQ = kRows * 128;   // one 64-column box of 128 rows (bytes)
 }  // namespace pf
-
-template <typename T, int KEYS>
-__global__ void __launch_bounds__(pf::kThreads, pf::Cfg<KEYS>::kMinBlocks)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
-    using namespace pf;
-    using C = Cfg<KEYS>;
-    constexpr int kKeys = KEYS;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~static_cast<uintptr_t>(1023));
-    const uint32_t sb = smem_u32(smem);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (C::SLACK == 0 && smem != smem_raw) {  // no room to align: the base must already be aligned
-        if (tid == 0) atomicOr(p.status, kStatusLayout);
-        return;
-    }
-    const int rb = blockIdx.x, hkv = blockIdx.y, b = blockIdx.z;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-    auto empty_bar = [&](int s) { return smem_u32(&bars[kStages + s]); };
-    auto s_bar = [&](int buf) { return smem_u32(&bars[2 * kStages + buf]); };
-    const uint32_t o_bar = smem_u32(&bars[2 * kStages + 2]);
-    const uint32_t cs_bar = smem_u32(&bars[2 * kStages + 3]);  // bounded sync of the 4 compute warps
-    uint32_t cs_phase = 0;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
-    int *warp_keys = reinterpret_cast<int *>(smem + C::OFF_MISC + 16);
-
-    // ---- this thread's row (compute warps): head, query position, last visible key
-    const int r = rb * kRows + tid;  // packed row
-    const bool row_live = tid < kRows && r < p.R;
-    const int hq = row_live ? hkv * p.g + r / p.Lq : 0;
-    const int qi = row_live ? r % p.Lq : 0;
-    const int n = p.Lk;
-    int lim = -1;  // last visible key of the row
-    if (row_live) {
-        lim = n - 1;
-        if (p.causal) {
-            const int c = qi + n - p.Lq;
-            lim = c < lim ? c : lim;
-        }
-    }
-
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), 1);
-        }
-        mbar_init(s_bar(0), 1);
-        mbar_init(s_bar(1), 1);
-        mbar_init(o_bar, 1);
-        mbar_init(cs_bar, 4);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0) {  // TMEM: S double buffer in columns [0, 256), O in [256, 384)
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(C::kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    // keys the block's rows can see (tiles to walk)
-    {
-        int kv = lim + 1;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) kv = max(kv, __shfl_xor_sync(0xffffffffu, kv, off));
-        if (lane == 0 && warp < 4) warp_keys[warp] = kv;
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const int kmax = max(max(warp_keys[0], warp_keys[1]), max(warp_keys[2], warp_keys[3]));
-    const int ntiles = (kmax + kKeys - 1) / kKeys;
-
-    pdl_wait_primary();
-
-    if (warp == 4) {
-        // ================================================= producer: K / V tiles by TMA
-        if (lane == 0) {
-            for (int j = 0; j < ntiles; ++j) {
-                const int s = j % kStages, use = j / kStages;
-                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
-                const uint32_t kd = sb + C::OFF_KV + s * C::kStageBytes, vd = kd + C::kTileKV;
-                mbar_expect_tx(full_bar(s), C::kStageBytes);
-                for (int c = 0; c < 2; ++c) {
-                    tma_load_4d_plain(kd + c * C::kBoxKV, &tmK, full_bar(s), c * 64, j * kKeys, hkv, b);
-                    tma_load_4d_plain(vd + c * C::kBoxKV, &tmV, full_bar(s), c * 64, j * kKeys, hkv, b);
-                }
-                mbar_arrive(full_bar(s));
-            }
-        }
-        __syncwarp();
-    } else {
-        // ================================================= compute warps: one row per thread
-        // Q rows into the operand layout (K-major, 128-byte swizzle): row tid,
-        // 16-byte chunk c of the head dim at box c / 8, swizzled chunk (c % 8) ^ (tid % 8)
-        {
-            const T *qg = reinterpret_cast<const T *>(p.q);
-            const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
-            for (int c = 0; c < kD / 8; ++c) {
-                const uint32_t dst =
-                    sb + C::OFF_Q + (c >> 3) * kBoxQ + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
-                cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
-            }
-            asm volatile("cp.async.wait_all;" ::: "memory");
-            fence_proxy_async_smem();
-        }
-        constexpr bool bf16 = std::is_same<T, __nv_bfloat16>::value;
-        const uint32_t idesc_s = instr_desc(bf16, kRows, kKeys, false);
-        const uint32_t idesc_o = instr_desc(bf16, kRows, kD, true);
-        const uint32_t t_o = tmem + 2 * kKeys;  // S buffers at tmem, tmem + kKeys
-        // S_jj = Q K_jj^T into S buffer jj % 2, issued by one thread once tile jj
-        // has landed (issue_s_ready: the caller knows it has).
-        auto issue_s_ready = [&](int jj) -> bool {
-            const int st = jj % kStages;
-            const uint32_t kbase = sb + C::OFF_KV + st * C::kStageBytes;
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
-                const uint32_t aoff = (kk >> 2) * kBoxQ + (kk & 3) * 32, boff = (kk >> 2) * C::kBoxKV + (kk & 3) * 32;
-                umma(tmem + (jj & 1) * kKeys, smem_desc(sb + C::OFF_Q + aoff, 16, 1024),
-                     smem_desc(kbase + boff, 16, 1024), idesc_s, kk > 0);
-            }
-            umma_commit(s_bar(jj & 1));
-            return true;
-        };
-        auto issue_s = [&](int jj) -> bool {
-            const int st = jj % kStages;
-            if (!mbar_wait(full_bar(st), (jj / kStages) & 1, abort_flag, p.status, kWaitLimitNs)) return false;
-            return issue_s_ready(jj);
-        };
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
-        float m = -INFINITY, l = 0.f;
-        // every Q row is in shared memory
-        bool ok = consumer_sync_bounded(cs_bar, cs_phase, abort_flag, p.status, kWaitLimitNs);
-        if (ok && tid == 0 && ntiles > 0) ok = issue_s(0);
-
-        for (int j = 0; j < ntiles && ok; ++j) {
-            const int s = j % kStages;
-            const uint32_t vb = sb + C::OFF_KV + s * C::kStageBytes + C::kTileKV;
-            // the next tile's S now if its K has landed, else just before this tile's PV
-            bool next_issued = false;
-            if (tid == 0 && j + 1 < ntiles &&
-                mbar_try_wait(full_bar((j + 1) % kStages), ((j + 1) / kStages) & 1)) {
-                ok = issue_s_ready(j + 1);
-                next_issued = true;
-            }
-            __syncwarp();
-            ok = mbar_wait(s_bar(j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs) && ok;
-            if (!__all_sync(0xffffffffu, ok)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-
-            // ---- this row's scores (raw fp32): the four TMEM loads in flight at once
-            uint32_t v0[32], v1[32], v2[32], v3[32];
-            {
-                const uint32_t ts = tmem + (j & 1) * kKeys + lane_off;
-                tmem_ld32(ts, v0);
-                tmem_ld32(ts + 32, v1);
-                if constexpr (kKeys == 128) {
-                    tmem_ld32(ts + 64, v2);
-                    tmem_ld32(ts + 96, v3);
-                }
-                tmem_wait_ld();
-            }
-            float x[kKeys];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                x[e] = __uint_as_float(v0[e]);
-                x[32 + e] = __uint_as_float(v1[e]);
-                if constexpr (kKeys == 128) {
-                    x[64 + e] = __uint_as_float(v2[e]);
-                    x[96 + e] = __uint_as_float(v3[e]);
-                }
-            }
-            // mask only where some row of the warp has keys of this tile hidden
-            const int key0 = j * kKeys;
-            if (!__all_sync(0xffffffffu, key0 + kKeys - 1 <= lim)) {
-#pragma unroll
-                for (int e = 0; e < kKeys; ++e) x[e] = key0 + e <= lim ? x[e] : -INFINITY;
-            }
-            // row max with independent chains, in base-2 units (scale > 0)
-            // row max: eight independent chains of three-input max
-            float mxa[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mxa[e] = fmaxf(x[2 * e], x[2 * e + 1]);
-#pragma unroll
-            for (int e = 16; e < kKeys; e += 16)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) mxa[c] = max3f(mxa[c], x[e + 2 * c], x[e + 2 * c + 1]);
-            const float mx = max3f(max3f(mxa[0], mxa[1], mxa[2]), max3f(mxa[3], mxa[4], mxa[5]),
-                                   fmaxf(mxa[6], mxa[7])) *
-                             p.scale_log2;
-            const float mn = fmaxf(m, mx);
-            const float base = mn == -INFINITY ? 0.f : mn;
-            const float alpha = fast_exp2(m - base);  // 0 while nothing was seen
-            // p = 2^(x * scale_log2 - base): one packed FMA per key pair and one
-            // ex2 per score; sums in four packed accumulators
-            const uint64_t sc2 = pack2f(p.scale_log2, p.scale_log2), nb2 = pack2f(-base, -base);
-            uint64_t sum2[4] = {pack2f(0.f, 0.f), pack2f(0.f, 0.f), pack2f(0.f, 0.f), pack2f(0.f, 0.f)};
-            uint32_t pk[kKeys / 2];
-#pragma unroll
-            for (int e = 0; e < kKeys; e += 2) {
-                float y0, y1;
-                unpack2f(ffma2(pack2f(x[e], x[e + 1]), sc2, nb2), y0, y1);
-                const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
-                sum2[(e >> 1) & 3] = fadd2(sum2[(e >> 1) & 3], pack2f(p0, p1));
-                pk[e / 2] = Mma<T>::pack(p0, p1);
-            }
-            float suma[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) unpack2f(sum2[q], suma[2 * q], suma[2 * q + 1]);
-            const float sum = ((suma[0] + suma[1]) + (suma[2] + suma[3])) + ((suma[4] + suma[5]) + (suma[6] + suma[7]));
-            l = l * alpha + sum;
-            m = mn;
-
-            if (j > 0) {
-                // the previous PV product is done: O may be rescaled and P rewritten
-                ok = mbar_wait(o_bar, (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
-                    // O row in 64-column halves (fewer live registers with two CTAs per SM)
-#pragma unroll
-                    for (int h = 0; h < kD / 64; ++h) {
-                        const uint32_t to = t_o + lane_off + h * 64;
-                        tmem_ld32(to, v0);
-                        tmem_ld32(to + 32, v1);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
-                            v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
-                        }
-                        tmem_st32(to, v0);
-                        tmem_st32(to + 32, v1);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            // ---- P row into the operand layout (keys as K, K-major, swizzled)
-#pragma unroll
-            for (int c = 0; c < kKeys / 8; ++c) {
-                const uint32_t dst = sb + C::OFF_P + (c >> 3) * kBoxQ + tid * 128 + ((((c & 7) ^ (tid & 7))) << 4);
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[c * 4]),
-                             "r"(pk[c * 4 + 1]), "r"(pk[c * 4 + 2]), "r"(pk[c * 4 + 3])
-                             : "memory");
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            if (!consumer_sync_bounded(cs_bar, cs_phase, abort_flag, p.status, kWaitLimitNs)) {
-                ok = false;
-                break;
-            }
-            if (tid == 0 && j + 1 < ntiles && !next_issued) ok = issue_s(j + 1) && ok;
-            if (tid == 0) {  // O += P V
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    const uint32_t aoff = (kk >> 2) * kBoxQ + (kk & 3) * 32;
-                    umma(t_o, smem_desc(sb + C::OFF_P + aoff, 16, 1024), smem_desc(vb + kk * 2048, C::kBoxKV, 1024),
-                         idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(o_bar);
-                umma_commit(empty_bar(s));
-            }
-            __syncwarp();
-        }
-
-        // ---- epilogue: O / l, lse
-        if (ok && ntiles > 0) {
-            ok = mbar_wait(o_bar, (ntiles - 1) & 1, abort_flag, p.status, kWaitLimitNs);
-            ok = __all_sync(0xffffffffu, ok);
-            tc_fence_after();
-        }
-        if (ok) {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            T *og = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)qi * p.o_sl + (long long)hq * p.o_sh;
-#pragma unroll
-            for (int c = 0; c < kD / 32; ++c) {
-                uint32_t v[32];
-                if (ntiles > 0) {
-                    tmem_ld32(t_o + lane_off + c * 32, v);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = 0u;
-                }
-                if (row_live) {
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        float f[8];
-#pragma unroll
-                        for (int z = 0; z < 8; ++z) f[z] = __uint_as_float(v[e + z]) * inv;
-                        store_row8<T>(og + c * 32 + e, f);
-                    }
-                }
-            }
-            if (row_live && p.lse)
-                p.lse[b * p.lse_sb + hq * p.lse_sh + qi] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-        } else if (tid == 0) {
-            // timed out: wait (bounded) for the tensor core's last work before TMEM is freed
-            volatile int no_abort = 0;
-            mbar_wait(o_bar, 0, &no_abort, nullptr, kWaitLimitNs / 8);
-            mbar_wait(o_bar, 1, &no_abort, nullptr, kWaitLimitNs / 8);
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols) : "memory");
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Two query tiles per CTA with 128-key K / V tiles (the kernel also runs
@@ -539,10 +178,13 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
     if (warp == kProducerWarp) {
         // ================================================= producer: K(0), V(0), K(1), ... by TMA
         if (lane == 0) {
+            // test hook: the first CTA leaves K(0)'s slot empty (no copy, no
+            // arrival), so the MMA thread's wait on it runs out
+            const int q_first = p.stall && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 ? 1 : 0;
             int issued = 0;
-            for (int q = 0; q < 2 * ntiles; ++q) {
+            for (int q = q_first; q < 2 * ntiles; ++q) {
                 const int s = q % kSlots, use = q / kSlots;
-                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, kWaitLimitNs)) break;
+                if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
                 const uint32_t dst = sb + L::OFF_KV + s * L::kSlotBytes;
                 const CUtensorMap *map = (q & 1) ? &tmV : &tmK;
                 mbar_expect_tx(full_bar(s), L::kSlotBytes);
@@ -554,8 +196,8 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             if (*abort_flag) {
                 // let the copies still in flight land before the CTA's shared memory is released
                 volatile int no_abort = 0;
-                for (int q = issued - kSlots < 0 ? 0 : issued - kSlots; q < issued; ++q)
-                    mbar_wait(full_bar(q % kSlots), (q / kSlots) & 1, &no_abort, nullptr, kWaitLimitNs / 16);
+                for (int q = issued - kSlots < q_first ? q_first : issued - kSlots; q < issued; ++q)
+                    mbar_wait(full_bar(q % kSlots), (q / kSlots) & 1, &no_abort, nullptr, p.wait_limit_ns / 16);
             }
         }
         __syncwarp();
@@ -571,7 +213,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             const uint64_t dk0 = smem_desc(sb + L::OFF_KV, 16, 1024);        // a slot holding K
             const uint64_t dv0 = smem_desc(sb + L::OFF_KV, kBox, 1024);      // a slot holding V
             auto wait = [&](uint32_t bar, uint32_t parity) {
-                return mbar_wait(bar, parity, abort_flag, p.status, kWaitLimitNs);
+                return mbar_wait(bar, parity, abort_flag, p.status, p.wait_limit_ns);
             };
             // S_g(j) = Q_g K(j)^T; K(j) is ring entry 2j
             auto issue_s = [&](int g, int j) {
@@ -671,7 +313,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // every product this thread issued is done before TMEM can be freed
             umma_commit(drain_bar);
             volatile int no_abort = 0;
-            mbar_wait(drain_bar, 0, &no_abort, p.status, kWaitLimitNs);
+            mbar_wait(drain_bar, 0, &no_abort, p.status, p.wait_limit_ns);
         }
         __syncwarp();
     } else {
@@ -696,8 +338,8 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         for (int j = 0; j < ntiles && ok; ++j) {
             // this tile's S: the group's buffer (two tiles), or buffer j % 2 (one tile)
             const uint32_t t_s = tmem + (TILES == 2 ? grp : (j & 1)) * kKeys + lane_off;
-            ok = TILES == 2 ? mbar_wait(s_bar(grp), j & 1, abort_flag, p.status, kWaitLimitNs)
-                            : mbar_wait(s_bar(j & 1), (j >> 1) & 1, abort_flag, p.status, kWaitLimitNs);
+            ok = TILES == 2 ? mbar_wait(s_bar(grp), j & 1, abort_flag, p.status, p.wait_limit_ns)
+                            : mbar_wait(s_bar(j & 1), (j >> 1) & 1, abort_flag, p.status, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -764,7 +406,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // after it; with one tile S(j) may have gone first, so wait for it.
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 if constexpr (TILES == 1) {
-                    ok = mbar_wait(o_bar(0), (j - 1) & 1, abort_flag, p.status, kWaitLimitNs);
+                    ok = mbar_wait(o_bar(0), (j - 1) & 1, abort_flag, p.status, p.wait_limit_ns);
                     if (!__all_sync(0xffffffffu, ok)) {
                         ok = false;
                         break;
@@ -796,8 +438,8 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             // the last PV: with two tiles o_bar's one commit; with one tile the
             // MMA thread's final (drain) commit -- up to two of o_bar's per-tile
             // phases can still be open here, which a parity wait cannot tell apart
-            ok = TILES == 2 ? mbar_wait(o_bar(grp), 0, abort_flag, p.status, kWaitLimitNs)
-                            : mbar_wait(drain_bar, 0, abort_flag, p.status, kWaitLimitNs);
+            ok = TILES == 2 ? mbar_wait(o_bar(grp), 0, abort_flag, p.status, p.wait_limit_ns)
+                            : mbar_wait(drain_bar, 0, abort_flag, p.status, p.wait_limit_ns);
             ok = __all_sync(0xffffffffu, ok);
             tc_fence_after();
         }
@@ -836,23 +478,6 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
     }
 }
 
-template <typename T, int KEYS>
-static void fill(KernelInfo *out) {
-    out->fn = reinterpret_cast<const void *>(&prefill_kernel<T, KEYS>);
-    out->threads = pf::kThreads;
-    out->smem = pf::Cfg<KEYS>::SMEM;
-    out->tile_keys = KEYS;
-    out->stages = pf::kStages;
-    out->variant = 3;  // FA_VARIANT_TCGEN05
-    out->rows = pf::kRows;
-    out->form = FA_TCGEN05_ONE_TILE;
-}
-
-// 128-key tiles, one CTA per SM.  (64-key tiles with two CTAs per SM measured
-// the same on a 4K causal prefill -- 332 vs 334 us -- the doubled per-tile
-// overhead cancelling the second CTA's interleaving.)
-constexpr int kPrefillKeys = 128;
-
 template <typename T, int TILES, int D>
 static void fill3(KernelInfo *out) {
     out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES, D>);
@@ -869,11 +494,6 @@ bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out) {
     if (dtype < 0 || dtype > 1 || dqk != dv || (dqk != 64 && dqk != 128)) return false;
     const bool h = dtype == 0;
     switch (form) {
-    case FA_TCGEN05_ONE_TILE:  // head dim 128 only
-        if (dqk != 128) return false;
-        if (h) fill<__half, kPrefillKeys>(out);
-        else fill<__nv_bfloat16, kPrefillKeys>(out);
-        return true;
     case FA_TCGEN05_TWO_TILES:
         if (dqk == 64) {
             if (h) fill3<__half, 2, 64>(out);

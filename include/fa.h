@@ -352,11 +352,9 @@ FA_API fa_status fa_force_variant(int variant);
 /*
  * Forms of the tcgen05 kernel (all: 128 packed rows per query tile, 128-key
  * K / V tiles, accumulators in TMEM, the whole key range per CTA):
- *   FA_TCGEN05_ONE_TILE       one tile per CTA; the softmax warps issue the
- *                             products themselves and S is double-buffered, so
- *                             the next tile's QK^T runs during this tile's softmax
- *                             (head dim 128 only; an earlier design, kept for
- *                             comparison -- the library no longer chooses it);
+ *   FA_TCGEN05_ONE_TILE       retired (an earlier one-tile design whose
+ *                             softmax warps issued the products; removed):
+ *                             forcing it is FA_ERR_INVALID_ARG;
  *   FA_TCGEN05_TWO_TILES      two tiles per CTA and a dedicated MMA warp: one
  *                             tile's products run while the other tile's
  *                             softmax does (S single-buffered per tile);
@@ -377,10 +375,11 @@ typedef enum {
 FA_API fa_status fa_force_tcgen05_form(int form);
 
 /*
- * Test hook for the failure path: the next split-KV compute call of this
- * process bounds its pipeline waits by wait_limit_ns (instead of 4 s) and its
- * first CTA leaves its first pipeline stage empty -- no copy, no arrival --
- * so that CTA's consumers give up after wait_limit_ns, record
+ * Test hook for the failure path: the next compute call of this process
+ * (split-KV or tcgen05 prefill kernel) bounds its pipeline waits by
+ * wait_limit_ns (instead of 4 s) and its first CTA leaves its first pipeline
+ * stage empty -- no copy, no arrival -- so that CTA's consumers give up after
+ * wait_limit_ns, record
  * FA_ERR_TIMEOUT in the device status word and return (as do the producer,
  * after a bounded wait for its copies in flight).  The call's outputs are
  * then unspecified; fa_check_status reports the timeout and later calls run
@@ -412,7 +411,7 @@ FA_API fa_status fa_profile_read(double *main_ms, int64_t *main_launches, double
  * rows_per_cta says which a call used) -- ordered batch-major, then row
  * block, then kv head, and owns t = ceil(visible keys / tile_keys) tiles.  In
  * the partition a unit with t > 0 tiles occupies t + seg_cost positions (its
- * tiles first; seg_cost stands for the fixed cost of a unit: 0 for the
+ * tiles first; seg_cost stands for the fixed cost of a unit: 1 for the
  * mma.sync kernel, 4 for the tcgen05 one).  The W positions of all units are
  * laid end to end and cut into ctas_used = min(num_ctas, ceil(W / min_share))
  * contiguous pieces, one per CTA, whose sizes differ by at most one position

@@ -137,7 +137,8 @@ def test_force_tcgen05_form_rejects_unknown():
     lib = fa.load_library()
     assert lib.fa_force_tcgen05_form(4) == INVALID
     assert lib.fa_force_tcgen05_form(-1) == INVALID
-    for form in (fa.TCGEN05_ONE_TILE, fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA, fa.TCGEN05_AUTO):
+    assert lib.fa_force_tcgen05_form(1) == INVALID  # the retired one-tile design
+    for form in (fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA, fa.TCGEN05_AUTO):
         assert lib.fa_force_tcgen05_form(form) == OK
 
 

@@ -3,9 +3,10 @@ pipeline stage of the split-KV kernel empty (a barrier phase nothing
 completes) and bounds the call's waits by 20 ms.  The waiting warps give up,
 record FA_ERR_TIMEOUT in the device status word and return; the host reads it
 with check_status, and the next call on the same context runs normally and
-matches the oracle.  Covered for the mma.sync kernel, its fp32 FMA form and
-the tcgen05 split-KV kernel (whose abort path must also wait for its tensor-core
-work and free its tensor memory before the next call can allocate it)."""
+matches the oracle.  Covered for the mma.sync kernel, its fp32 FMA form, the
+tcgen05 split-KV kernel and both forms of the tcgen05 prefill kernel (whose
+abort paths must also wait for their tensor-core work and free their tensor
+memory before the next call can allocate it)."""
 import time
 
 import pytest
@@ -27,6 +28,7 @@ LIMIT_NS = 20_000_000  # 20 ms
 def _reset():
     yield
     fa.force_variant(fa.VARIANT_AUTO)
+    fa.force_tcgen05_form(fa.TCGEN05_AUTO)
     torch.cuda.synchronize()
     fa.check_status()
 
@@ -67,3 +69,35 @@ def test_timeout_is_reported_and_the_context_stays_usable(variant):
     fa.check_status()
     ro, rl = oracle_full(q, k, v, w.causal, seqlens=sl)
     compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, w.dtype, "after a timeout")
+
+
+@pytest.mark.parametrize("form", [fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA])
+def test_prefill_timeout_is_reported_and_the_context_stays_usable(form):
+    # 512 packed rows per kv head (two or four row blocks), causal, ragged keys:
+    # the stalled CTA (the grid's first, the last row block) has tiles to wait for
+    w = wl.Workload("stall_pf", "fwd", "blhd", torch.bfloat16, B=1, Lq=256, Hq=4, Hkv=2, Lk=700, Dqk=128, Dv=128,
+                    causal=True, seed=34)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+
+    def call():
+        fa.force_variant(fa.VARIANT_TCGEN05)
+        fa.force_tcgen05_form(form)
+        return fa.fa_fwd(q, k, v, causal=True)
+
+    fa.check_status()
+    fa.test_stall_next_call(LIMIT_NS)
+    t0 = time.perf_counter()
+    call()
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert fa.last_dispatch()["tcgen05_form"] == form
+    with pytest.raises(fa.FaError) as e:
+        fa.check_status()
+    assert e.value.status == FA_ERR_TIMEOUT
+    assert elapsed < 2.0, elapsed
+    fa.check_status()
+    o, lse = call()  # allocates the tensor memory the stalled CTA held
+    torch.cuda.synchronize()
+    fa.check_status()
+    ro, rl = oracle_full(q, k, v, True)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, w.dtype, "prefill after a timeout")

@@ -27,7 +27,7 @@ def _reset():
     fa.check_status()
 
 
-FORMS = [fa.TCGEN05_ONE_TILE, fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA]
+FORMS = [fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA]
 
 
 CASES = [  # B, Lq, Hq, Hkv, Lk, causal
@@ -150,10 +150,3 @@ def test_head_dim_64_parity(form, case):
     compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 hd64 form {form}")
 
 
-def test_head_dim_64_one_tile_form_is_refused():
-    q = torch.zeros(1, 128, 1, 64, dtype=torch.bfloat16, device=DEV)
-    k = torch.zeros(1, 256, 1, 64, dtype=torch.bfloat16, device=DEV)
-    fa.force_variant(fa.VARIANT_TCGEN05)
-    fa.force_tcgen05_form(fa.TCGEN05_ONE_TILE)
-    with pytest.raises(fa.FaError, match="tcgen05"):
-        fa.fa_fwd(q, k, k, causal=True)
