@@ -180,6 +180,7 @@ struct Shapes {
     int B, Lq, Hq, Lk, Hkv, Dqk, Dv, g, R, RB, BR;
     int rpc;        // packed rows per row block: RB = ceil(R / rpc) row blocks per (batch, kv head)
     int KDqk, KDv;  // head dims of the kernel instance that runs the call (>= Dqk, Dv)
+    int page = 0;   // paged cache: keys per block (0: dense)
 };
 
 // Head dims: any multiple of 8 from 8 to 256 (a TMA row stride must be a
@@ -266,6 +267,7 @@ fa_status check_shapes(const fa_tensor *q, const fa_tensor *k, const fa_tensor *
         if ((int64_t)pg->max_pages * page > INT32_MAX / 2)
             return fail(FA_ERR_UNSUPPORTED, "max_blocks_per_seq * page too large");
         s->Lk = (int)((int64_t)pg->max_pages * page);
+        s->page = (int)page;
     } else if (k->shape[0] != s->B || v->shape[0] != s->B) {
         return fail(FA_ERR_INVALID_ARG, "batch mismatch: q %d, k %lld, v %lld", s->B, (long long)k->shape[0],
                     (long long)v->shape[0]);
@@ -428,7 +430,10 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
         }
     } else {
         ok = variant == FA_VARIANT_SCALAR ? fa::get_scalar_kernel(s.dtype, s.KDqk, s.KDv, &pl->main)
-                                          : fa::get_mma_kernel(s.dtype, s.KDqk, s.KDv, &pl->main);
+                                          : fa::get_mma_kernel(s.dtype, s.KDqk, s.KDv,
+                                                               // pages in whole 64-column chunks of the call's dims
+                                                               s.Dqk == s.KDqk && s.Dv == s.KDv ? s.page : 0,
+                                                               &pl->main);
     }
     if (variant == FA_VARIANT_SCALAR && ok && s.R != 1)
         return fail(FA_ERR_UNSUPPORTED, "the scalar variant handles one packed row (g * Lq = 1), got %d", s.R);
@@ -471,6 +476,7 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
         host_schedule(s, causal, tile_shift, pl->seg_cost, (int)P, pl->min_share, &W, &pt, &need);
         if (num_splits <= 0 && W <= P) {  // small problem: one tile per CTA, as many CTAs as tiles
             pl->min_share = 1;
+            pl->seg_cost = 0;  // (no CTA holds two units: nothing to weigh)
             host_schedule(s, causal, tile_shift, pl->seg_cost, (int)P, pl->min_share, &W, &pt, &need);
         }
         pl->W = W;
@@ -548,6 +554,41 @@ fa_status encode_kv_map(const fa_tensor *t, int box_rows, CUtensorMap *map, cons
     CUresult r = fn(map, dt, 4, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     CU_TENSOR_MAP_SWIZZLE_128B, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(FA_ERR_UNSUPPORTED, "%s: cuTensorMapEncodeTiled failed (%d)", name, (int)r);
+    return FA_OK;
+}
+
+// Paged cache [blocks, page, H, D] (page < tile, D a multiple of 64) as a 5-D
+// TMA map {64, page, D / 64, H, blocks}: one box is one page of one head with
+// all its 64-column chunks, chunk after chunk in shared memory (128-byte
+// swizzle), so a tile takes one box per page for K and one for V instead of
+// one per page and chunk.
+fa_status encode_page_map(const fa_tensor *t, CUtensorMap *map, const char *name) {
+    auto fn = encode_fn();
+    if (!fn) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int64_t elt = 2, D = t->shape[3];
+    cuuint64_t dims[5] = {64, (cuuint64_t)t->shape[1], (cuuint64_t)(D / 64), (cuuint64_t)t->shape[2],
+                          (cuuint64_t)t->shape[0]};
+    // row within the page, chunk, head, block (elements); an extent-1
+    // dimension is never stepped and gets a harmless legal stride
+    int64_t st[4] = {t->stride[1], 64, t->stride[2], t->stride[0]};
+    for (int i = 0; i < 4; ++i)
+        if (dims[i + 1] == 1 || st[i] == 0) st[i] = 64;
+    cuuint64_t strides[4];
+    for (int i = 0; i < 4; ++i) strides[i] = (cuuint64_t)(st[i] * elt);
+    cuuint32_t box[5] = {64, (cuuint32_t)t->shape[1], (cuuint32_t)(D / 64), 1, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUtensorMapDataType dt = t->dtype == FA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    // whole head rows are read, so a 256-byte promotion pulls in nothing else
+    // when rows start on 256-byte lines and fill them
+    const bool lines256 = reinterpret_cast<uintptr_t>(t->data) % 256 == 0 && (D * elt) % 256 == 0 &&
+                          (t->shape[1] == 1 || (t->stride[1] * elt) % 256 == 0) &&
+                          (t->shape[2] == 1 || (t->stride[2] * elt) % 256 == 0) &&
+                          (t->shape[0] == 1 || (t->stride[0] * elt) % 256 == 0);
+    CUresult r = fn(map, dt, 5, t->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B,
+                    lines256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(FA_ERR_UNSUPPORTED, "%s: cuTensorMapEncodeTiled (pages) failed (%d)", name, (int)r);
     return FA_OK;
 }
 
@@ -654,6 +695,9 @@ fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor 
         p.max_pages = pg->max_pages;
         p.page_shift = log2_exact((int)k->shape[1]);
         p.num_blocks = (int)k->shape[0];
+        // pages smaller than a tile on the mma.sync kernel's page-interleaved
+        // instance: one 5-D box per page
+        p.kv_ilv = pl.main.ilv;
     }
 
     if (ap) {
@@ -723,8 +767,13 @@ fa_status run(Shapes s, const fa_tensor *q, const fa_tensor *k, const fa_tensor 
     if (launch_main) {
         CUtensorMap tmK, tmV;
         const int box_rows = pg ? (int)std::min<int64_t>(k->shape[1], pl.main.tile_keys) : pl.main.tile_keys;
-        if ((st = encode_kv_map(k, box_rows, &tmK, "k"))) return st;
-        if ((st = encode_kv_map(v, box_rows, &tmV, "v"))) return st;
+        if (p.kv_ilv) {
+            if ((st = encode_page_map(k, &tmK, "k_pages"))) return st;
+            if ((st = encode_page_map(v, &tmV, "v_pages"))) return st;
+        } else {
+            if ((st = encode_kv_map(k, box_rows, &tmK, "k"))) return st;
+            if ((st = encode_kv_map(v, box_rows, &tmV, "v"))) return st;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)pl.P);
         cfg.blockDim = dim3((unsigned)pl.main.threads);

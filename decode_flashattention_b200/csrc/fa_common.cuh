@@ -55,6 +55,12 @@ struct Params {
     int max_pages;         // block-table entries per batch
     int page_shift;        // log2(page)
     int num_blocks;
+    // Paged pages smaller than a tile, mma.sync kernel: each page's K (and V)
+    // rows come in one 5-D box holding all of its 64-column chunks, so in a
+    // stage slot page `sub` of the tile starts at sub * page * 128 * chunks
+    // bytes and its chunk c at + c * page * 128 (else chunk c of the whole
+    // tile starts at c * TK * 128, as for dense K / V).
+    int kv_ilv;
     int seqlen_add;        // tokens appended to every cache by this call (added to seqlens[b])
     // Packed variable-length inputs (cu_q non-null): q / o are [1, total_q, H, D]
     // and k / v [1, total_k, Hkv, D]; sequence b owns query tokens
@@ -262,6 +268,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
         " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "l"(policy)
+        : "memory");
+}
+
+// The same for a 5-D tile (one page of a paged cache with all its 64-column
+// chunks: coordinates {0, row, 0, head, block}).
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3, int c4, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4),
         "l"(policy)
         : "memory");
 }

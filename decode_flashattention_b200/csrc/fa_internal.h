@@ -15,10 +15,13 @@ struct KernelInfo {
     int variant;     // fa_variant
     int rows;        // packed query rows per CTA (tcgen05 kernels)
     int form;        // fa_tcgen05_form (tcgen05 kernels)
+    int ilv = 0;     // mma.sync kernel: paged pages gathered in 5-D boxes (Params::kv_ilv)
 };
 
-// Main split-KV kernel using mma.sync (keys as M, packed rows as N).
-bool get_mma_kernel(int dtype, int dqk, int dv, KernelInfo *out);
+// Main split-KV kernel using mma.sync (keys as M, packed rows as N).  page > 0:
+// a paged cache whose pages are whole 64-column chunks of the call's head
+// dims; pages smaller than the instance's tile take its page-interleaved form.
+bool get_mma_kernel(int dtype, int dqk, int dv, int page, KernelInfo *out);
 // LSE-weighted combine of split partials (per-row or per-unit form), the
 // choice of form for `units` units of row blocks of rpc rows on `sms` SMs, and
 // its grid for `rows` output rows (R packed rows per kv head).

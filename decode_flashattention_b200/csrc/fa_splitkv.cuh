@@ -55,8 +55,11 @@ constexpr int kMetaFinal = 16; // the CTA's last tile
 
 // KB: 16-key blocks per consumer warp per tile (2: 128-key tiles; 1: 64-key
 // tiles, for head dims whose 128-key stage would not leave room for a ring).
-template <int DQK, int DV, int STAGES, bool FMA, int KB = 2>
+// ILV: paged K / V with pages smaller than a tile, each page gathered in one
+// 5-D box with all its 64-column chunks (Params::kv_ilv).
+template <int DQK, int DV, int STAGES, bool FMA, int KB = 2, bool ILV_ = false>
 struct SplitCfg {
+    static constexpr bool ILV = ILV_;
     static constexpr int KEYS_PER_WARP = 16 * KB;
     static constexpr int TK = KEYS_PER_WARP * kConsumerWarps;  // keys per tile
     static constexpr int TK_SHIFT = KB == 2 ? 7 : 6;
@@ -232,6 +235,27 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
                         tma_load_4d(vdst + c * C::BOX_BYTES, tmV, bar, c * 64, G.k0 + j, hkv, kb, policy);
                 }
             }
+        } else if constexpr (C::ILV) {
+            // pages smaller than a tile, each page's K / V rows with all their
+            // chunks in one 5-D box: the page's rows land at sub * page * 128
+            // * chunks in the slot, chunk after chunk
+            __syncwarp();
+            const int nsub = C::TK >> p.page_shift;
+            const int count = (do_k ? nsub : 0) + (do_v ? nsub : 0);
+            for (int idx = lane; idx < count; idx += 32) {
+                const bool is_k = do_k && idx < nsub;
+                const int sub = do_k ? (is_k ? idx : idx - nsub) : idx;
+                const int key = j + (sub << p.page_shift);
+                const int page = key >> p.page_shift;
+                int blk = p.num_blocks;
+                if (page < p.max_pages) {
+                    const int e = __ldg(p.block_table + (long long)b * p.bt_stride + page);
+                    if (e >= 0 && e < p.num_blocks) blk = e;
+                }
+                const uint32_t off = (uint32_t)(sub << p.page_shift) * 128u * (is_k ? C::KBOX : C::VBOX);
+                if (is_k) tma_load_5d(kdst + off, tmK, bar, 0, 0, 0, hkv, blk, policy);
+                else tma_load_5d(vdst + off, tmV, bar, 0, 0, 0, hkv, blk, policy);
+            }
         } else {
             __syncwarp();
             const int sub_shift = p.page_shift < C::TK_SHIFT ? p.page_shift : C::TK_SHIFT;
@@ -363,11 +387,12 @@ __device__ __forceinline__ void splitkv_produce(const CUtensorMap *tmK, const CU
 }
 
 
-template <typename T, int DQK, int DV, int STAGES, bool FMA, int KB = 2>
+template <typename T, int DQK, int DV, int STAGES, bool FMA, int KB = 2, bool ILV = false>
 __global__ void __launch_bounds__(kThreads, 1)
     splitkv_kernel(const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const Params p) {
-    using C = SplitCfg<DQK, DV, STAGES, FMA, KB>;
+    using C = SplitCfg<DQK, DV, STAGES, FMA, KB, ILV>;
+    static_assert(!ILV || !FMA, "the page-interleaved layout is read by the mma.sync consumer only");
     static_assert(!FMA || KB == 2, "the FMA consumer gives each lane one of 32 keys per warp");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -446,7 +471,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r_lo = 2 * (lane & 3);         // accumulator rows of this lane: r_lo, r_lo + 1
     uint32_t ep_phase = 0;
 
-    // Per-lane ldmatrix offsets inside a stage (the 128-byte swizzle XORs the
+    // Where the 16-key blocks and 64-column chunks of a stage's K and V sit:
+    // block kb of this warp at kblk[kb] / vblk[kb] from the slot, chunk c at
+    // c * chs further (the whole tile's chunks one after the other, or, for
+    // pages smaller than a tile gathered in 5-D boxes, each page's chunks
+    // one after the other -- Params::kv_ilv).
+    const uint32_t chs = ILV ? (128u << p.page_shift) : (uint32_t)C::BOX_BYTES;
+    uint32_t kblk[KB], vblk[KB];  // (ILV only; the plain layout's are kw * 128 + kb * 2048)
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+        const int r = kw + kb * 16;  // the block's first key within the tile
+        const uint32_t in_page = (uint32_t)(r & ((1 << p.page_shift) - 1)) * 128u;
+        const uint32_t page0 = (uint32_t)(r >> p.page_shift) * chs;
+        kblk[kb] = page0 * C::KBOX + in_page;
+        vblk[kb] = page0 * C::VBOX + in_page;
+    }
+    // Per-lane ldmatrix offsets inside a block (the 128-byte swizzle XORs the
     // 16-byte chunk index with key & 7, and key & 7 == lane & 7 here).
     uint32_t koff[DQK / 16], voff[DV / 16];
     {
@@ -455,13 +495,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < DQK / 16; ++kk) {
             const int d = kk * 16 + ((lane >> 4) & 1) * 8;
-            koff[kk] = (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4) + kkey * 128;
+            koff[kk] = (d >> 6) * chs + ((((d & 63) >> 3) ^ sw) << 4) + kkey * 128;
         }
         const int vkey = (lane & 7) + ((lane >> 4) & 1) * 8;  // A = V^T block: (d lo|hi) x (k0-7|k8-15)
 #pragma unroll
         for (int t = 0; t < DV / 16; ++t) {
             const int d = t * 16 + ((lane >> 3) & 1) * 8;
-            voff[t] = (d >> 6) * C::BOX_BYTES + ((((d & 63) >> 3) ^ sw) << 4) + vkey * 128;
+            voff[t] = (d >> 6) * chs + ((((d & 63) >> 3) ^ sw) << 4) + vkey * 128;
         }
     }
 
@@ -711,8 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             StageMeta md = {0, 0, 0, 0, kMetaFirst | kMetaLast | (it == -1 ? kMetaWhole : 0), 0, 0, 0};
             if (!warm) md = meta[s];
             if (md.flags & kMetaDone) break;
-            const uint32_t kbase = smem_base + s * C::STAGE_BYTES + kw * 128;
-            const uint32_t vbase = kbase + C::KBOX * C::BOX_BYTES;
+            const uint32_t kst = smem_base + s * C::STAGE_BYTES;  // the stage's K
+            const uint32_t vst = kst + C::KBOX * C::BOX_BYTES;    // and V
+            const uint32_t kbase = kst + kw * 128;                // this warp's keys (plain layout)
+            const uint32_t vbase = vst + kw * 128;
 
             if (md.flags & kMetaFirst) {
                 // Q as the B operand: lane holds row (lane >> 2), dims 2*(lane & 3) + {0, 1} (+8).
@@ -752,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
                     uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4(kbase + kb * 16 * 128 + koff[kk], a0, a1, a2, a3);
+                    ldmatrix_x4((ILV ? kst + kblk[kb] : kbase + kb * 16 * 128) + koff[kk], a0, a1, a2, a3);
                     if (kk & 1) Mma<T>::run(sd[kb], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
                     else Mma<T>::run(sc[kb], a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
                 }
@@ -814,7 +856,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int key = idx / (C::VBOX * 8);
                     const int rem = idx % (C::VBOX * 8);
                     if (jbase + key >= n) {
-                        const uint32_t a = vbase + (rem >> 3) * C::BOX_BYTES + key * 128 + (rem & 7) * 16;
+                        const uint32_t a = ILV ? vst + vblk[key >> 4] + (rem >> 3) * chs + (key & 15) * 128 + (rem & 7) * 16
+                                               : vbase + (rem >> 3) * C::BOX_BYTES + key * 128 + (rem & 7) * 16;
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
                     }
                 }
@@ -827,7 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                 for (int kb = 0; kb < KB; ++kb) {
                     uint32_t a0, a1, a2, a3;
-                    ldmatrix_x4_trans(vbase + kb * 16 * 128 + voff[t], a0, a1, a2, a3);
+                    ldmatrix_x4_trans((ILV ? vst + vblk[kb] : vbase + kb * 16 * 128) + voff[t], a0, a1, a2, a3);
                     Mma<T>::run(acc[t], a0, a1, a2, a3, pb[kb][0], pb[kb][1]);
                 }
             }

@@ -59,6 +59,7 @@ constexpr int kPvN = 64;             // N of the PV products (rows, zero padded)
 
 template <int DQK, int DV, int NR, int KS, int VS>
 struct TcCfg {
+    static constexpr bool ILV = false;  // paged K / V in the plain per-chunk layout
     static constexpr int TK = 128;
     static constexpr int TK_SHIFT = 7;
     static constexpr int KBOX = DQK / 64;
