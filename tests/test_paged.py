@@ -82,6 +82,28 @@ def test_head_dims_and_types(d, dt):
     _check(*_case(32, d=d, dt=dt, seed=d[0] + (dt == torch.float16)))
 
 
+@pytest.mark.parametrize("page,d", [(16, (256, 256)), (32, (256, 256)), (16, (64, 64)), (16, (192, 128)),
+                                    (16, (96, 96)), (32, (40, 40)), (16, (128, 64))])
+def test_pages_below_the_tile_every_head_dim(page, d):
+    """Pages smaller than the tile: one 5-D box per page where the head dims
+    are the kernel instance's own (whole 64-column chunks; the 64-key tiles
+    of head dim 256 included), one box per page and chunk otherwise."""
+    _check(*_case(page, d=d, Lk=700, seed=page + d[0] + d[1]))
+
+
+@pytest.mark.parametrize("page", [16, 32, 64])
+def test_small_pages_equal_dense_call_bitwise(page):
+    """Pages gathered one 5-D box per page land the keys where the dense
+    call's boxes put them: the same arithmetic, the same bits."""
+    w, q, kp, vp, bt, sl = _case(page, B=3, Lk=640, seed=13 + page)
+    k = oracle.gather_pages(kp.cpu(), bt.cpu().numpy(), sl.numpy()).to(DEV)
+    v = oracle.gather_pages(vp.cpu(), bt.cpu().numpy(), sl.numpy()).to(DEV)
+    o1, l1 = fa.fa_decode_kvcache_paged(q, kp, vp, bt, sl.to(DEV))
+    o2, l2 = fa.fa_decode_kvcache(q, k, v, sl.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 @pytest.mark.parametrize("g,lq", [(1, 1), (4, 1), (8, 1), (2, 4), (1, 8)])
 def test_gqa_and_small_q_causal(g, lq):
     _check(*_case(64, Lq=lq, Hq=2 * g, Hkv=2, causal=True, seed=10 * g + lq))
