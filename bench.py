@@ -176,8 +176,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ helpers
-def tensor_roofline(w, seqlens, ms_per_call, prof, traffic=None):
-    """Roofline of a call on the tcgen05 kernel: bound by the tensor cores.
+def tensor_roofline(w, seqlens, ms_per_call, prof, traffic=None,
+                    kernel="tcgen05 dense kernel (whole call)"):
+    """Roofline of a prefill-shaped call: bound by the tensor cores.
     achieved = the call's multiply-add flops / its time; peak = the measured
     sustained cuBLAS bf16 rate (the kernel runs back to back for seconds), the
     same for fp16 (the nominal fp16 and bf16 rates are equal)."""
@@ -192,10 +193,13 @@ def tensor_roofline(w, seqlens, ms_per_call, prof, traffic=None):
     else:
         peak, kind = 1400.0, "fallback (sustained)"
     achieved = flops / (ms_per_call / 1e3) / 1e12
-    return {"bound": "tensor", "kernel": "tcgen05 dense kernel (whole call)", "achieved": round(achieved, 2),
+    iso = {"main": round(prof["main_ms"] / max(prof["main_launches"], 1) * 1e3, 3)}
+    if prof.get("combine_ms"):
+        iso["combine"] = round(prof["combine_ms"] / max(prof["main_launches"], 1) * 1e3, 3)
+    return {"bound": "tensor", "kernel": kernel, "achieved": round(achieved, 2),
             "peak": peak, "peak_kind": kind, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "traffic": traffic, "algorithmic_flops_per_launch": flops, "kernel_us": round(ms_per_call * 1e3, 3),
-            "isolated_us": {"tcgen05": round(prof["main_ms"] / max(prof["main_launches"], 1) * 1e3, 3)}}
+            "isolated_us": iso}
 
 
 def workload_of(args):
@@ -646,7 +650,7 @@ def run_ours(args):
     total_bytes = sum_over_ranks(case.bytes_per_step * K, world, device)
     value = total_bytes / (ms / 1e3) / 1e12
     peak, peak_kind = peaks()
-    tc = dispatch.get("variant") == fa.VARIANT_TCGEN05
+    tc = dispatch.get("variant") == fa.VARIANT_TCGEN05 or w.tensor_bound
     us_call = ms / K * 1e3
     traffic = recorded_traffic(name) if not args.batch else None
     clocks = sampler.summary()
@@ -657,7 +661,9 @@ def run_ours(args):
     # boundaries included) -- a lower bound on its own bandwidth.  The isolated
     # per-kernel event times give the kernels' shares, reported beside it (the
     # ncu launch list of the same command gives the same shares).
-    roof = (tensor_roofline(w, case.sl0, ms / K, prof, traffic) if tc
+    roof = (tensor_roofline(w, case.sl0, ms / K, prof, traffic,
+                            "tcgen05 dense kernel (whole call)" if dispatch.get("variant") == fa.VARIANT_TCGEN05
+                            else "split-KV kernel + combine (whole call)") if tc
             else hbm_roofline(case, us_call, prof, peak, peak_kind, traffic))
     cpu = cpu_baseline(w, case.ins0, case.sl0, args.cpu_seconds) if world == 1 else None
 

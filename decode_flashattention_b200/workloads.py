@@ -37,6 +37,7 @@ class Workload:
     seqlen_hi: int = 0
     description: str = ""
     page: int = 0             # "paged": keys per cache block
+    tensor_bound: bool = False  # prefill-shaped: measured against the tensor rate (flops), not HBM
 
     @property
     def g(self) -> int:
@@ -93,7 +94,17 @@ WORKLOADS["gqa_decode_hd256_bf16"] = Workload(
 # Long prefill (the tcgen05 kernel): GQA 4, 4K queries over 4K keys, causal.
 WORKLOADS["gqa_prefill4k_bf16"] = Workload(
     "gqa_prefill4k_bf16", "fwd", "blhd", torch.bfloat16, B=1, Lq=4096, Hq=32, Hkv=8, Lk=4096, Dqk=128, Dv=128,
-    causal=True, seed=1007, description="prefill bf16 B1 Lq4096 Hq32 Hkv8 D128 Lk4096, causal (tcgen05 kernel)")
+    causal=True, seed=1007, description="prefill bf16 B1 Lq4096 Hq32 Hkv8 D128 Lk4096, causal (tcgen05 kernel)",
+    tensor_bound=True)
+
+# Prefill-shaped call with the MLA head dims (192 / 128), GQA 4: the tcgen05
+# split-KV kernel in row blocks of 64 (the dense tcgen05 kernel covers head
+# dims 64 and 128 only).
+WORKLOADS["mla_prefill2k_bf16"] = Workload(
+    "mla_prefill2k_bf16", "fwd", "blhd", torch.bfloat16, B=1, Lq=2048, Hq=32, Hkv=8, Lk=8192, Dqk=192, Dv=128,
+    causal=True, seed=1009, tensor_bound=True,
+    description="prefill-shaped MLA head dims bf16 B1 Lq2048 Hq32 Hkv8 Dqk192 Dv128 Lk8192, causal "
+                "(tcgen05 split-KV kernel, 64-row blocks)")
 
 # The five configurations the metric is quoted on, in order (C1 ... C5).
 CONFIG_IDS = {"C1": "gqa_prefill_fp16", "C2": "decode_hld_fp16", "C3": "specdec_hld_fp16",

@@ -76,7 +76,8 @@ def test_mla_specdec_bf16_reduced():
 
 
 @pytest.mark.parametrize("name,nrows", [("gqa_kvcache_bf16", 96), ("mla_specdec_bf16", 48),
-                                        ("decode_hld_fp16", 32), ("specdec_hld_fp16", 64)])
+                                        ("decode_hld_fp16", 32), ("specdec_hld_fp16", 64),
+                                        ("mla_prefill2k_bf16", 48)])
 def test_full_size_sampled_rows(name, nrows):
     """At the benchmark's full sizes and launch configuration, compare sampled rows."""
     w = wl.WORKLOADS[name]
