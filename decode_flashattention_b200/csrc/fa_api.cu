@@ -380,12 +380,13 @@ fa_status make_plan(Shapes &s, int causal, int num_splits, bool kvcache, int64_t
     // over the keys, so it needs enough CTAs to beat the split-KV kernel, which
     // spreads the keys over every SM (measured with 64-dim heads: 2 CTAs lose at
     // every key length, 32 CTAs win from 128 keys on, 128 CTAs win 4-8x).
-    const bool tc_dims = s.Dqk == s.Dv && (s.Dqk == 128 || s.Dqk == 64);
+    const bool tc_dims = (s.Dqk == s.Dv && (s.Dqk == 128 || s.Dqk == 64)) || (s.Dqk == 192 && s.Dv == 128);
     const int64_t tc_ctas = (int64_t)((s.R + 127) / 128) * s.Hkv * s.B;
     const bool tc_shape = !kvcache && s.R >= 128 && tc_dims && tc_ctas >= 32;
     if (variant == FA_VARIANT_TCGEN05 || (g_force_variant.load() == FA_VARIANT_AUTO && tc_shape)) {
         if (kvcache || !tc_dims)
-            return fail(FA_ERR_UNSUPPORTED, "the tcgen05 variant handles dense fa_fwd calls with head dims 64/64 or 128/128");
+            return fail(FA_ERR_UNSUPPORTED,
+                        "the tcgen05 variant handles dense fa_fwd calls with head dims 64/64, 128/128 or 192/128");
         // Two 128-row tiles per CTA while that still gives every SM a CTA (the
         // tiles' softmax and products overlap); with fewer CTAs than SMs one
         // tile per CTA, in the same MMA-warp pipeline with S double-buffered.

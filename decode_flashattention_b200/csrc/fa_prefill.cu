@@ -44,10 +44,10 @@ constexpr int kBoxQ = kRows * 128;   // one 64-column box of 128 rows (bytes)
 // ---------------------------------------------------------------------------
 // Two query tiles per CTA with 128-key K / V tiles (the kernel also runs
 // with one tile): every QK^T product is M 128 x N 128 x K 16, every PV product
-// M 128 x N D x K 16, and per 128 keys the MMA warp issues 32 products (16
-// for D = 64) with four commits and two waits.  K and V tiles stream
-// separately through a ring of three slots (K(j), V(j), K(j + 1), ...; 128
-// keys x D each).  S is single-buffered per group; per tile j the MMA warp
+// M 128 x N Dv x K 16, and per 128 keys the MMA warp issues 32 products (16
+// for head dim 64, 40 for 192/128) with four commits and two waits.  K and V
+// tiles stream separately through a ring of three slots (two for Dqk = 192;
+// K(j), V(j), K(j + 1), ...; 128 keys each).  S is single-buffered per group; per tile j the MMA warp
 // issues, for group A then group B,
 //   PV_g(j) once the group has written P_g(j) (so it has read S_g(j)),
 //   S_g(j + 1) right behind it (the tensor core runs one thread's products
@@ -61,40 +61,47 @@ constexpr int kBoxQ = kRows * 128;   // one 64-column box of 128 rows (bytes)
 // O is rescaled only on those tiles.
 namespace pf3 {
 constexpr int kKeys = 128;
-constexpr int kSlots = 3;
 constexpr int kBox = kKeys * 128;                // one 64-column box of 128 rows (bytes)
-// full[kSlots], empty[kSlots], s_done[2], p_ready[2], o_done[2], q_ready, drain
-constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
 constexpr int kThreads = 320;                    // an MMA warp, a producer warp, 8 softmax warps
 constexpr int kMmaWarp = 0, kProducerWarp = 1, kFirstSoftmaxWarp = 2;
-constexpr uint32_t kTmemCols = 512;              // S_A, S_B (128 columns each), O_A, O_B (D each)
+constexpr uint32_t kTmemCols = 512;              // S_A, S_B (128 columns each), O_A, O_B (Dv each)
 constexpr float kLazyMax = 8.f;                  // log2 of the largest p before the max moves
-// Shared-memory layout for head dim D (64 or 128): rows of Q, K and V are
-// D / 64 boxes of 64 columns.
-template <int D>
+// Shared-memory layout for head dims (DQK, DV) = (64, 64), (128, 128) or
+// (192, 128): rows of Q and K are DQK / 64 boxes of 64 columns, rows of V
+// DV / 64.  K and V tiles take turns in a ring of equal slots (K(0), V(0),
+// K(1), ...): three, or two for DQK = 192, whose two 48 KB query tiles leave
+// room for two 48 KB slots only.
+template <int DQK, int DV>
 struct Cfg3 {
-    static constexpr int kBoxes = D / 64;
-    static constexpr int kTileQ = kBoxes * kBox;     // one 128-row query tile
-    static constexpr int kSlotBytes = kBoxes * kBox; // a K or V tile: 128 keys x D
+    static constexpr int kBoxesQK = DQK / 64, kBoxesV = DV / 64;
+    static constexpr int kTileQ = kBoxesQK * kBox;   // one 128-row query tile
+    static constexpr int kKBytes = kBoxesQK * kBox;  // a K tile: 128 keys x DQK
+    static constexpr int kVBytes = kBoxesV * kBox;   // a V tile: 128 keys x DV
+    static constexpr int kSlotBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
+    static constexpr int kSlots = DQK > 128 ? 2 : 3;
+    // full[kSlots], empty[kSlots], s_done[2], p_ready[2], o_done[2], q_ready, drain
+    static constexpr int NBAR = 2 * kSlots + 2 + 2 + 2 + 2;
     static constexpr int OFF_Q = 0;                  // Q_A, Q_B
     static constexpr int OFF_KV = OFF_Q + 2 * kTileQ;
     static constexpr int OFF_BAR = OFF_KV + kSlots * kSlotBytes;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base, abort flag, 8 warp maxima
     static constexpr int SMEM = OFF_MISC + 64 + 1024;    // + alignment slack
-    static_assert(D == 64 || D == 128, "head dims 64 and 128");
+    static_assert((DQK == 64 && DV == 64) || (DQK == 128 && DV == 128) || (DQK == 192 && DV == 128),
+                  "head dims 64/64, 128/128 and 192/128");
     static_assert(SMEM <= 232448, "fits the per-CTA shared memory");
-    static_assert(2 * kKeys + 2 * D <= (int)kTmemCols, "S_A, S_B, O_A, O_B fit TMEM");
+    static_assert(2 * kKeys + 2 * DV <= (int)kTmemCols, "S_A, S_B, O_A, O_B fit TMEM");
 };
 }  // namespace pf3
 
 // TILES: query tiles per CTA (2; or 1 when two-tile CTAs would leave SMs idle);
-// D: head dim (64 or 128, Dqk = Dv).
-template <typename T, int TILES, int D>
+// DQK, DV: head dims (64/64, 128/128 or 192/128).
+template <typename T, int TILES, int DQK, int DV>
 __global__ void __launch_bounds__(pf3::kThreads, 1)
     prefill3_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const Params p) {
     using namespace pf;
     using namespace pf3;
-    using L = Cfg3<D>;
+    using L = Cfg3<DQK, DV>;
+    constexpr int kSlots = L::kSlots;
     constexpr int kCtaRows = TILES * kRows;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -187,8 +194,8 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                 if (use > 0 && !mbar_wait(empty_bar(s), (use - 1) & 1, abort_flag, p.status, p.wait_limit_ns)) break;
                 const uint32_t dst = sb + L::OFF_KV + s * L::kSlotBytes;
                 const CUtensorMap *map = (q & 1) ? &tmV : &tmK;
-                mbar_expect_tx(full_bar(s), L::kSlotBytes);
-                for (int c = 0; c < L::kBoxes; ++c)
+                mbar_expect_tx(full_bar(s), (q & 1) ? L::kVBytes : L::kKBytes);
+                for (int c = 0; c < ((q & 1) ? L::kBoxesV : L::kBoxesQK); ++c)
                     tma_load_4d_plain(dst + c * kBox, map, full_bar(s), c * 64, (q >> 1) * kKeys, hkv, b);
                 mbar_arrive(full_bar(s));
                 issued = q + 1;
@@ -205,7 +212,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         // ================================================= MMA issue (one thread)
         if (lane == 0) {
             const uint32_t idesc = instr_desc(bf16, kRows, kKeys, false);   // S: N = 128 keys, K-major K
-            const uint32_t idesc_o = instr_desc(bf16, kRows, D, true);     // PV: N = 128 dims, MN-major V
+            const uint32_t idesc_o = instr_desc(bf16, kRows, DV, true);    // PV: N = DV dims, MN-major V
             // Operand descriptors: a base descriptor plus a constant offset in
             // 16-byte units (every shared address stays below 256 KB, so the sum
             // never carries out of the address field).
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                 const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * L::kSlotBytes) >> 4);
                 const uint64_t dq = dq0 + (uint64_t)((g * L::kTileQ) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < DQK / 16; ++kk) {
                     const uint32_t off = (uint32_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
                     umma(tmem + g * kKeys, dq + off, dk + off, idesc, kk > 0);
                 }
@@ -236,7 +243,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                 auto issue_s1 = [&](int j) {
                     const uint64_t dk = dk0 + (uint64_t)((((2 * j) % kSlots) * L::kSlotBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < DQK / 16; ++kk) {
                         const uint32_t off = (uint32_t)(((kk >> 2) * kBox + (kk & 3) * 32) >> 4);
                         umma(tmem + (j & 1) * kKeys, dq0 + off, dk + off, idesc, kk > 0);
                     }
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk)  // P_g(j): 16 keys = 8 TMEM columns per step
-                        umma_ts(tmem + 2 * kKeys + g * D, tmem + g * kKeys + kk * 8,
+                        umma_ts(tmem + 2 * kKeys + g * DV, tmem + g * kKeys + kk * 8,
                                 dv + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                     // O_g is final after the last tile's PV; before that, the commit
                     // of S_g(j + 1) (issued after PV_g(j), and a commit covers all of
@@ -321,7 +328,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
         {
             const T *qg = reinterpret_cast<const T *>(p.q);
             const T *src = qg + b * p.q_sb + (long long)qi * p.q_sl + (long long)hq * p.q_sh;
-            for (int c = 0; c < D / 8; ++c) {
+            for (int c = 0; c < DQK / 8; ++c) {
                 const uint32_t dst =
                     sb + L::OFF_Q + grp * L::kTileQ + (c >> 3) * kBoxQ + trow * 128 + ((((c & 7) ^ (trow & 7))) << 4);
                 cp_async_16(dst, src + c * 8, row_live ? 16u : 0u);
@@ -332,7 +339,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             if (lane == 0) mbar_arrive(q_bar);
         }
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t t_o = tmem + 2 * kKeys + grp * D + lane_off;
+        const uint32_t t_o = tmem + 2 * kKeys + grp * DV + lane_off;
         float m = -INFINITY, l = 0.f;  // m in base-2 units of the scaled scores
         bool ok = grp < ngroups;  // a group without rows has nothing to do
         for (int j = 0; j < ntiles && ok; ++j) {
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
                     tc_fence_after();
                 }
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h) {
+                for (int h = 0; h < DV / 64; ++h) {
                     uint32_t v0[32], v1[32];
                     tmem_ld32(t_o + h * 64, v0);
                     tmem_ld32(t_o + h * 64 + 32, v1);
@@ -447,7 +454,7 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
             const float inv = l > 0.f ? 1.f / l : 0.f;
             T *og = reinterpret_cast<T *>(p.o) + b * p.o_sb + (long long)qi * p.o_sl + (long long)hq * p.o_sh;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < DV / 32; ++c) {
                 uint32_t v[32];
                 if (ntiles > 0) {
                     tmem_ld32(t_o + c * 32, v);
@@ -478,40 +485,34 @@ __global__ void __launch_bounds__(pf3::kThreads, 1)
     }
 }
 
-template <typename T, int TILES, int D>
+template <typename T, int TILES, int DQK, int DV>
 static void fill3(KernelInfo *out) {
-    out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES, D>);
+    out->fn = reinterpret_cast<const void *>(&prefill3_kernel<T, TILES, DQK, DV>);
     out->threads = pf3::kThreads;
-    out->smem = pf3::Cfg3<D>::SMEM;
+    out->smem = pf3::Cfg3<DQK, DV>::SMEM;
     out->tile_keys = pf3::kKeys;
-    out->stages = pf3::kSlots;
+    out->stages = pf3::Cfg3<DQK, DV>::kSlots;
     out->variant = 3;  // FA_VARIANT_TCGEN05
     out->rows = TILES * pf::kRows;
     out->form = TILES == 2 ? FA_TCGEN05_TWO_TILES : FA_TCGEN05_ONE_TILE_MMA;
 }
 
+template <typename T, int TILES>
+static bool fill3_dims(int dqk, int dv, KernelInfo *out) {
+    if (dqk == 64 && dv == 64) { fill3<T, TILES, 64, 64>(out); return true; }
+    if (dqk == 128 && dv == 128) { fill3<T, TILES, 128, 128>(out); return true; }
+    if (dqk == 192 && dv == 128) { fill3<T, TILES, 192, 128>(out); return true; }
+    return false;
+}
+
 bool get_prefill_kernel(int dtype, int dqk, int dv, int form, KernelInfo *out) {
-    if (dtype < 0 || dtype > 1 || dqk != dv || (dqk != 64 && dqk != 128)) return false;
     const bool h = dtype == 0;
+    if (dtype < 0 || dtype > 1) return false;
     switch (form) {
     case FA_TCGEN05_TWO_TILES:
-        if (dqk == 64) {
-            if (h) fill3<__half, 2, 64>(out);
-            else fill3<__nv_bfloat16, 2, 64>(out);
-        } else {
-            if (h) fill3<__half, 2, 128>(out);
-            else fill3<__nv_bfloat16, 2, 128>(out);
-        }
-        return true;
+        return h ? fill3_dims<__half, 2>(dqk, dv, out) : fill3_dims<__nv_bfloat16, 2>(dqk, dv, out);
     case FA_TCGEN05_ONE_TILE_MMA:
-        if (dqk == 64) {
-            if (h) fill3<__half, 1, 64>(out);
-            else fill3<__nv_bfloat16, 1, 64>(out);
-        } else {
-            if (h) fill3<__half, 1, 128>(out);
-            else fill3<__nv_bfloat16, 1, 128>(out);
-        }
-        return true;
+        return h ? fill3_dims<__half, 1>(dqk, dv, out) : fill3_dims<__nv_bfloat16, 1>(dqk, dv, out);
     default:
         return false;
     }

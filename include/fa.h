@@ -103,7 +103,7 @@ typedef enum fa_variant {
     FA_VARIANT_AUTO = 0,
     FA_VARIANT_MMA = 1,     /* split-KV kernel, mma.sync tensor-core products */
     FA_VARIANT_SCALAR = 2,  /* split-KV kernel, fp32 FMA products (one packed row) */
-    FA_VARIANT_TCGEN05 = 3, /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 64/64 or 128/128) */
+    FA_VARIANT_TCGEN05 = 3, /* dense kernel on tcgen05 + TMEM (>= 128 packed rows, head dims 64/64, 128/128, 192/128) */
     FA_VARIANT_TCGEN05_SPLIT = 4 /* split-KV kernel on tcgen05 + TMEM: row blocks of 16 / 32 / 64 packed rows */
 } fa_variant;
 
@@ -327,7 +327,7 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      TMEM) on blocks of 128 or 256 packed query rows (see
  *                      fa_tcgen05_form), whole key range per CTA, no split
  *                      and no combine; dense fa_fwd calls with head dims
- *                      64/64 or 128/128.
+ *                      64/64, 128/128 or 192/128.
  *   FA_VARIANT_TCGEN05_SPLIT  the split-KV kernel on the 5th-gen tensor
  *                      cores: a unit is a block of up to 64 packed query rows
  *                      (16, 32 or 64: the g * Lq rows of a GQA group with
@@ -337,8 +337,8 @@ FA_API void fa_last_dispatch(fa_dispatch_info *info);
  *                      both accumulated in TMEM; head dims up to 192 / 128
  *                      (every call API: dense, kvcache, paged, varlen, append).
  * The library's own choice: FA_VARIANT_TCGEN05 for dense fa_fwd calls with at
- * least 128 packed rows (g * Lq >= 128) and head dims 64/64 or 128/128
- * (prefill-shaped calls); FA_VARIANT_TCGEN05_SPLIT for more than 8 packed
+ * least 128 packed rows (g * Lq >= 128), head dims 64/64, 128/128 or 192/128
+ * and at least 32 CTAs of rows (prefill-shaped calls); FA_VARIANT_TCGEN05_SPLIT for more than 8 packed
  * rows (g * Lq > 8) with Dqk <= 192 and Dv <= 128 once the K / V re-reads it
  * saves over blocks of 8 rows reach 128 MB (B * Lk * Hkv * (Dqk + Dv) * 2
  * bytes per block, Lk the cache capacity for the kvcache calls: below that its

@@ -150,3 +150,46 @@ def test_head_dim_64_parity(form, case):
     compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 hd64 form {form}")
 
 
+
+
+MLA_CASES = [  # B, Lq, Hq, Hkv, Lk, causal
+    (1, 200, 2, 1, 300, True), (2, 130, 4, 2, 129, False), (1, 300, 2, 1, 100, True), (1, 1000, 4, 4, 1000, True),
+    (1, 64, 8, 2, 700, False),
+]
+
+
+@pytest.mark.parametrize("form", [fa.TCGEN05_TWO_TILES, fa.TCGEN05_ONE_TILE_MMA])
+@pytest.mark.parametrize("case", MLA_CASES, ids=[str(c) for c in MLA_CASES])
+def test_mla_head_dims_parity(form, case):
+    """Head dims 192 / 128 (Q and K rows of three 64-column boxes, V rows of
+    two; K and V take turns in two ring slots)."""
+    B, Lq, Hq, Hkv, Lk, causal = case
+    dt = torch.float16 if (Lq + form) % 2 else torch.bfloat16
+    w = wl.Workload("pf192", "fwd", "blhd", dt, B=B, Lq=Lq, Hq=Hq, Hkv=Hkv, Lk=Lk, Dqk=192, Dv=128, causal=causal,
+                    seed=Lq + Lk + 192 * form)
+    q, k, v, _ = wl.make_inputs(w, DEV)
+    fa.force_variant(fa.VARIANT_TCGEN05)
+    fa.force_tcgen05_form(form)
+    o, lse = fa.fa_fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    d = fa.last_dispatch()
+    assert d["variant"] == fa.VARIANT_TCGEN05 and d["tcgen05_form"] == form
+    ro, rl = oracle_full(q, k, v, causal)
+    compare(o_to_numpy(o), lse_to_numpy(lse), ro, rl, dt, f"tcgen05 192/128 form {form}")
+
+
+def test_mla_head_dims_automatic_choice():
+    """A large prefill-shaped call with head dims 192 / 128 runs on the dense
+    tcgen05 kernel; other non-square dims stay on the split-KV kernels."""
+    q = torch.zeros(1, 2048, 32, 192, dtype=torch.bfloat16, device=DEV)
+    k = torch.zeros(1, 512, 8, 192, dtype=torch.bfloat16, device=DEV)
+    v = torch.zeros(1, 512, 8, 128, dtype=torch.bfloat16, device=DEV)
+    fa.fa_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    d = fa.last_dispatch()
+    assert (d["variant"], d["tcgen05_form"]) == (fa.VARIANT_TCGEN05, fa.TCGEN05_TWO_TILES), d
+    q2 = torch.zeros(1, 2048, 32, 160, dtype=torch.bfloat16, device=DEV)
+    k2 = torch.zeros(1, 512, 8, 160, dtype=torch.bfloat16, device=DEV)
+    fa.fa_fwd(q2, k2, v, causal=True)
+    torch.cuda.synchronize()
+    assert fa.last_dispatch()["variant"] == fa.VARIANT_TCGEN05_SPLIT
