@@ -1,5 +1,7 @@
 """Host-side pieces of bench.py that need no GPU: the kernel-source hash that
-guards the recorded ncu traffic changes with the code, not with comments."""
+guards the recorded ncu traffic changes with the code, not with comments; the
+recorded traffic is used only for the sources it was taken on; the tensor
+roofline of the prefill-shaped workloads counts the call's flops."""
 import os
 import shutil
 
